@@ -1,0 +1,463 @@
+/*
+ * oracle.c -- plain, slow, fp64 CPU reference for masked causal attention.
+ *
+ * TEST INFRASTRUCTURE ONLY. The library's product path never calls, links or
+ * loads this file; only the tests, the smoke check and the benchmark's CPU
+ * baseline leg use it. It shares no code, header or constant with the CUDA
+ * kernels.
+ *
+ * Every function follows the definitions on these pages:
+ *   [CS] "Attention Variants Compared" (cheatsheet): the code of swa_mask and
+ *        strided_mask, the task table (count_nonmasked, tiled_softmax_dot).
+ *   [SW] "Learn: Sparse & Sliding-Window Attention": section 3 "The math"
+ *        (A = softmax(QK^T/sqrt(d_k) + log M) V, log M in {0, -inf}, dense
+ *        causal M_ij = 1[j <= i], band M_ij = 1[i-w < j <= i]); section 4
+ *        (rolling KV window at decode: keep the last w tokens, evict the
+ *        oldest).
+ *   [IG] "Exploring Attention Variants: Flash Attention, Sliding-Window, and
+ *        Sparse Attention Implementation": SWA mask M[i][j] = 0 for
+ *        j in [i-W+1, i] else -inf; strided = logical OR of the window mask
+ *        and the stride mask; attention_row(q, K, V, mask_row) -> (out,
+ *        weights).
+ *   [DA] "Attention Variants -- Sliding Window, Sparse, Differential": the
+ *        problem statement (two attention maps from separate Q/K
+ *        projections, one subtracted from the other).
+ *
+ * Readings taken where the pages are silent (each listed in the design
+ * notes): the window holds W keys (i-W+1 .. i); stride keys are the absolute
+ * multiples of S from 0 (range(0, i+1, stride)); the differential output is
+ * sum_j (w1_ij - lambda_h * w2_ij) v_j with both maps under the same mask;
+ * query head h reads KV head h / (Hq/Hkv); a decode step writes the new
+ * token into slot pos % W and then attends.
+ *
+ * Inputs are float32 arrays holding bf16 values exactly; every product and
+ * sum is taken in double.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORC_MASK_SWA 0
+#define ORC_MASK_STRIDED 1
+#define ORC_MASK_CAUSAL 2
+
+/* ---------------------------------------------------------------------- */
+/* Masks, one row at a time, in the pages' additive form: 0.0 = attends,  */
+/* -inf = masked.                                                          */
+/* ---------------------------------------------------------------------- */
+
+/* [CS] swa_mask / [IG]: row i starts all -inf, then j = lo .. i set to 0.0
+ * with lo = max(0, i - window + 1). window >= n gives full causal. */
+void orc_swa_mask_row(int n, int window, int i, double* row) {
+  for (int j = 0; j < n; ++j) row[j] = -INFINITY;
+  int lo = i - window + 1;
+  if (lo < 0) lo = 0;
+  for (int j = lo; j <= i; ++j) row[j] = 0.0;
+}
+
+/* [CS] strided_mask: the local window first, then every stride-th key from 0
+ * up to and including i is set to 0.0; [IG]: the union (logical OR). */
+void orc_strided_mask_row(int n, int window, int stride, int i, double* row) {
+  orc_swa_mask_row(n, window, i, row);
+  for (int j = 0; j < i + 1; j += stride) row[j] = 0.0;
+}
+
+/* [SW] section 3: dense causal attention is M_ij = 1[j <= i]. Written on its
+ * own (not as swa_mask with a large window) so that the two can be compared. */
+void orc_causal_mask_row(int n, int i, double* row) {
+  for (int j = 0; j < n; ++j) row[j] = (j <= i) ? 0.0 : -INFINITY;
+}
+
+void orc_mask_row(int kind, int n, int window, int stride, int i, double* row) {
+  if (kind == ORC_MASK_SWA) orc_swa_mask_row(n, window, i, row);
+  else if (kind == ORC_MASK_STRIDED) orc_strided_mask_row(n, window, stride, i, row);
+  else orc_causal_mask_row(n, i, row);
+}
+
+/* The full n x n matrix, row-major, built row by row. */
+void orc_mask(int kind, int n, int window, int stride, double* M) {
+  for (int i = 0; i < n; ++i) orc_mask_row(kind, n, window, stride, i, M + (int64_t)i * n);
+}
+
+/* [CS] count_nonmasked(M): the number of attended cells, ||M||_0 in [SW]. */
+int64_t orc_count_nonmasked(const double* M, int64_t count) {
+  int64_t c = 0;
+  for (int64_t t = 0; t < count; ++t) c += (M[t] == 0.0);
+  return c;
+}
+
+/* ---------------------------------------------------------------------- */
+/* One attention row.                                                      */
+/* ---------------------------------------------------------------------- */
+
+/* [IG] attention_row / [SW] section 3: s_j = scale * q.k_j + M_ij,
+ * w = softmax(s) (max subtracted), out = sum_j w_j v_j. K is n x dk, V is
+ * n x dv, both row-major float. weights may be NULL. A masked entry's score
+ * is -inf whatever q.k_j is, so its dot product is not formed. */
+void orc_attention_row(const double* q, const float* K, const float* V, const double* mask_row,
+                       int n, int dk, int dv, double scale, double* out, double* weights,
+                       double* scratch_s, double* lse) {
+  double mx = -INFINITY;
+  for (int j = 0; j < n; ++j) {
+    double s = -INFINITY;
+    if (mask_row[j] == 0.0) {
+      double dot = 0.0;
+      const float* kj = K + (int64_t)j * dk;
+      for (int c = 0; c < dk; ++c) dot += q[c] * (double)kj[c];
+      s = scale * dot + mask_row[j];
+    }
+    scratch_s[j] = s;
+    if (s > mx) mx = s;
+  }
+  double denom = 0.0;
+  for (int j = 0; j < n; ++j) {
+    double e = (scratch_s[j] == -INFINITY) ? 0.0 : exp(scratch_s[j] - mx);
+    scratch_s[j] = e;
+    denom += e;
+  }
+  for (int c = 0; c < dv; ++c) out[c] = 0.0;
+  for (int j = 0; j < n; ++j) {
+    double w = scratch_s[j] / denom;
+    if (weights) weights[j] = w;
+    if (w == 0.0) continue;
+    const float* vj = V + (int64_t)j * dv;
+    for (int c = 0; c < dv; ++c) out[c] += w * (double)vj[c];
+  }
+  if (lse) *lse = mx + log(denom);
+}
+
+/* Stand-alone form on double inputs (used by the tests on tiny cases). */
+void orc_attention_row_f64(const double* q, const double* K, const double* V, const double* mask_row,
+                           int n, int dk, int dv, double scale, double* out, double* weights) {
+  double* s = (double*)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1));
+  double mx = -INFINITY;
+  for (int j = 0; j < n; ++j) {
+    double v = -INFINITY;
+    if (mask_row[j] == 0.0) {
+      double dot = 0.0;
+      for (int c = 0; c < dk; ++c) dot += q[c] * K[(int64_t)j * dk + c];
+      v = scale * dot + mask_row[j];
+    }
+    s[j] = v;
+    if (v > mx) mx = v;
+  }
+  double denom = 0.0;
+  for (int j = 0; j < n; ++j) {
+    s[j] = (s[j] == -INFINITY) ? 0.0 : exp(s[j] - mx);
+    denom += s[j];
+  }
+  for (int c = 0; c < dv; ++c) out[c] = 0.0;
+  for (int j = 0; j < n; ++j) {
+    double w = s[j] / denom;
+    if (weights) weights[j] = w;
+    for (int c = 0; c < dv; ++c) out[c] += w * V[(int64_t)j * dv + c];
+  }
+  free(s);
+}
+
+/* [CS] tiled_softmax_dot(q, Ks, Vs, tile): the flash-style softmax. Keys are
+ * taken `tile` at a time; a running max m, running sum l and a running
+ * output are rescaled by exp(m_old - m_new) whenever the max grows. Only
+ * used to check that the tiled form equals the full softmax. */
+void orc_tiled_softmax_dot(const double* q, const double* K, const double* V, const double* mask_row,
+                           int n, int dk, int dv, double scale, int tile, double* out) {
+  double m = -INFINITY, l = 0.0;
+  for (int c = 0; c < dv; ++c) out[c] = 0.0;
+  for (int t0 = 0; t0 < n; t0 += tile) {
+    int t1 = t0 + tile < n ? t0 + tile : n;
+    double tm = -INFINITY;
+    for (int j = t0; j < t1; ++j) {
+      if (mask_row[j] != 0.0) continue;
+      double dot = 0.0;
+      for (int c = 0; c < dk; ++c) dot += q[c] * K[(int64_t)j * dk + c];
+      double s = scale * dot;
+      if (s > tm) tm = s;
+    }
+    if (tm == -INFINITY) continue; /* nothing attended in this tile */
+    double m_new = m > tm ? m : tm;
+    double alpha = (m == -INFINITY) ? 0.0 : exp(m - m_new);
+    l *= alpha;
+    for (int c = 0; c < dv; ++c) out[c] *= alpha;
+    for (int j = t0; j < t1; ++j) {
+      if (mask_row[j] != 0.0) continue;
+      double dot = 0.0;
+      for (int c = 0; c < dk; ++c) dot += q[c] * K[(int64_t)j * dk + c];
+      double p = exp(scale * dot - m_new);
+      l += p;
+      for (int c = 0; c < dv; ++c) out[c] += p * V[(int64_t)j * dv + c];
+    }
+    m = m_new;
+  }
+  for (int c = 0; c < dv; ++c) out[c] /= l;
+}
+
+/* ---------------------------------------------------------------------- */
+/* Whole tensors: [B, H, N, d] row-major, query head h reads KV head       */
+/* h / (Hq / Hkv). Rows are split over threads.                            */
+/* ---------------------------------------------------------------------- */
+
+typedef struct {
+  int kind, B, Hq, Hkv, N, dk, dv, W, S;
+  double scale;
+  const float *q, *k, *v;        /* plain attention */
+  const float *q1, *k1, *q2, *k2; /* differential */
+  const float* lambda;
+  const int64_t* rows; /* flat row ids (b*Hq + h)*N + i, or NULL for all */
+  int64_t nrows;
+  double* out; /* nrows x dv */
+  double* lse; /* nrows, may be NULL */
+  int nthreads, tid;
+} orc_job_t;
+
+static void row_coords(const orc_job_t* J, int64_t r, int* b, int* hq, int* i) {
+  int64_t flat = J->rows ? J->rows[r] : r;
+  *i = (int)(flat % J->N);
+  int64_t bh = flat / J->N;
+  *hq = (int)(bh % J->Hq);
+  *b = (int)(bh / J->Hq);
+}
+
+static void* attn_worker(void* arg) {
+  orc_job_t* J = (orc_job_t*)arg;
+  int G = J->Hq / J->Hkv;
+  double* mrow = (double*)malloc(sizeof(double) * (size_t)J->N);
+  double* s = (double*)malloc(sizeof(double) * (size_t)J->N);
+  double* qd = (double*)malloc(sizeof(double) * (size_t)J->dk);
+  for (int64_t r = J->tid; r < J->nrows; r += J->nthreads) {
+    int b, hq, i;
+    row_coords(J, r, &b, &hq, &i);
+    int hk = hq / G;
+    const float* qrow = J->q + (((int64_t)b * J->Hq + hq) * J->N + i) * J->dk;
+    for (int c = 0; c < J->dk; ++c) qd[c] = (double)qrow[c];
+    const float* K = J->k + ((int64_t)b * J->Hkv + hk) * J->N * (int64_t)J->dk;
+    const float* V = J->v + ((int64_t)b * J->Hkv + hk) * J->N * (int64_t)J->dv;
+    orc_mask_row(J->kind, J->N, J->W, J->S, i, mrow);
+    orc_attention_row(qd, K, V, mrow, J->N, J->dk, J->dv, J->scale, J->out + r * J->dv, NULL, s,
+                      J->lse ? J->lse + r : NULL);
+  }
+  free(mrow);
+  free(s);
+  free(qd);
+  return NULL;
+}
+
+/* [DA] problem statement: two maps from separate Q/K, one subtracted from
+ * the other, over the shared V: out_i = sum_j (w1_ij - lambda_h w2_ij) v_j. */
+static void* diff_worker(void* arg) {
+  orc_job_t* J = (orc_job_t*)arg;
+  int G = J->Hq / J->Hkv;
+  int N = J->N;
+  double* mrow = (double*)malloc(sizeof(double) * (size_t)N);
+  double* s = (double*)malloc(sizeof(double) * (size_t)N);
+  double* w1 = (double*)malloc(sizeof(double) * (size_t)N);
+  double* w2 = (double*)malloc(sizeof(double) * (size_t)N);
+  double* o = (double*)malloc(sizeof(double) * (size_t)J->dv);
+  double* qd = (double*)malloc(sizeof(double) * (size_t)J->dk);
+  for (int64_t r = J->tid; r < J->nrows; r += J->nthreads) {
+    int b, hq, i;
+    row_coords(J, r, &b, &hq, &i);
+    int hk = hq / G;
+    int64_t qoff = (((int64_t)b * J->Hq + hq) * N + i) * J->dk;
+    int64_t koff = ((int64_t)b * J->Hkv + hk) * N * (int64_t)J->dk;
+    const float* V = J->v + ((int64_t)b * J->Hkv + hk) * N * (int64_t)J->dv;
+    orc_mask_row(J->kind, N, J->W, J->S, i, mrow);
+    for (int c = 0; c < J->dk; ++c) qd[c] = (double)J->q1[qoff + c];
+    orc_attention_row(qd, J->k1 + koff, V, mrow, N, J->dk, J->dv, J->scale, o, w1, s, NULL);
+    for (int c = 0; c < J->dk; ++c) qd[c] = (double)J->q2[qoff + c];
+    orc_attention_row(qd, J->k2 + koff, V, mrow, N, J->dk, J->dv, J->scale, o, w2, s, NULL);
+    double lam = (double)J->lambda[hq];
+    double* out = J->out + r * J->dv;
+    for (int c = 0; c < J->dv; ++c) out[c] = 0.0;
+    for (int j = 0; j < N; ++j) {
+      double w = w1[j] - lam * w2[j];
+      if (w == 0.0) continue;
+      const float* vj = V + (int64_t)j * J->dv;
+      for (int c = 0; c < J->dv; ++c) out[c] += w * (double)vj[c];
+    }
+  }
+  free(mrow);
+  free(s);
+  free(w1);
+  free(w2);
+  free(o);
+  free(qd);
+  return NULL;
+}
+
+static int run_threads(orc_job_t* proto, void* (*fn)(void*)) {
+  int nt = proto->nthreads < 1 ? 1 : proto->nthreads;
+  if (nt > 256) nt = 256;
+  pthread_t th[256];
+  orc_job_t jobs[256];
+  for (int t = 0; t < nt; ++t) {
+    jobs[t] = *proto;
+    jobs[t].nthreads = nt;
+    jobs[t].tid = t;
+  }
+  int started = 0;
+  for (int t = 1; t < nt; ++t) {
+    if (pthread_create(&th[t], NULL, fn, &jobs[t]) != 0) break;
+    started = t;
+  }
+  fn(&jobs[0]);
+  for (int t = 1; t <= started; ++t) pthread_join(th[t], NULL);
+  if (started != nt - 1) { /* a thread failed to start: do its share here */
+    for (int t = started + 1; t < nt; ++t) fn(&jobs[t]);
+  }
+  return 0;
+}
+
+/* Masked attention (kind = swa / strided / causal) over [B,H,N,d] tensors.
+ * rows: flat row ids to compute, or NULL with nrows = B*Hq*N for all rows.
+ * out: nrows x dv doubles; lse: nrows natural-log sums (may be NULL). */
+int orc_attention(int kind, const float* q, const float* k, const float* v, int B, int Hq, int Hkv,
+                  int N, int dk, int dv, int W, int S, double scale, const int64_t* rows,
+                  int64_t nrows, double* out, double* lse, int nthreads) {
+  if (Hkv <= 0 || Hq % Hkv != 0 || N <= 0) return 1;
+  orc_job_t J;
+  memset(&J, 0, sizeof(J));
+  J.kind = kind; J.B = B; J.Hq = Hq; J.Hkv = Hkv; J.N = N; J.dk = dk; J.dv = dv;
+  J.W = W; J.S = S; J.scale = scale; J.q = q; J.k = k; J.v = v;
+  J.rows = rows; J.nrows = nrows; J.out = out; J.lse = lse; J.nthreads = nthreads;
+  return run_threads(&J, attn_worker);
+}
+
+int orc_diff_attention(int kind, const float* q1, const float* k1, const float* q2, const float* k2,
+                       const float* v, const float* lambda, int B, int Hq, int Hkv, int N, int dk,
+                       int dv, int W, int S, double scale, const int64_t* rows, int64_t nrows,
+                       double* out, int nthreads) {
+  if (Hkv <= 0 || Hq % Hkv != 0 || N <= 0) return 1;
+  orc_job_t J;
+  memset(&J, 0, sizeof(J));
+  J.kind = kind; J.B = B; J.Hq = Hq; J.Hkv = Hkv; J.N = N; J.dk = dk; J.dv = dv;
+  J.W = W; J.S = S; J.scale = scale; J.q1 = q1; J.k1 = k1; J.q2 = q2; J.k2 = k2; J.v = v;
+  J.lambda = lambda; J.rows = rows; J.nrows = nrows; J.out = out; J.nthreads = nthreads;
+  return run_threads(&J, diff_worker);
+}
+
+/* ---------------------------------------------------------------------- */
+/* Decode over a rolling W-slot cache ([SW] section 4: keep only the most  */
+/* recent w tokens' K/V, evict the oldest).                                */
+/* ---------------------------------------------------------------------- */
+
+/* T steps. q: [T,B,Hq,d]; k_new, v_new: [T,B,Hkv,d]; caches: [B,Hkv,W,d]
+ * (updated in place); pos: [T,B] absolute position of each step's token.
+ * Each step first stores the new token in slot pos % W (overwriting the
+ * token at pos - W, the oldest), then attends over the positions still in
+ * the window, max(0, pos-W+1) .. pos, each read from its slot p % W. */
+int orc_decode(const float* q, const float* k_new, const float* v_new, float* k_cache,
+               float* v_cache, const int32_t* pos, int T, int B, int Hq, int Hkv, int d, int W,
+               double scale, double* out) {
+  if (Hkv <= 0 || Hq % Hkv != 0 || W <= 0) return 1;
+  int G = Hq / Hkv;
+  double* s = (double*)malloc(sizeof(double) * (size_t)W);
+  double* qd = (double*)malloc(sizeof(double) * (size_t)d);
+  for (int t = 0; t < T; ++t) {
+    for (int b = 0; b < B; ++b) {
+      int p = pos[(int64_t)t * B + b];
+      int slot = p % W;
+      for (int hk = 0; hk < Hkv; ++hk) {
+        int64_t src = (((int64_t)t * B + b) * Hkv + hk) * d;
+        int64_t dst = (((int64_t)b * Hkv + hk) * W + slot) * d;
+        memcpy(k_cache + dst, k_new + src, sizeof(float) * (size_t)d);
+        memcpy(v_cache + dst, v_new + src, sizeof(float) * (size_t)d);
+      }
+      int first = p - W + 1;
+      if (first < 0) first = 0;
+      int cnt = p - first + 1;
+      for (int hq = 0; hq < Hq; ++hq) {
+        int hk = hq / G;
+        const float* qrow = q + (((int64_t)t * B + b) * Hq + hq) * d;
+        for (int c = 0; c < d; ++c) qd[c] = (double)qrow[c];
+        const float* Kc = k_cache + ((int64_t)b * Hkv + hk) * (int64_t)W * d;
+        const float* Vc = v_cache + ((int64_t)b * Hkv + hk) * (int64_t)W * d;
+        double mx = -INFINITY;
+        for (int u = 0; u < cnt; ++u) {
+          int sl = (first + u) % W;
+          double dot = 0.0;
+          for (int c = 0; c < d; ++c) dot += qd[c] * (double)Kc[(int64_t)sl * d + c];
+          s[u] = scale * dot;
+          if (s[u] > mx) mx = s[u];
+        }
+        double denom = 0.0;
+        for (int u = 0; u < cnt; ++u) {
+          s[u] = exp(s[u] - mx);
+          denom += s[u];
+        }
+        double* o = out + (((int64_t)t * B + b) * Hq + hq) * d;
+        for (int c = 0; c < d; ++c) o[c] = 0.0;
+        for (int u = 0; u < cnt; ++u) {
+          int sl = (first + u) % W;
+          double w = s[u] / denom;
+          for (int c = 0; c < d; ++c) o[c] += w * (double)Vc[(int64_t)sl * d + c];
+        }
+      }
+    }
+  }
+  free(s);
+  free(qd);
+  return 0;
+}
+
+/* ---------------------------------------------------------------------- */
+/* Which key tiles a query tile touches, read off the explicit mask.       */
+/* ---------------------------------------------------------------------- */
+
+/* For query tile qt (rows qt*Bq .. qt*Bq+Bq-1, clipped to N) scan every cell
+ * of the explicit mask row. An attended cell that the window mask also
+ * attends marks key tile j / Bk; an attended cell outside the window (only
+ * the strided mask has those; they are multiples of S) marks stride tile
+ * (j / S) / Bk. cells += every attended cell. Writes the marked tiles into
+ * tiles[] as stride tiles first (0x40000000 | ct, ascending) then window
+ * tiles (kt, ascending); returns their number, or -1 if cap is too small, or
+ * -2 if an outside-window cell is not a multiple of S. */
+int64_t orc_schedule_qtile(int kind, int N, int W, int S, int Bq, int Bk, int qt, int32_t* tiles,
+                           int64_t cap, int64_t* cells) {
+  int nkt = (N + Bk - 1) / Bk;
+  int nst = (S > 0) ? ((N + S - 1) / S + Bk - 1) / Bk : 0;
+  uint8_t* band = (uint8_t*)calloc((size_t)nkt + 1, 1);
+  uint8_t* strd = (uint8_t*)calloc((size_t)nst + 1, 1);
+  double* row = (double*)malloc(sizeof(double) * (size_t)N);
+  double* wrow = (double*)malloc(sizeof(double) * (size_t)N);
+  int64_t c = 0;
+  int bad = 0;
+  int r0 = qt * Bq, r1 = qt * Bq + Bq;
+  if (r1 > N) r1 = N;
+  for (int i = r0; i < r1; ++i) {
+    orc_mask_row(kind, N, W, S, i, row);
+    /* the window part of the same row: for the strided mask the band is the
+     * swa_mask row (its first loop); for swa/causal the whole row is band */
+    if (kind == ORC_MASK_STRIDED) orc_swa_mask_row(N, W, i, wrow);
+    for (int j = 0; j < N; ++j) {
+      if (row[j] != 0.0) continue;
+      ++c;
+      int in_band = (kind == ORC_MASK_STRIDED) ? (wrow[j] == 0.0) : 1;
+      if (in_band) {
+        band[j / Bk] = 1;
+      } else {
+        if (j % S != 0) bad = 1;
+        strd[(j / S) / Bk] = 1;
+      }
+    }
+  }
+  int64_t n = 0;
+  for (int t = 0; t < nst; ++t)
+    if (strd[t]) {
+      if (n < cap) tiles[n] = 0x40000000 | t;
+      ++n;
+    }
+  for (int t = 0; t < nkt; ++t)
+    if (band[t]) {
+      if (n < cap) tiles[n] = t;
+      ++n;
+    }
+  free(band);
+  free(strd);
+  free(row);
+  free(wrow);
+  if (cells) *cells = c;
+  if (bad) return -2;
+  return n > cap ? -1 : n;
+}

@@ -1,0 +1,378 @@
+"""Pins for the fp64 oracle: what the pages print or fix, closed forms,
+textbook special cases (torch's fp64 scaled_dot_product_attention), and
+brute force on tiny inputs. Each test would fail on a plausible slip in the
+oracle: a dropped term, a wrong sign, an off-by-one window, a swapped
+operand, a wrong GQA map."""
+import math
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+from conftest import read_grid, read_numbers
+from differential_attention_swa_b200.inputs import attn_inputs, diff_inputs, randn_bf16
+
+
+def grid_of(M):
+    return ["".join("x" if v == 0.0 else "." for v in row) for row in M]
+
+
+# ------------------------------------------------------------------ masks --
+
+def test_swa_mask_8_4_matches_hand_derived_grid(orc):
+    M = orc.swa_mask(8, 4)
+    assert grid_of(M) == read_grid("swa_mask_n8_w4.txt")
+    assert set(np.unique(M).tolist()) == {0.0, -math.inf}
+    assert orc.count_nonmasked(M) == 26
+
+
+def test_strided_mask_8_2_3_matches_hand_derived_grid(orc):
+    M = orc.strided_mask(8, 2, 3)
+    assert grid_of(M) == read_grid("strided_mask_n8_w2_s3.txt")
+    assert orc.count_nonmasked(M) == 24
+
+
+def test_causal_8_count(orc):
+    assert orc.count_nonmasked(orc.causal_mask(8)) == 36
+
+
+@pytest.mark.parametrize("n", [1, 2, 7, 33])
+def test_window_at_least_n_is_full_causal(orc, n):
+    C = orc.causal_mask(n)
+    for W in (n, n + 1, 10 * n):
+        assert np.array_equal(orc.swa_mask(n, W), C)
+        for S in (1, 2, 5, n + 3):
+            assert np.array_equal(orc.strided_mask(n, W, S), C)
+
+
+def test_brute_force_masks_all_small(orc):
+    """The cheatsheet's loops against the lesson's predicate form
+    M_ij = 1[i - w < j <= i] (and its OR with j % S == 0, j <= i), for every
+    n <= 24, every window and every stride."""
+    for n in range(1, 25):
+        ii, jj = np.meshgrid(np.arange(n), np.arange(n), indexing="ij")
+        for W in range(1, n + 2):
+            band = (ii - W < jj) & (jj <= ii)
+            assert np.array_equal(orc.swa_mask(n, W) == 0.0, band), (n, W)
+            for S in range(1, n + 2):
+                want = band | ((jj % S == 0) & (jj <= ii))
+                assert np.array_equal(orc.strided_mask(n, W, S) == 0.0, want), (n, W, S)
+
+
+def band_closed(N, W):
+    return N * (N + 1) // 2 if W >= N else N * W - W * (W - 1) // 2
+
+
+def strided_closed(N, W, S):
+    # sum over rows of min(i+1, W) window keys plus the multiples of S below lo_i
+    i = np.arange(N, dtype=np.int64)
+    lo = np.maximum(0, i - W + 1)
+    return int(np.minimum(i + 1, W).sum() + ((lo + S - 1) // S).sum())
+
+
+@pytest.mark.parametrize("N,W,S,want", [
+    (256, 64, 0, 14368), (256, 16, 8, 7696), (8192, 4096, 0, 25167872),
+    (16384, 128, 128, 3129408), (131072, 1024, 0, 133693952), (4096, 4096, 0, 8390656)])
+def test_closed_form_counts(N, W, S, want):
+    got = strided_closed(N, W, S) if S else band_closed(N, W)
+    assert got == want
+
+
+@pytest.mark.parametrize("N,W,S", [(256, 64, 0), (256, 16, 8), (300, 17, 5), (8192, 4096, 0),
+                                   (1000, 1, 3), (513, 600, 7)])
+def test_explicit_count_matches_closed_form(orc, N, W, S):
+    if N <= 1024:
+        M = orc.strided_mask(N, W, S) if S else orc.swa_mask(N, W)
+        got = orc.count_nonmasked(M)
+    else:  # row by row: the full matrix is 8 bytes per cell
+        kind = "strided" if S else "swa"
+        got = sum(orc.count_nonmasked(orc.mask_row(kind, N, i, W, S)) for i in range(N))
+    want = strided_closed(N, W, S) if S else band_closed(N, W)
+    assert got == want
+
+
+def test_stride_at_least_n_adds_only_key_zero(orc):
+    n, W = 40, 6
+    for S in (n, n + 1, 100):
+        want = orc.swa_mask(n, W).copy()
+        want[:, 0] = 0.0
+        assert np.array_equal(orc.strided_mask(n, W, S), want)
+
+
+# ----------------------------------------------------- softmax & rows ------
+
+def test_rows_sum_to_one_and_masked_weights_are_zero(orc):
+    rng = np.random.default_rng(0)
+    n, d = 37, 8
+    K, V = rng.normal(size=(n, d)), rng.normal(size=(n, d))
+    M = orc.strided_mask(n, 5, 4)
+    for i in range(n):
+        out, w = orc.attention_row(rng.normal(size=d), K, V, M[i], 1 / math.sqrt(d))
+        assert abs(w.sum() - 1.0) < 1e-12
+        assert np.all(w[M[i] != 0.0] == 0.0)
+        assert np.all(w[M[i] == 0.0] > 0.0)
+        assert np.allclose(out, w @ V, rtol=0, atol=1e-12)
+
+
+def test_attention_row_matches_page_example_shape(orc):
+    """The instagit snippet: n = 8, d = 8, rng seed 0, SWA window 4, the last
+    token's row. Checked against a softmax written out with numpy."""
+    rng = np.random.default_rng(0)
+    n, d = 8, 8
+    q = rng.normal(size=d)
+    K = rng.normal(size=(n, d))
+    V = rng.normal(size=(n, d))
+    row = orc.swa_mask(n, 4)[7]
+    out, w = orc.attention_row(q, K, V, row, 1.0 / math.sqrt(d))
+    s = K[4:8] @ q / math.sqrt(d)
+    e = np.exp(s - s.max())
+    want_w = np.zeros(n)
+    want_w[4:8] = e / e.sum()
+    assert np.allclose(w, want_w, rtol=0, atol=1e-14)
+    assert np.allclose(out, want_w @ V, rtol=0, atol=1e-13)
+
+
+@pytest.mark.parametrize("tile", [1, 3, 4, 37])
+def test_tiled_softmax_equals_full_softmax(orc, tile):
+    rng = np.random.default_rng(1)
+    n, dk, dv = 37, 8, 5
+    K, V = rng.normal(size=(n, dk)) * 3, rng.normal(size=(n, dv))
+    M = orc.strided_mask(n, 6, 5)
+    for i in range(n):
+        q = rng.normal(size=dk)
+        full, _ = orc.attention_row(q, K, V, M[i], 0.7)
+        tiled = orc.tiled_softmax_dot(q, K, V, M[i], 0.7, tile)
+        assert np.allclose(tiled, full, rtol=1e-12, atol=1e-12)
+
+
+def test_row_zero_is_v0_and_window_one_is_identity(orc):
+    q, k, v = attn_inputs(1, 2, 2, 50, 16, seed=3)
+    out = orc.attention("swa", q, k, v, W=8)
+    assert np.array_equal(out[0, :, 0, :], v[0, :, 0, :].float().numpy().astype(np.float64))
+    out1 = orc.attention("swa", q, k, v, W=1)
+    assert np.array_equal(out1, v.float().numpy().astype(np.float64))
+    out1s = orc.attention("strided", q, k, v, W=1, S=1000)
+    # window 1 plus key 0: row i mixes only v_0 and v_i
+    assert np.array_equal(out1s[:, :, 0], out1[:, :, 0])
+
+
+# ---------------------------------------------- textbook library routine ---
+
+def sdpa_ref(q, k, v, allowed, scale):
+    """torch's fp64 scaled_dot_product_attention with a boolean mask,
+    KV heads repeated to the query heads (consecutive grouping)."""
+    G = q.shape[1] // k.shape[1]
+    q64, k64, v64 = (t.double() for t in (q, k, v))
+    k64 = k64.repeat_interleave(G, dim=1)
+    v64 = v64.repeat_interleave(G, dim=1)
+    return F.scaled_dot_product_attention(q64, k64, v64, attn_mask=torch.from_numpy(allowed),
+                                          scale=scale).numpy()
+
+
+@pytest.mark.parametrize("kind,B,Hq,Hkv,N,d,dv,W,S", [
+    ("swa", 1, 2, 2, 64, 16, 16, 9, 0),
+    ("swa", 2, 4, 2, 130, 32, 32, 40, 0),
+    ("swa", 1, 6, 2, 77, 16, 24, 1000, 0),
+    ("strided", 1, 2, 1, 150, 16, 16, 7, 11),
+    ("strided", 2, 4, 4, 97, 8, 8, 3, 1),
+    ("causal", 1, 3, 1, 55, 16, 16, 0, 0),
+])
+def test_attention_matches_torch_sdpa_fp64(orc, kind, B, Hq, Hkv, N, d, dv, W, S):
+    q, k, v = attn_inputs(B, Hq, Hkv, N, d, dv, seed=11)
+    scale = 1.0 / math.sqrt(d)
+    out, lse = orc.attention(kind, q, k, v, W=W, S=S, scale=scale, with_lse=True)
+    ii, jj = np.meshgrid(np.arange(N), np.arange(N), indexing="ij")
+    if kind == "causal":
+        allowed = jj <= ii
+    else:
+        allowed = (ii - W < jj) & (jj <= ii)
+        if kind == "strided":
+            allowed |= (jj % S == 0) & (jj <= ii)
+    ref = sdpa_ref(q, k, v, allowed, scale)
+    assert np.abs(out - ref).max() < 1e-12
+    # natural-log sum of exp over the attended scores
+    G = Hq // Hkv
+    s = np.einsum("bhid,bhjd->bhij", q.double().numpy(),
+                  k.double().repeat_interleave(G, dim=1).numpy()) * scale
+    s = np.where(allowed, s, -np.inf)
+    mx = s.max(-1, keepdims=True)
+    want_lse = (mx + np.log(np.exp(s - mx).sum(-1, keepdims=True)))[..., 0]
+    assert np.abs(lse - want_lse).max() < 1e-12
+
+
+def test_attention_row_subset_matches_full(orc):
+    q, k, v = attn_inputs(2, 4, 2, 90, 16, seed=5)
+    full = orc.attention("strided", q, k, v, W=10, S=7)
+    rows = np.array([0, 5, 89, 90, 179, 4 * 90 + 33, 8 * 90 - 1])
+    part = orc.attention("strided", q, k, v, W=10, S=7, rows=rows)
+    assert np.array_equal(part, full.reshape(-1, 16)[rows])
+
+
+# ------------------------------------------------------------ differential --
+
+def test_diff_lambda_zero_is_plain_attention(orc):
+    q1, k1, q2, k2, v = diff_inputs(1, 2, 2, 70, 16, 24, seed=2)
+    lam = np.zeros(2, dtype=np.float32)
+    out = orc.diff_attention(q1, k1, q2, k2, v, lam)
+    plain = orc.attention("causal", q1, k1, v, scale=1 / 4)
+    assert np.abs(out - plain).max() < 1e-13
+
+
+def test_diff_same_maps_is_one_minus_lambda(orc):
+    q1, k1, _, _, v = diff_inputs(1, 2, 2, 70, 16, 24, seed=2)
+    lam = np.array([0.8, 0.3], dtype=np.float32)
+    out = orc.diff_attention(q1, k1, q1, k1, v, lam)
+    plain = orc.attention("causal", q1, k1, v, scale=1 / 4)
+    want = plain * (1.0 - lam.astype(np.float64))[None, :, None, None]
+    assert np.abs(out - want).max() < 1e-12
+
+
+@pytest.mark.parametrize("W", [None, 13])
+def test_diff_matches_sdpa_difference(orc, W):
+    B, Hq, Hkv, N, dqk, dv = 1, 4, 2, 66, 16, 32
+    q1, k1, q2, k2, v = diff_inputs(B, Hq, Hkv, N, dqk, dv, seed=9)
+    lam = np.array([0.8, 0.5, 0.1, 1.2], dtype=np.float32)
+    out = orc.diff_attention(q1, k1, q2, k2, v, lam, W=W, scale=0.125)
+    ii, jj = np.meshgrid(np.arange(N), np.arange(N), indexing="ij")
+    Wv = N if W is None else W
+    allowed = (ii - Wv < jj) & (jj <= ii)
+    a1 = sdpa_ref(q1, k1, v, allowed, 0.125)
+    a2 = sdpa_ref(q2, k2, v, allowed, 0.125)
+    want = a1 - lam.astype(np.float64)[None, :, None, None] * a2
+    assert np.abs(out - want).max() < 1e-12
+
+
+# ----------------------------------------------------------------- decode --
+
+@pytest.mark.parametrize("W,pos0,T", [(8, 3, 12), (8, 20, 9), (5, 0, 7), (16, 16, 3)])
+def test_decode_equals_window_softmax_over_history(orc, W, pos0, T):
+    """Step t attends exactly the W most recent positions of the history,
+    whatever slot order the rolling buffer holds them in, across wrap-around
+    and before the buffer first fills (pos < W - 1)."""
+    B, Hq, Hkv, d = 2, 4, 2, 16
+    L = pos0 + T
+    Kh = randn_bf16((B, Hkv, L, d), 1).float()
+    Vh = randn_bf16((B, Hkv, L, d), 2).float()
+    q = randn_bf16((T, B, Hq, d), 3).float()
+    kc = torch.full((B, Hkv, W, d), float("nan"))  # unfilled slots must never be read
+    vc = torch.full((B, Hkv, W, d), float("nan"))
+    for p in range(max(0, pos0 - W), pos0):
+        kc[:, :, p % W] = Kh[:, :, p]
+        vc[:, :, p % W] = Vh[:, :, p]
+    k_new = Kh[:, :, pos0:].permute(2, 0, 1, 3).contiguous()
+    v_new = Vh[:, :, pos0:].permute(2, 0, 1, 3).contiguous()
+    pos = np.array([[pos0 + t] * B for t in range(T)], dtype=np.int32)
+    out, kc2, vc2 = orc.decode(q, k_new, v_new, kc, vc, pos)
+    G = Hq // Hkv
+    for t in range(T):
+        p = pos0 + t
+        lo = max(0, p - W + 1)
+        Kw = Kh[:, :, lo:p + 1].double().repeat_interleave(G, dim=1)
+        Vw = Vh[:, :, lo:p + 1].double().repeat_interleave(G, dim=1)
+        ref = F.scaled_dot_product_attention(q[t].double()[:, :, None], Kw, Vw, scale=1 / 4)[:, :, 0]
+        assert np.abs(out[t] - ref.numpy()).max() < 1e-12
+    # the cache afterwards holds the last W positions at slot p % W
+    last = pos0 + T - 1
+    for p in range(max(0, last - W + 1), last + 1):
+        assert np.array_equal(kc2[:, :, p % W], Kh[:, :, p].numpy())
+
+
+# --------------------------------------------------------------- schedule --
+
+def tiles_touched_from_mask(allowed, band_allowed, Bq, Bk, S):
+    """Block-reduce boolean masks: which key tiles / stride tiles hold an
+    attended cell for each query tile."""
+    N = allowed.shape[0]
+    out = []
+    for qt in range((N + Bq - 1) // Bq):
+        rows = slice(qt * Bq, min(N, qt * Bq + Bq))
+        a, b = allowed[rows], band_allowed[rows]
+        extra = a & ~b
+        st = sorted({(j // S) // Bk for j in np.nonzero(extra.any(0))[0]}) if S else []
+        kt = sorted({j // Bk for j in np.nonzero(b.any(0))[0]})
+        out.append(([0x40000000 | t for t in st] + kt, int(a.sum())))
+    return out
+
+
+@pytest.mark.parametrize("kind,N,W,S,Bq,Bk", [
+    ("swa", 256, 64, 0, 128, 128), ("strided", 256, 16, 8, 128, 128), ("swa", 300, 50, 0, 64, 32),
+    ("strided", 517, 33, 5, 128, 16), ("swa", 100, 1000, 0, 32, 32), ("strided", 130, 1, 1, 64, 64),
+    ("causal", 200, 0, 0, 64, 32)])
+def test_schedule_matches_block_reduction(orc, kind, N, W, S, Bq, Bk):
+    ii, jj = np.meshgrid(np.arange(N), np.arange(N), indexing="ij")
+    if kind == "causal":
+        allowed = jj <= ii
+        band = allowed
+    else:
+        band = (ii - W < jj) & (jj <= ii)
+        allowed = band | ((jj % S == 0) & (jj <= ii)) if kind == "strided" else band
+    lists, cells = orc.schedule(kind, N, W, S, Bq, Bk)
+    want = tiles_touched_from_mask(allowed, band, Bq, Bk, S)
+    assert lists == [w[0] for w in want]
+    assert cells == [w[1] for w in want]
+    assert sum(cells) == int(allowed.sum())
+
+
+def test_schedule_tile_totals_at_workload_sizes(orc):
+    """Band tiles per (b, h) at 128 x 128 tiles; sampled tiles checked
+    against the explicit mask, totals against the interval count."""
+    def total(N, W, S):
+        t = 0
+        for qt in range((N + 127) // 128):
+            r0, r1 = qt * 128, min(N - 1, qt * 128 + 127)
+            t += r1 // 128 - max(0, r0 - W + 1) // 128 + 1
+            if S:
+                m = (max(0, r1 - W + 1) + S - 1) // S
+                t += (m + 127) // 128
+        return t
+    assert total(8192, 4096, 0) == 1584
+    assert total(131072, 1024, 0) == 9180
+    assert total(16384, 128, 128) == 382
+    for qt in (0, 1, 31, 63):
+        tiles, cells = orc.schedule_qtile("swa", 8192, 4096, 0, 128, 128, qt)
+        lo = max(0, qt * 128 - 4095) // 128
+        assert tiles == list(range(lo, qt + 1))
+    for qt in (0, 1, 2, 127):
+        tiles, cells = orc.schedule_qtile("strided", 16384, 128, 128, 128, 128, qt)
+        r1 = qt * 128 + 127
+        want_st = [0x40000000] if max(0, r1 - 127) > 0 else []
+        assert tiles == want_st + list(range(max(0, qt * 128 - 127) // 128, qt + 1))
+        assert cells == strided_closed(r1 + 1, 128, 128) - strided_closed(qt * 128, 128, 128)
+
+
+# ------------------------------------------------------- printed numbers ---
+
+def test_nsa_keys_printed_on_cheatsheet(orc):
+    nums = read_numbers("page_numbers.txt")
+    n = orc.count_nsa(1024, 32, 4, 128)
+    assert n == nums["nsa_keys_N1024_l32_k4_w128"] == 288
+    assert math.floor(10 * 1024 / n) / 10 == nums["nsa_reduction_printed"]
+
+
+def test_kv_cache_bytes_scales_with_window(orc):
+    nums = read_numbers("page_numbers.txt")
+    L, H, d = nums["kv_example_layers"], nums["kv_example_kv_heads"], nums["kv_example_d_head"]
+    N, W = nums["kv_example_seq_len"], nums["kv_example_window"]
+    full = orc.kv_cache_bytes(N, L, H, d, dtype=2)
+    swa = orc.kv_cache_bytes(N, L, H, d, dtype=2, window=W)
+    assert full == 2 * 80 * 8 * 128 * 131072 * 2 == 42949672960
+    assert swa == 1342177280
+    # the page's own scaling rule swa_kv = full_kv * (window / seq_len)
+    assert swa == full * W // N
+    # linear in min(N, W): doubling N past W changes nothing
+    assert orc.kv_cache_bytes(2 * N, L, H, d, window=W) == swa
+    assert orc.kv_cache_bytes(W // 2, L, H, d, window=W) * 2 == swa
+    # lesson quiz: 32k-token cache vs a 2048 window is 16x smaller
+    assert orc.kv_cache_bytes(32768, 1, 1, 1) // orc.kv_cache_bytes(32768, 1, 1, 1, window=2048) == \
+        nums["kv_reduction_w2048_s32768"]
+
+
+def test_core_flops_table(orc):
+    nums = read_numbers("page_numbers.txt")
+    b, s, d, w = 2, 64, 16, 8
+    dense = np.zeros((s, s))  # every pair allowed
+    assert orc.core_flops(orc.count_nonmasked(dense), d, b) == 4 * b * s * s * d
+    # a two-sided window of exactly w keys per row: s*w entries -> 4bswd
+    assert orc.core_flops(s * w, d, b) == 4 * b * s * w * d
+    assert (32768 * 32768) // (32768 * 2048) == nums["score_flops_reduction_w2048_s32768"]
