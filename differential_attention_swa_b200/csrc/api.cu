@@ -1,0 +1,253 @@
+// api.cu -- the extern "C" entry points declared in include/swa_attn.h:
+// argument checks (before any launch), TMA descriptor encoding, launches,
+// the schedule export and the device error flag.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/swa_attn.h"
+#include "internal.h"
+#include "schedule.cuh"
+
+namespace swa {
+
+// Device word the kernels set when a bounded wait runs out.
+__device__ int g_device_error = 0;
+
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+bool get_encoder() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  return g_encode != nullptr;
+}
+
+// 3-D bf16 view (inner = head dim, rows, outer = batch*heads) with a
+// 64 x 128 box and the 128-byte swizzle the MMA descriptors expect.
+bool encode_rows(CUtensorMap* m, const void* base, int d, int64_t rows, int64_t outer, int64_t row_stride_el,
+                 int64_t outer_stride_el) {
+  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)rows, (cuuint64_t)outer};
+  cuuint64_t strides[2] = {(cuuint64_t)row_stride_el * 2, (cuuint64_t)outer_stride_el * 2};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool head_dim_ok(int d) { return d == 64 || d == 128; }
+
+swa_status_t run_prefill(int kind, bool diff, const void* q, const void* k, const void* q2, const void* k2,
+                         const void* v, void* o, float* lse, const float* lambda, int B, int Hq, int Hkv, int N,
+                         int dqk, int dv, int W, int S, float scale, const swa_debug_t* dbg, void* stream) {
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return SWA_ERR_INVALID_ARG;
+  if (diff && (!aligned16(q2) || !aligned16(k2) || lambda == nullptr)) return SWA_ERR_INVALID_ARG;
+  if (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)) return SWA_ERR_INVALID_ARG;
+  if (B < 1 || Hq < 1 || Hkv < 1 || N < 1 || W < 1 || Hq % Hkv != 0) return SWA_ERR_INVALID_ARG;
+  if (kind == kMaskStrided && S < 1) return SWA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return SWA_ERR_INVALID_ARG;
+  if ((int64_t)B * Hq > (1 << 30) / 8) return SWA_ERR_INVALID_ARG;
+  if (!head_dim_ok(dqk) || !head_dim_ok(dv)) return SWA_ERR_UNSUPPORTED;
+  if (!diff && dqk != dv) return SWA_ERR_UNSUPPORTED;
+  if (diff && dqk != 64) return SWA_ERR_UNSUPPORTED;  // K1 and K2 share one ring slot
+  if (dbg && dbg->tiles && (dbg->tiles_cap < 1 || dbg->ntiles == nullptr)) return SWA_ERR_INVALID_ARG;
+  if (!get_encoder()) return SWA_ERR_CUDA;
+
+  const int G = Hq / Hkv;
+  PrefillMaps maps;
+  std::memset(&maps, 0, sizeof(maps));
+  const int64_t nB = (int64_t)B;
+  bool ok = encode_rows(&maps.q, q, dqk, N, nB * Hq, dqk, (int64_t)N * dqk) &&
+            encode_rows(&maps.k, k, dqk, N, nB * Hkv, dqk, (int64_t)N * dqk) &&
+            encode_rows(&maps.v, v, dv, N, nB * Hkv, dv, (int64_t)N * dv);
+  if (ok && diff)
+    ok = encode_rows(&maps.q2, q2, dqk, N, nB * Hq, dqk, (int64_t)N * dqk) &&
+         encode_rows(&maps.k2, k2, dqk, N, nB * Hkv, dqk, (int64_t)N * dqk);
+  if (ok && kind == kMaskStrided) {
+    // stride row m is key m*S: a view whose row stride is S rows of K/V
+    const int64_t rows = (N + (int64_t)S - 1) / S;
+    ok = encode_rows(&maps.ks, k, dqk, rows, nB * Hkv, (int64_t)S * dqk, (int64_t)N * dqk) &&
+         encode_rows(&maps.vs, v, dv, rows, nB * Hkv, (int64_t)S * dv, (int64_t)N * dv);
+  }
+  if (!ok) return SWA_ERR_INVALID_ARG;
+  if (!diff) maps.q2 = maps.q, maps.k2 = maps.k;
+  if (kind != kMaskStrided) maps.ks = maps.k, maps.vs = maps.v;
+
+  PrefillParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.N = N; p.W = W; p.S = (kind == kMaskStrided) ? S : 0;
+  p.G = G; p.kind = kind;
+  p.nq = (N + 127) / 128;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.o = o; p.lse = lse; p.lambda = lambda;
+  if (dbg) {
+    p.dbg_cells = dbg->cells;
+    p.dbg_tiles = dbg->tiles;
+    p.dbg_ntiles = dbg->ntiles;
+    p.dbg_cap = dbg->tiles_cap;
+    p.inject_timeout = dbg->inject_timeout;
+  }
+  int64_t nunits;
+  if (diff) {
+    p.mode = kModeDiff;
+    nunits = nB * Hq * p.nq;
+  } else if (G % 2 == 0) {
+    p.mode = kModeHeadPairs;
+    nunits = nB * Hkv * (G / 2) * p.nq;
+  } else {
+    p.mode = kModeTilePairs;
+    nunits = nB * Hq * ((p.nq + 1) / 2);
+  }
+  if (nunits > 0x7fffffff) return SWA_ERR_INVALID_ARG;
+  p.err_flag = device_error_ptr();
+  if (p.err_flag == nullptr) return SWA_ERR_CUDA;
+  cudaError_t e = launch_prefill(maps, p, dqk, dv, diff, (int)nunits, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
+}
+
+}  // namespace
+
+int* device_error_ptr() {
+  static int* ptrs[64] = {nullptr};
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (ptrs[dev] == nullptr) {
+    void* a = nullptr;
+    if (cudaGetSymbolAddress(&a, g_device_error) != cudaSuccess) return nullptr;
+    ptrs[dev] = static_cast<int*>(a);
+  }
+  return ptrs[dev];
+}
+
+int read_and_clear_device_error(cudaStream_t stream, int* err) {
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return -1;
+  int zero = 0;
+  if (cudaMemcpyFromSymbol(err, g_device_error, sizeof(int)) != cudaSuccess) return -1;
+  if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int)) != cudaSuccess) return -1;
+  return 0;
+}
+
+}  // namespace swa
+
+using namespace swa;
+
+extern "C" {
+
+swa_status_t swa_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                          int N, int d, int W, float scale, void* stream) {
+  return run_prefill(kMaskWindow, false, q, k, nullptr, nullptr, v, o, lse, nullptr, B, Hq, Hkv, N, d, d, W, 0,
+                     scale, nullptr, stream);
+}
+
+swa_status_t strided_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                              int Hkv, int N, int d, int W, int stride, float scale, void* stream) {
+  if (stride < 1) return SWA_ERR_INVALID_ARG;
+  return run_prefill(kMaskStrided, false, q, k, nullptr, nullptr, v, o, lse, nullptr, B, Hq, Hkv, N, d, d, W,
+                     stride, scale, nullptr, stream);
+}
+
+swa_status_t diff_attn_fwd(const void* q1, const void* k1, const void* q2, const void* k2, const void* v, void* o,
+                           const float* lambda, int B, int Hq, int Hkv, int N, int d_qk, int d_v, int W, float scale,
+                           void* stream) {
+  return run_prefill(kMaskWindow, true, q1, k1, q2, k2, v, o, nullptr, lambda, B, Hq, Hkv, N, d_qk, d_v, W, 0,
+                     scale, nullptr, stream);
+}
+
+swa_status_t swa_prefill_debug(int kind, const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                               int Hq, int Hkv, int N, int d, int W, int stride, float scale, const swa_debug_t* dbg,
+                               void* stream) {
+  if (kind != kMaskWindow && kind != kMaskStrided) return SWA_ERR_INVALID_ARG;
+  return run_prefill(kind, false, q, k, nullptr, nullptr, v, o, lse, nullptr, B, Hq, Hkv, N, d, d, W, stride, scale,
+                     dbg, stream);
+}
+
+size_t swa_decode_workspace_bytes(int B, int Hq, int Hkv, int d, int W) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || W < 1 || Hq % Hkv != 0 || (d != 64 && d != 128)) return 0;
+  return decode_partial_bytes(B, Hq, Hkv, d, W);
+}
+
+swa_status_t swa_decode_step(const void* q, const void* k_new, const void* v_new, void* k_cache, void* v_cache,
+                             const int32_t* pos, void* o, int B, int Hq, int Hkv, int d, int W, float scale,
+                             void* workspace, size_t ws_bytes, void* stream) {
+  if (!aligned16(q) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) || !aligned16(v_cache) ||
+      !aligned16(o) || pos == nullptr || (reinterpret_cast<uintptr_t>(pos) & 3u))
+    return SWA_ERR_INVALID_ARG;
+  if (B < 1 || Hq < 1 || Hkv < 1 || W < 1 || Hq % Hkv != 0) return SWA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return SWA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return SWA_ERR_UNSUPPORTED;
+  const int G = Hq / Hkv;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return SWA_ERR_UNSUPPORTED;
+  const size_t need = decode_partial_bytes(B, Hq, Hkv, d, W);
+  if (!aligned16(workspace) || ws_bytes < need) return SWA_ERR_INVALID_ARG;
+  DecodeParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.q = q; p.k_new = k_new; p.v_new = v_new; p.k_cache = k_cache; p.v_cache = v_cache; p.pos = pos; p.o = o;
+  p.partial = static_cast<float*>(workspace);
+  p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.d = d; p.W = W; p.G = G;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  cudaError_t e = launch_decode(p, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
+}
+
+int64_t swa_schedule(int kind, int N, int W, int stride, int Bq, int Bk, int32_t* qtile_offsets, int32_t* tiles,
+                     int64_t cap) {
+  if (N < 1 || Bq < 1 || Bk < 1 || kind < 0 || kind > 2) return -1;
+  if (kind != kMaskCausal && W < 1) return -1;
+  if (kind == kMaskStrided && stride < 1) return -1;
+  const int nq = (N + Bq - 1) / Bq;
+  int64_t n = 0;
+  for (int qt = 0; qt < nq; ++qt) {
+    if (qtile_offsets) qtile_offsets[qt] = (int32_t)n;
+    const QTileKeys keys = qtile_keys(kind, N, W, stride, Bq, Bk, qt);
+    const int cnt = qtile_nkeys(keys);
+    for (int e = 0; e < cnt; ++e, ++n)
+      if (tiles && n < cap) tiles[n] = qtile_entry(keys, e);
+  }
+  if (qtile_offsets) qtile_offsets[nq] = (int32_t)n;
+  return n;
+}
+
+int64_t swa_count_nonmasked(int kind, int N, int W, int stride) {
+  if (N < 0 || kind < 0 || kind > 2) return -1;
+  if (kind != kMaskCausal && W < 1) return -1;
+  if (kind == kMaskStrided && stride < 1) return -1;
+  if (N == 0) return 0;
+  return count_attended(kind, N, W, stride);
+}
+
+swa_status_t swa_last_device_error(void* stream) {
+  int err = 0;
+  if (read_and_clear_device_error(static_cast<cudaStream_t>(stream), &err) != 0) return SWA_ERR_CUDA;
+  return static_cast<swa_status_t>(err);
+}
+
+const char* swa_status_string(swa_status_t s) {
+  switch (s) {
+    case SWA_OK: return "ok";
+    case SWA_ERR_INVALID_ARG: return "invalid argument";
+    case SWA_ERR_UNSUPPORTED: return "unsupported head dimension or group size";
+    case SWA_ERR_CUDA: return "CUDA error";
+    case SWA_ERR_TIMEOUT: return "in-kernel wait timed out";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

@@ -1,0 +1,67 @@
+// internal.h -- declarations shared by the library's translation units (not
+// part of the public ABI).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+namespace swa {
+
+// Work-unit layouts of the prefill kernel (two 128-row "subs" per CTA).
+enum UnitMode {
+  kModeHeadPairs = 0,  // two query heads of one KV group, same rows
+  kModeTilePairs = 1,  // two consecutive query tiles of one head
+  kModeDiff = 2        // the two maps of differential attention
+};
+
+struct PrefillParams {
+  int B, Hq, Hkv, N, W, S;
+  int G;     // Hq / Hkv
+  int kind;  // MaskKind
+  int mode;  // UnitMode
+  int nq;    // query tiles of 128 rows
+  float scale_log2;  // scale * log2(e)
+  void* o;
+  float* lse;
+  const float* lambda;
+  int64_t* dbg_cells;
+  int32_t* dbg_tiles;
+  int32_t* dbg_ntiles;
+  int dbg_cap;
+  int inject_timeout;
+  int* err_flag;  // device word that receives SWA_ERR_TIMEOUT
+};
+
+struct PrefillMaps {
+  CUtensorMap q, q2, k, k2, v, ks, vs;
+};
+
+cudaError_t launch_prefill(const PrefillMaps& maps, const PrefillParams& p, int dqk, int dv, bool diff,
+                           int nunits, cudaStream_t stream);
+int prefill_smem_bytes(int dqk, int dv, bool diff);
+
+struct DecodeParams {
+  const void* q;
+  const void* k_new;
+  const void* v_new;
+  void* k_cache;
+  void* v_cache;
+  const int32_t* pos;
+  void* o;
+  float* partial;  // [B*Hq][nsplit][d + 2]
+  int B, Hq, Hkv, d, W, G;
+  int nsplit, chunk;
+  float scale_log2;
+};
+
+int decode_nsplit(int B, int Hkv, int W);
+size_t decode_partial_bytes(int B, int Hq, int Hkv, int d, int W);
+cudaError_t launch_decode(const DecodeParams& p, cudaStream_t stream);
+
+int* device_error_ptr();
+int read_and_clear_device_error(cudaStream_t stream, int* err);
+
+}  // namespace swa

@@ -1,0 +1,631 @@
+// prefill.cu -- masked attention forward on sm_100a (tcgen05 + TMA).
+//
+// Computes A = softmax(Q K^T * scale + log M) V ("Learn: Sparse &
+// Sliding-Window Attention", section 3) for the window, local+strided and
+// differential masks. The flash-style online softmax ("Attention Variants
+// Compared", tiled_softmax_dot; "Exploring Attention Variants", Flash
+// Attention section) keeps the N x N matrix off HBM.
+//
+// One CTA = one work unit of two "subs". A sub is 128 query rows of one head
+// with its own score tile S and output accumulator O in tensor memory and its
+// own softmax warpgroup. The two subs share the stream of K/V tiles:
+//   * two heads of one GQA group, same rows (Hq/Hkv even);
+//   * two consecutive 128-row query tiles of one head (otherwise);
+//   * the two maps of differential attention (Q1/K1 and Q2/K2, shared V).
+// While one softmax warpgroup works on its scores, the tensor core runs the
+// other sub's MMAs, so the exponentials overlap the matrix products.
+//
+// Warp roles (384 threads):
+//   warp 0      TMA producer: Q once, then K and V tiles through a ring of
+//               shared-memory slots.
+//   warp 1      TMEM owner and MMA issuer (one thread): S_t = Q_t K^T into
+//               TMEM, then O_t += P_t V once softmax t has written P_t.
+//   warps 4-7   softmax of sub 0, warps 8-11 softmax of sub 1: one thread
+//               per query row (TMEM lane), fp32 online softmax in the log2
+//               domain, P as bf16 into shared memory (128-byte swizzle),
+//               lazy rescaling of O, then the epilogue O / l -> bf16.
+// Every wait is bounded; on a timeout the CTA records SWA_ERR_TIMEOUT,
+// drains what it has in flight, frees TMEM and returns.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "internal.h"
+#include "ptx.cuh"
+#include "schedule.cuh"
+
+namespace swa {
+
+constexpr int BM = 128;  // query rows per sub (TMEM lanes)
+constexpr int BN = 128;  // keys per tile (S columns)
+constexpr int kThreads = 384;
+constexpr float kLog2e = 1.4426950408889634f;
+// Lazy rescale threshold (log2 units): O and l keep a stale row max until a
+// new score exceeds it by more than this, so P stays below 2^8.
+constexpr float kRescaleTau = 8.0f;
+
+template <int DQK, int DV, bool DIFF>
+struct PrefillCfg {
+  static constexpr int kQBytes = BM * DQK * 2;
+  static constexpr int kKBytes = BN * DQK * 2 * (DIFF ? 2 : 1);
+  static constexpr int kVBytes = BN * DV * 2;
+  static constexpr int kSlot = kKBytes > kVBytes ? kKBytes : kVBytes;
+  static constexpr int kPBytes = BM * BN * 2;
+  static constexpr int kTiles = 2 * kQBytes + 2 * kPBytes;
+  static constexpr int kBudget = 227 * 1024 - 1024 - 1024;  // minus alignment slack and barriers
+  static constexpr int kSlotsRaw = (kBudget - kTiles) / kSlot;
+  static constexpr int kSlots = kSlotsRaw > 8 ? 8 : kSlotsRaw;
+  static_assert(kSlots >= 2, "shared memory too small for the K/V ring");
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffP = 2 * kQBytes;
+  static constexpr int kOffSlots = kTiles;
+  static constexpr int kOffBar = kTiles + kSlots * kSlot;
+  static constexpr int kSmemBytes = kOffBar + 1024 + 1024;  // barriers area + alignment slack
+  static constexpr int kTmemCols = 512;
+  static constexpr int kOCol0 = 256;
+  static constexpr int kOCol1 = 256 + DV;
+  static_assert(256 + 2 * DV <= kTmemCols, "TMEM budget");
+};
+
+// Barrier block layout (8-byte mbarriers, then a few words).
+struct BarLayout {
+  static constexpr int kQ = 0;
+  static constexpr int kFull = 1;       // + slot
+  static constexpr int kEmpty = 9;      // + slot
+  static constexpr int kS = 17;         // + sub
+  static constexpr int kP = 19;         // + sub
+  static constexpr int kO = 21;         // + sub
+  static constexpr int kX = 23;         // differential hand-off of 1/l2
+  static constexpr int kFinal = 24;     // MMA drain on abort
+  static constexpr int kCount = 25;
+  static constexpr int kWordsOff = 256; // bytes: tmem base, abort flag
+  static constexpr int kF2Off = 512;    // bytes: 128 floats
+};
+
+struct Unit {
+  int b, hkv;
+  int hq[2];
+  int qt[2];
+  int valid[2];
+};
+
+__device__ __forceinline__ Unit decode_unit(const PrefillParams& p, int u) {
+  Unit r;
+  if (p.mode == kModeHeadPairs) {
+    const int half = p.G / 2;
+    const int per_b = p.Hkv * half;
+    const int qt = p.nq - 1 - u / (p.B * per_b);
+    const int bh = u % (p.B * per_b);
+    r.b = bh / per_b;
+    const int rem = bh % per_b;
+    r.hkv = rem / half;
+    const int gp = rem % half;
+    r.hq[0] = r.hkv * p.G + 2 * gp;
+    r.hq[1] = r.hq[0] + 1;
+    r.qt[0] = r.qt[1] = qt;
+    r.valid[0] = r.valid[1] = 1;
+  } else if (p.mode == kModeTilePairs) {
+    const int nqp = (p.nq + 1) / 2;
+    const int qp = nqp - 1 - u / (p.B * p.Hq);
+    const int bh = u % (p.B * p.Hq);
+    r.b = bh / p.Hq;
+    r.hq[0] = r.hq[1] = bh % p.Hq;
+    r.hkv = r.hq[0] / p.G;
+    r.qt[0] = 2 * qp;
+    r.qt[1] = 2 * qp + 1;
+    r.valid[0] = 1;
+    r.valid[1] = r.qt[1] < p.nq;
+  } else {  // differential: both maps of the same rows
+    const int qt = p.nq - 1 - u / (p.B * p.Hq);
+    const int bh = u % (p.B * p.Hq);
+    r.b = bh / p.Hq;
+    r.hq[0] = r.hq[1] = bh % p.Hq;
+    r.hkv = r.hq[0] / p.G;
+    r.qt[0] = r.qt[1] = qt;
+    r.valid[0] = r.valid[1] = 1;
+  }
+  return r;
+}
+
+// The unit's key items: stride tiles 0 .. nst-1, then window tiles
+// blo .. bhi (union over the two subs, which is contiguous).
+struct Items {
+  QTileKeys k[2];
+  int nst, blo, bhi, n;
+};
+
+__device__ __forceinline__ Items unit_items(const PrefillParams& p, const Unit& un) {
+  Items it;
+  it.nst = 0;
+  it.blo = 0x7fffffff;
+  it.bhi = -1;
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    if (un.valid[t]) {
+      it.k[t] = qtile_keys(p.kind, p.N, p.W, p.S, BM, BN, un.qt[t]);
+      it.nst = imax(it.nst, it.k[t].n_stride);
+      it.blo = imin(it.blo, it.k[t].band_lo);
+      it.bhi = imax(it.bhi, it.k[t].band_hi);
+    } else {
+      it.k[t].band_lo = 1;
+      it.k[t].band_hi = 0;
+      it.k[t].n_stride = 0;
+    }
+  }
+  it.n = it.nst + (it.bhi - it.blo + 1);
+  return it;
+}
+
+__device__ __forceinline__ bool item_is_stride(const Items& it, int u) { return u < it.nst; }
+__device__ __forceinline__ int item_tile(const Items& it, int u) {
+  return u < it.nst ? u : it.blo + (u - it.nst);
+}
+__device__ __forceinline__ bool item_in_sub(const Items& it, int t, int u) {
+  if (u < it.nst) return u < it.k[t].n_stride;
+  const int kt = it.blo + (u - it.nst);
+  return kt >= it.k[t].band_lo && kt <= it.k[t].band_hi;
+}
+
+__device__ __forceinline__ void record_timeout(volatile int* abort_flag, int* err_flag) {
+  *abort_flag = 1;
+  atomicExch(err_flag, 4 /* SWA_ERR_TIMEOUT */);
+}
+
+template <int DQK, int DV, bool DIFF>
+__global__ void __launch_bounds__(kThreads, 1)
+    prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_q2,
+                   const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_k2,
+                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_ks,
+                   const __grid_constant__ CUtensorMap tm_vs, const PrefillParams p) {
+  using C = PrefillCfg<DQK, DV, DIFF>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bars = sbase + C::kOffBar;
+  auto bar = [&](int i) -> uint32_t { return bars + 8u * i; };
+  uint32_t* words = reinterpret_cast<uint32_t*>(smem + C::kOffBar + BarLayout::kWordsOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(words + 1);
+  float* f2s = reinterpret_cast<float*>(smem + C::kOffBar + BarLayout::kF2Off);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  const Unit un = decode_unit(p, blockIdx.x);
+  const Items it = unit_items(p, un);
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(BarLayout::kQ), 1);
+    for (int s = 0; s < C::kSlots; ++s) {
+      mbar_init(bar(BarLayout::kFull + s), 1);
+      mbar_init(bar(BarLayout::kEmpty + s), 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(bar(BarLayout::kS + t), 1);
+      mbar_init(bar(BarLayout::kP + t), 128);
+      mbar_init(bar(BarLayout::kO + t), 1);
+    }
+    mbar_init(bar(BarLayout::kX), 128);
+    mbar_init(bar(BarLayout::kFinal), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(words), C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = words[0];
+
+  if (warp == 0) {
+    // ------------------------------------------------------ producer ---
+    if (lane == 0) {
+      tma_prefetch_map(&tm_q);
+      tma_prefetch_map(&tm_k);
+      tma_prefetch_map(&tm_v);
+      if (DIFF) {
+        tma_prefetch_map(&tm_q2);
+        tma_prefetch_map(&tm_k2);
+      }
+      if (p.kind == kMaskStrided) {
+        tma_prefetch_map(&tm_ks);
+        tma_prefetch_map(&tm_vs);
+      }
+      const int nvalid = un.valid[0] + un.valid[1];
+      mbar_arrive_expect_tx(bar(BarLayout::kQ), nvalid * C::kQBytes);
+      for (int t = 0; t < 2; ++t) {
+        if (!un.valid[t]) continue;
+        const CUtensorMap* m = (DIFF && t == 1) ? &tm_q2 : &tm_q;
+        for (int bx = 0; bx < DQK / 64; ++bx)
+          tma_load_3d(sbase + C::kOffQ + t * C::kQBytes + bx * 16384, m, bar(BarLayout::kQ), bx * 64,
+                      un.qt[t] * BM, un.b * p.Hq + un.hq[t]);
+      }
+      const int zkv = un.b * p.Hkv + un.hkv;
+      int L = 0;
+      int issued[8];
+      for (int s = 0; s < 8; ++s) issued[s] = 0;
+      bool ok = true;
+      for (int u = 0; u < it.n && ok; ++u) {
+        const bool st = item_is_stride(it, u);
+        const int row = item_tile(it, u) * BN;
+        // K (or K1 and K2)
+        {
+          const int slot = L % C::kSlots, use = L / C::kSlots;
+          ++L;
+          if (use > 0 && !mbar_wait(bar(BarLayout::kEmpty + slot), (use - 1) & 1, abort_flag)) {
+            record_timeout(abort_flag, p.err_flag);
+            ok = false;
+            break;
+          }
+          if (!(p.inject_timeout && blockIdx.x == 0 && u == 0)) {
+            mbar_arrive_expect_tx(bar(BarLayout::kFull + slot), C::kKBytes);
+            const uint32_t dst = sbase + C::kOffSlots + slot * C::kSlot;
+            const CUtensorMap* m = st ? &tm_ks : &tm_k;
+            for (int bx = 0; bx < DQK / 64; ++bx)
+              tma_load_3d(dst + bx * 16384, m, bar(BarLayout::kFull + slot), bx * 64, row, zkv);
+            if (DIFF)
+              for (int bx = 0; bx < DQK / 64; ++bx)
+                tma_load_3d(dst + BN * DQK * 2 + bx * 16384, &tm_k2, bar(BarLayout::kFull + slot),
+                            bx * 64, row, zkv);
+            issued[slot] = use + 1;
+          }
+        }
+        // V
+        {
+          const int slot = L % C::kSlots, use = L / C::kSlots;
+          ++L;
+          if (use > 0 && !mbar_wait(bar(BarLayout::kEmpty + slot), (use - 1) & 1, abort_flag)) {
+            record_timeout(abort_flag, p.err_flag);
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(bar(BarLayout::kFull + slot), C::kVBytes);
+          const uint32_t dst = sbase + C::kOffSlots + slot * C::kSlot;
+          const CUtensorMap* m = st ? &tm_vs : &tm_v;
+          for (int bx = 0; bx < DV / 64; ++bx)
+            tma_load_3d(dst + bx * 16384, m, bar(BarLayout::kFull + slot), bx * 64, row, zkv);
+          issued[slot] = use + 1;
+        }
+      }
+      if (!ok || *abort_flag) {
+        // drain: every load issued lands before the CTA may exit
+        for (int s = 0; s < C::kSlots; ++s)
+          if (issued[s] > 0) mbar_wait_timed(bar(BarLayout::kFull + s), (issued[s] - 1) & 1);
+        mbar_wait_timed(bar(BarLayout::kQ), 0);
+      }
+    }
+  } else if (warp == 1) {
+    // ----------------------------------------------------------- MMA ---
+    if (lane == 0) {
+      const uint32_t idesc_s = idesc_bf16_f32(BM, BN, false);
+      const uint32_t idesc_pv = idesc_bf16_f32(BM, DV, true);
+      const int zq = un.b * p.Hq;
+      int kcount[2] = {0, 0};
+      int pending_v[2] = {-1, -1};  // V slot of the item whose PV is still to issue
+      int64_t dbg_row[2] = {-1, -1};
+      for (int t = 0; t < 2; ++t)
+        if (un.valid[t] && p.dbg_tiles && !(DIFF && t == 1))
+          dbg_row[t] = (int64_t)(zq + un.hq[t]) * p.nq + un.qt[t];
+      bool ok = mbar_wait(bar(BarLayout::kQ), 0, abort_flag);
+      if (!ok) record_timeout(abort_flag, p.err_flag);
+      tc_fence_after();
+      int L = 0;
+      int prev_vslot = -1;
+      auto issue_pv = [&](int t) -> bool {
+        const int vslot = pending_v[t];
+        const uint32_t vb = sbase + C::kOffSlots + vslot * C::kSlot;
+        const uint32_t pb = sbase + C::kOffP + t * C::kPBytes;
+        const uint32_t dcol = tmem + (t == 0 ? C::kOCol0 : C::kOCol1);
+        const int first = (kcount[t] == 1);  // this PV is the sub's first
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk) {
+          const uint64_t a = sw128_desc(pb + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+          const uint64_t b = sw128_desc(vb + kk * 2048, 16384, 1024);
+          umma_bf16_ss(dcol, a, b, idesc_pv, (first && kk == 0) ? 0u : 1u);
+        }
+        umma_commit(bar(BarLayout::kO + t));
+        pending_v[t] = -1;
+        return true;
+      };
+      for (int u = 0; u < it.n && ok; ++u) {
+        const int kslot = L % C::kSlots, kuse = L / C::kSlots;
+        ++L;
+        const int vslot = L % C::kSlots, vuse = L / C::kSlots;
+        ++L;
+        if (!mbar_wait(bar(BarLayout::kFull + kslot), kuse & 1, abort_flag)) {
+          record_timeout(abort_flag, p.err_flag);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        for (int t = 0; t < 2 && ok; ++t) {
+          const bool in = item_in_sub(it, t, u);
+          if (!in && pending_v[t] < 0) continue;
+          if (kcount[t] > 0) {
+            if (!mbar_wait(bar(BarLayout::kP + t), (kcount[t] - 1) & 1, abort_flag)) {
+              record_timeout(abort_flag, p.err_flag);
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+          }
+          if (in) {
+            const uint32_t qb = sbase + C::kOffQ + t * C::kQBytes;
+            const uint32_t kb = sbase + C::kOffSlots + kslot * C::kSlot + ((DIFF && t == 1) ? BN * DQK * 2 : 0);
+            const uint32_t dcol = tmem + t * BN;
+#pragma unroll
+            for (int kk = 0; kk < DQK / 16; ++kk) {
+              const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+              umma_bf16_ss(dcol, sw128_desc(qb + off, 16, 1024), sw128_desc(kb + off, 16, 1024), idesc_s,
+                           kk > 0 ? 1u : 0u);
+            }
+            umma_commit(bar(BarLayout::kS + t));
+            if (dbg_row[t] >= 0 && kcount[t] < p.dbg_cap)
+              p.dbg_tiles[dbg_row[t] * p.dbg_cap + kcount[t]] =
+                  item_is_stride(it, u) ? (kStrideTag | item_tile(it, u)) : item_tile(it, u);
+          }
+          if (pending_v[t] >= 0) issue_pv(t);
+          if (in) ++kcount[t];
+        }
+        if (!ok) break;
+        umma_commit(bar(BarLayout::kEmpty + kslot));
+        if (prev_vslot >= 0) umma_commit(bar(BarLayout::kEmpty + prev_vslot));
+        // V of this item must be resident before its PVs (issued next round)
+        if (!mbar_wait(bar(BarLayout::kFull + vslot), vuse & 1, abort_flag)) {
+          record_timeout(abort_flag, p.err_flag);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        for (int t = 0; t < 2; ++t)
+          if (item_in_sub(it, t, u)) pending_v[t] = vslot;
+        prev_vslot = vslot;
+      }
+      for (int t = 0; t < 2 && ok; ++t) {
+        if (pending_v[t] < 0) continue;
+        if (!mbar_wait(bar(BarLayout::kP + t), (kcount[t] - 1) & 1, abort_flag)) {
+          record_timeout(abort_flag, p.err_flag);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        issue_pv(t);
+      }
+      for (int t = 0; t < 2; ++t)
+        if (dbg_row[t] >= 0) p.dbg_ntiles[dbg_row[t]] = kcount[t];
+      if (!ok || *abort_flag) {
+        umma_commit(bar(BarLayout::kFinal));
+        mbar_wait_timed(bar(BarLayout::kFinal), 0);
+      }
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------- softmax ---
+    const int t = (warp - 4) >> 2;       // sub
+    const int qw = warp & 3;             // TMEM lane quarter
+    const int r = qw * 32 + lane;        // row within the sub's tile
+    const uint32_t lane_addr = static_cast<uint32_t>(qw * 32) << 16;
+    const uint32_t s_tmem = tmem + lane_addr + t * BN;
+    const uint32_t o_tmem = tmem + lane_addr + (t == 0 ? C::kOCol0 : C::kOCol1);
+    const uint32_t pbase = sbase + C::kOffP + t * C::kPBytes;
+    const bool valid_sub = un.valid[t] != 0;
+    const int i = un.qt[t] * BM + r;                 // query index
+    const bool row_ok = valid_sub && i < p.N;
+    const int Wc = (p.kind == kMaskCausal) ? p.N : p.W;
+    const int lo = window_lo(i, Wc);
+    const int mst = (p.kind == kMaskStrided) ? stride_rows_below(lo, p.S) : 0;
+    const float cl2 = p.scale_log2;
+
+    float m_run = -INFINITY;  // running max, log2 units (scores * scale * log2 e)
+    float l_run = 0.f;
+    long long cells = 0;
+    int k = 0;
+    bool ok = true;
+
+    if (valid_sub) {
+      for (int u = 0; u < it.n; ++u) {
+        if (!item_in_sub(it, t, u)) continue;
+        // attended columns [c0, c1] of this row in this tile
+        int c0, c1;
+        const int tile = item_tile(it, u);
+        if (item_is_stride(it, u)) {
+          c0 = 0;
+          c1 = imin(mst - 1 - tile * BN, BN - 1);
+        } else {
+          c0 = imax(lo - tile * BN, 0);
+          c1 = imin(i - tile * BN, BN - 1);
+        }
+        if (!row_ok) { c0 = 1; c1 = 0; }
+        if (c1 >= c0) cells += c1 - c0 + 1;
+        const bool full = (c0 == 0 && c1 == BN - 1);
+
+        const bool got = mbar_wait(bar(BarLayout::kS + t), k & 1, abort_flag);
+        if (!__all_sync(0xffffffffu, got)) { if (lane == 0) record_timeout(abort_flag, p.err_flag); ok = false; break; }
+        tc_fence_after();
+
+        float s[BN];
+        tmem_ld64(s_tmem, s);
+        tmem_ld64(s_tmem + 64, s + 64);
+        if (!__all_sync(0xffffffffu, full)) {
+#pragma unroll
+          for (int c = 0; c < BN; ++c)
+            if (c < c0 || c > c1) s[c] = -INFINITY;
+        }
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < BN; ++c) mx = fmaxf(mx, s[c]);
+        const float m_tile = mx * cl2;  // -inf stays -inf
+        float m_use = m_run, alpha = 1.f;
+        bool rescale = false;
+        if (m_tile > m_run) {
+          if (m_run == -INFINITY) {
+            m_use = m_tile;  // nothing accumulated yet: O row is 0 (or not written)
+            alpha = 0.f;
+          } else if (m_tile - m_run > kRescaleTau) {
+            m_use = m_tile;
+            alpha = ex2_approx(m_run - m_tile);
+            rescale = true;
+          }
+        }
+        const float msub = (m_use == -INFINITY) ? 0.f : m_use;
+        float rs = 0.f;
+        uint32_t pk[BN / 2];
+#pragma unroll
+        for (int c = 0; c < BN; c += 2) {
+          const float p0 = ex2_approx(fmaf(s[c], cl2, -msub));
+          const float p1 = ex2_approx(fmaf(s[c + 1], cl2, -msub));
+          rs += p0 + p1;
+          pk[c / 2] = pack_bf16(p0, p1);
+        }
+        l_run = l_run * alpha + rs;
+        m_run = m_use;
+
+        if (k > 0) {
+          const bool go = mbar_wait(bar(BarLayout::kO + t), (k - 1) & 1, abort_flag);
+          if (!__all_sync(0xffffffffu, go)) { if (lane == 0) record_timeout(abort_flag, p.err_flag); ok = false; break; }
+          tc_fence_after();
+          if (__any_sync(0xffffffffu, rescale)) {
+            const float f = rescale ? alpha : 1.f;
+#pragma unroll 1
+            for (int c = 0; c < DV; c += 32) {
+              float o[32];
+              tmem_ld32(o_tmem + c, o);
+#pragma unroll
+              for (int e = 0; e < 32; ++e) o[e] *= f;
+              tmem_st32(o_tmem + c, o);
+            }
+          }
+        }
+        // P row -> shared memory, 128-byte swizzle (16-byte chunk j of row r
+        // goes to chunk j ^ (r & 7) of the row's 128-byte line)
+#pragma unroll
+        for (int j = 0; j < BN / 8; ++j) {
+          const uint32_t box = j >> 3, cb = j & 7;
+          const uint32_t addr = pbase + box * 16384 + r * 128 + ((cb ^ (r & 7)) << 4);
+          st_shared_v4(addr, pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(bar(BarLayout::kP + t));
+        ++k;
+      }
+    }
+
+    // ---------------------------------------------------- epilogue ---
+    if (ok && valid_sub && k > 0) {
+      const bool got = mbar_wait(bar(BarLayout::kO + t), (k - 1) & 1, abort_flag);
+      ok = __all_sync(0xffffffffu, got);
+      if (!ok && lane == 0) record_timeout(abort_flag, p.err_flag);
+    }
+    if (ok && valid_sub && k > 0) {
+      tc_fence_after();
+      const int hq = un.hq[t];
+      const int64_t orow = ((int64_t)(un.b * p.Hq + hq) * p.N + i);
+      if (DIFF) {
+        if (t == 1) {
+          f2s[r] = (l_run > 0.f) ? p.lambda[hq] / l_run : 0.f;
+          mbar_arrive(bar(BarLayout::kX));
+        } else {
+          const bool g1 = mbar_wait(bar(BarLayout::kO + 1), (k - 1) & 1, abort_flag);
+          const bool g2 = mbar_wait(bar(BarLayout::kX), 0, abort_flag);
+          if (!__all_sync(0xffffffffu, g1 && g2)) {
+            if (lane == 0) record_timeout(abort_flag, p.err_flag);
+          } else {
+            tc_fence_after();
+            const float inv1 = 1.f / l_run;
+            const float f2 = f2s[r];
+            const uint32_t o2_tmem = tmem + lane_addr + C::kOCol1;
+            __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.o) + orow * DV;
+#pragma unroll 1
+            for (int c = 0; c < DV; c += 32) {
+              float a[32], b2[32];
+              tmem_ld32(o_tmem + c, a);
+              tmem_ld32(o2_tmem + c, b2);
+              if (row_ok) {
+#pragma unroll
+                for (int e = 0; e < 32; e += 8) {
+                  st_global_v4(dst + c + e, pack_bf16(a[e] * inv1 - b2[e] * f2, a[e + 1] * inv1 - b2[e + 1] * f2),
+                               pack_bf16(a[e + 2] * inv1 - b2[e + 2] * f2, a[e + 3] * inv1 - b2[e + 3] * f2),
+                               pack_bf16(a[e + 4] * inv1 - b2[e + 4] * f2, a[e + 5] * inv1 - b2[e + 5] * f2),
+                               pack_bf16(a[e + 6] * inv1 - b2[e + 6] * f2, a[e + 7] * inv1 - b2[e + 7] * f2));
+                }
+              }
+            }
+          }
+        }
+      } else {
+        const float inv = 1.f / l_run;
+        __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.o) + orow * DV;
+#pragma unroll 1
+        for (int c = 0; c < DV; c += 32) {
+          float a[32];
+          tmem_ld32(o_tmem + c, a);
+          if (row_ok) {
+#pragma unroll
+            for (int e = 0; e < 32; e += 8)
+              st_global_v4(dst + c + e, pack_bf16(a[e] * inv, a[e + 1] * inv), pack_bf16(a[e + 2] * inv, a[e + 3] * inv),
+                           pack_bf16(a[e + 4] * inv, a[e + 5] * inv), pack_bf16(a[e + 6] * inv, a[e + 7] * inv));
+          }
+        }
+        if (p.lse && row_ok) p.lse[orow] = (m_run + __log2f(l_run)) * 0.6931471805599453f;
+      }
+      if (p.dbg_cells && !(DIFF && t == 1)) {
+        long long c = row_ok ? cells : 0;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) c += __shfl_xor_sync(0xffffffffu, c, off);
+        if (lane == 0)
+          atomicAdd(reinterpret_cast<unsigned long long*>(p.dbg_cells + (int64_t)(un.b * p.Hq + hq) * p.nq + un.qt[t]),
+                    static_cast<unsigned long long>(c));
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+template <int DQK, int DV, bool DIFF>
+static cudaError_t launch_one(const PrefillMaps& maps, const PrefillParams& p, int nunits, cudaStream_t stream) {
+  using C = PrefillCfg<DQK, DV, DIFF>;
+  auto kern = prefill_kernel<DQK, DV, DIFF>;
+  static bool attr_set = false;  // per process; the attribute is per function
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  kern<<<nunits, kThreads, C::kSmemBytes, stream>>>(maps.q, maps.q2, maps.k, maps.k2, maps.v, maps.ks, maps.vs, p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_prefill(const PrefillMaps& maps, const PrefillParams& p, int dqk, int dv, bool diff,
+                           int nunits, cudaStream_t stream) {
+  if (diff) {
+    if (dqk == 64 && dv == 128) return launch_one<64, 128, true>(maps, p, nunits, stream);
+    if (dqk == 64 && dv == 64) return launch_one<64, 64, true>(maps, p, nunits, stream);
+    return cudaErrorInvalidValue;
+  }
+  if (dqk == 128 && dv == 128) return launch_one<128, 128, false>(maps, p, nunits, stream);
+  if (dqk == 64 && dv == 64) return launch_one<64, 64, false>(maps, p, nunits, stream);
+  return cudaErrorInvalidValue;
+}
+
+int prefill_smem_bytes(int dqk, int dv, bool diff) {
+  if (diff) {
+    if (dqk == 64 && dv == 128) return PrefillCfg<64, 128, true>::kSmemBytes;
+    if (dqk == 64 && dv == 64) return PrefillCfg<64, 64, true>::kSmemBytes;
+    return -1;
+  }
+  if (dqk == 128 && dv == 128) return PrefillCfg<128, 128, false>::kSmemBytes;
+  if (dqk == 64 && dv == 64) return PrefillCfg<64, 64, false>::kSmemBytes;
+  return -1;
+}
+
+}  // namespace swa

@@ -1,0 +1,98 @@
+// schedule.cuh -- which key tiles a query tile touches.
+//
+// One definition, compiled for both sides: the prefill kernel enumerates its
+// key tiles with these functions and swa_schedule() exports the same lists
+// for the parity tests. The mask is never stored; each function evaluates
+// the window / stride predicate on the tile's edge rows.
+//
+// Masks ("Learn: Sparse & Sliding-Window Attention", section 3; "Attention
+// Variants Compared", swa_mask / strided_mask code):
+//   window:  key j attended by row i iff  lo_i <= j <= i,  lo_i = max(0, i-W+1)
+//   strided: window OR (j % S == 0 and j <= i).
+// A cell outside the window is a stride cell iff j % S == 0 and j < lo_i, so
+// the union splits into disjoint window cells and stride cells, and each
+// attended cell is visited exactly once.
+//
+// Stride cells are gathered by a strided view of K/V: stride row m holds key
+// m*S. A "stride tile" ct holds stride rows ct*Bk .. ct*Bk+Bk-1.
+#pragma once
+
+#ifdef __CUDACC__
+#define SWA_HD __host__ __device__ __forceinline__
+#else
+#define SWA_HD inline
+#endif
+
+namespace swa {
+
+constexpr int kStrideTag = 0x40000000;
+
+enum MaskKind { kMaskWindow = 0, kMaskStrided = 1, kMaskCausal = 2 };
+
+SWA_HD int imin(int a, int b) { return a < b ? a : b; }
+SWA_HD int imax(int a, int b) { return a > b ? a : b; }
+
+// First attended key of row i under the window.
+SWA_HD int window_lo(int i, int W) { return imax(0, i - W + 1); }
+
+// Number of stride rows m with m*S < lo (keys below the window of a row
+// whose window starts at lo).
+SWA_HD int stride_rows_below(int lo, int S) { return (lo + S - 1) / S; }
+
+struct QTileKeys {
+  int band_lo;   // first window key tile
+  int band_hi;   // last window key tile
+  int n_stride;  // stride tiles 0 .. n_stride-1
+};
+
+// Key tiles of query tile qt (rows qt*Bq .. min(N, qt*Bq+Bq) - 1). W >= N
+// (or kind == causal) is full causal. The window part is the contiguous
+// range from the tile holding the first row's lo to the tile holding the
+// last row; every tile in it has an attended cell because consecutive rows'
+// windows overlap or abut. Stride tiles are those with a stride row below
+// the last row's lo (the largest lo in the tile).
+SWA_HD QTileKeys qtile_keys(int kind, int N, int W, int S, int Bq, int Bk, int qt) {
+  QTileKeys r;
+  const int r0 = qt * Bq;
+  const int r1 = imin(N - 1, r0 + Bq - 1);
+  const int Wc = (kind == kMaskCausal) ? N : W;
+  r.band_lo = window_lo(r0, Wc) / Bk;
+  r.band_hi = r1 / Bk;
+  r.n_stride = 0;
+  if (kind == kMaskStrided && S > 0) {
+    const int m = stride_rows_below(window_lo(r1, Wc), S);
+    r.n_stride = (m + Bk - 1) / Bk;
+  }
+  return r;
+}
+
+SWA_HD int qtile_nkeys(const QTileKeys& k) { return k.n_stride + (k.band_hi - k.band_lo + 1); }
+
+// Entry e of the query tile's visiting order: stride tiles first (oldest
+// keys), then window tiles ascending. Encoded as in swa_debug_t.
+SWA_HD int qtile_entry(const QTileKeys& k, int e) {
+  return e < k.n_stride ? (kStrideTag | e) : (k.band_lo + (e - k.n_stride));
+}
+
+// Closed-form ||M||_0 of one N x N mask.
+SWA_HD long long count_attended(int kind, int N, int W, int S) {
+  if (kind == kMaskCausal || W >= N) {
+    long long n = N;
+    long long band = n * (n + 1) / 2;
+    return band;  // no stride cells: every lo_i is 0
+  }
+  long long n = N, w = W;
+  long long band = n * w - w * (w - 1) / 2;
+  if (kind != kMaskStrided || S <= 0) return band;
+  // stride cells: sum over rows i >= W of ceil((i - W + 1) / S)
+  // = sum over t = 1 .. N-W of ceil(t / S)
+  long long T = n - w;  // rows with lo_i = t for t = 1 .. T
+  long long s = S;
+  long long q = T / s, rem = T % s;
+  // t = 1..q*s: ceil(t/s) = block index b+1 for t in (b*s, (b+1)*s]
+  long long full = s * q * (q + 1) / 2;
+  long long tail = rem * (q + 1);
+  return band + full + tail;
+}
+
+}  // namespace swa

@@ -1,0 +1,167 @@
+/*
+ * swa_attn.h -- C ABI of the B200 (sm_100a) masked-attention library.
+ *
+ * One operation, in several masks: the masked attention forward
+ *     A = softmax(Q K^T * scale + log M) V,   log M_ij = 0 (allowed) or -inf,
+ * from "Learn: Sparse & Sliding-Window Attention", section 3 "The math". The
+ * mask is never stored; each query tile visits only the key tiles its mask
+ * touches, so the work grows with the number of attended cells.
+ *
+ * Conventions shared by every entry point:
+ *   - Tensors are row-major, contiguous, bf16 unless stated: Q [B, Hq, N, d],
+ *     K and V [B, Hkv, N, d]. Query head h reads KV head h / (Hq / Hkv)
+ *     (grouped-query attention, "Sliding Window Attention" glossary page,
+ *     GQA entry; the consecutive grouping is this library's reading).
+ *   - Every pointer argument named as device memory must be device memory of
+ *     the current CUDA device, 16-byte aligned. The caller allocates and owns
+ *     every buffer; the library allocates nothing at call time and keeps no
+ *     pointer after the call returns.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream). Calls
+ *     are asynchronous on that stream: on return the work is queued, not
+ *     done.
+ *   - Argument errors are reported before anything is launched
+ *     (SWA_ERR_INVALID_ARG / SWA_ERR_UNSUPPORTED). A failed launch returns
+ *     SWA_ERR_CUDA. Every wait inside a kernel is bounded (about two
+ *     seconds); a kernel whose wait runs out records SWA_ERR_TIMEOUT in a
+ *     device flag, releases what it holds and returns; swa_last_device_error
+ *     reports it.
+ *   - Outputs are bf16 rounded to nearest even from fp32 accumulators.
+ */
+#ifndef SWA_ATTN_H
+#define SWA_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SWA_OK = 0,
+  SWA_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size or ratio  */
+  SWA_ERR_UNSUPPORTED = 2, /* valid but not built: head dim outside {64,128} */
+  SWA_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed           */
+  SWA_ERR_TIMEOUT = 4      /* a bounded in-kernel wait ran out            */
+} swa_status_t;
+
+/* Optional device-side debug outputs of the prefill kernels (pass NULL to
+ * skip). Indexing is per (b, hq, query tile of 128 rows):
+ * idx = (b * Hq + hq) * ceil(N / 128) + qt.
+ *   cells  [B*Hq*nq] int64: attended cells the kernel processed for that
+ *          query tile are ADDED here (zero it first).
+ *   tiles  [B*Hq*nq*tiles_cap] int32: the key tiles the kernel visited, in
+ *          visiting order: a window tile is its index kt (keys kt*128 ..
+ *          kt*128+127); a stride tile is 0x40000000 | ct (stride keys
+ *          m*S for m in ct*128 .. ct*128+127).
+ *   ntiles [B*Hq*nq] int32: how many entries were visited (may exceed
+ *          tiles_cap; only the first tiles_cap are written).
+ *   inject_timeout: nonzero makes the kernel withhold its first key tile so
+ *          that its waits run out and it returns SWA_ERR_TIMEOUT through
+ *          swa_last_device_error (a test of the error path; nothing hangs).
+ */
+typedef struct {
+  int64_t* cells;
+  int32_t* tiles;
+  int32_t* ntiles;
+  int32_t tiles_cap;
+  int32_t inject_timeout;
+} swa_debug_t;
+
+/* Sliding-window attention forward.
+ * Source: "Learn: Sparse & Sliding-Window Attention", section 3a, band mask
+ * M_ij = 1[i - W < j <= i]; "Attention Variants Compared", swa_mask code
+ * (lo = max(0, i - window + 1); window >= n gives full causal).
+ *   q [B,Hq,N,d], k, v [B,Hkv,N,d] bf16 (device, read only);
+ *   o [B,Hq,N,d] bf16 (device, written);
+ *   lse [B,Hq,N] fp32 natural-log sum of exp of the scaled scores, or NULL;
+ *   d in {64, 128}; W >= 1 (W >= N is full causal); Hq % Hkv == 0;
+ *   scale > 0 multiplies Q K^T (1/sqrt(d) for the usual attention). */
+swa_status_t swa_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                          int B, int Hq, int Hkv, int N, int d, int W, float scale, void* stream);
+
+/* Local + strided attention forward: the window mask OR every stride-th key
+ * (keys j with j % stride == 0 and j <= i). Each attended cell counts once.
+ * Source: "Attention Variants Compared", strided_mask code ("local window,
+ * then every stride-th token back to 0"); "Exploring Attention Variants",
+ * Sparse Attention section (the two masks combined by logical OR).
+ * Arguments as swa_attn_fwd, plus stride >= 1. */
+swa_status_t strided_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                              int B, int Hq, int Hkv, int N, int d, int W, int stride,
+                              float scale, void* stream);
+
+/* Differential attention forward:
+ *     o = softmax(Q1 K1^T * scale + log M) V - lambda[h] * softmax(Q2 K2^T * scale + log M) V
+ * over one shared V, both maps under the same window mask (W >= N: causal).
+ * Source: "Attention Variants -- Sliding Window, Sparse, Differential", the
+ * problem statement (two maps from separate Q/K projections, one subtracted
+ * from the other); "Attention Variants Compared", variants table
+ * (Differential: 2 times N squared compute).
+ *   q1, q2 [B,Hq,N,d_qk], k1, k2 [B,Hkv,N,d_qk], v [B,Hkv,N,d_v] bf16;
+ *   o [B,Hq,N,d_v] bf16; lambda: device fp32 [Hq];
+ *   d_qk == 64 (K1 and K2 tiles share one shared-memory slot), d_v in
+ *   {64, 128}; other head dims return SWA_ERR_UNSUPPORTED. */
+swa_status_t diff_attn_fwd(const void* q1, const void* k1, const void* q2, const void* k2,
+                           const void* v, void* o, const float* lambda, int B, int Hq, int Hkv,
+                           int N, int d_qk, int d_v, int W, float scale, void* stream);
+
+/* One decode step over a rolling W-slot KV cache.
+ * Source: "Learn: Sparse & Sliding-Window Attention", section 4 (keep a
+ * rolling window of the most recent w tokens, evict the oldest) and
+ * section 6 (the cache stays O(w)); "Sliding Window Attention" glossary page
+ * (fixed-size KV cache).
+ *   q [B,Hq,d]; k_new, v_new [B,Hkv,d] bf16 (device, read only);
+ *   k_cache, v_cache [B,Hkv,W,d] bf16 (device, updated: slot pos[b] % W of
+ *     sequence b receives k_new/v_new);
+ *   pos: device int32 [B], absolute position (>= 0) of the new token;
+ *   o [B,Hq,d] bf16 (device, written);
+ *   workspace: device scratch of at least swa_decode_workspace_bytes(...)
+ *     bytes, 16-byte aligned; its contents need not be initialised.
+ * The step writes the new token first, then attends over the positions
+ * max(0, pos-W+1) .. pos, which the cache's slots hold in rotated order. */
+swa_status_t swa_decode_step(const void* q, const void* k_new, const void* v_new, void* k_cache,
+                             void* v_cache, const int32_t* pos, void* o, int B, int Hq, int Hkv,
+                             int d, int W, float scale, void* workspace, size_t ws_bytes,
+                             void* stream);
+
+/* Scratch bytes swa_decode_step needs for these sizes (0 on bad sizes). */
+size_t swa_decode_workspace_bytes(int B, int Hq, int Hkv, int d, int W);
+
+/* Prefill with debug outputs. kind 0 = sliding window (stride ignored),
+ * kind 1 = local + strided. Same arithmetic as swa_attn_fwd /
+ * strided_attn_fwd; dbg may be NULL. */
+swa_status_t swa_prefill_debug(int kind, const void* q, const void* k, const void* v, void* o,
+                               float* lse, int B, int Hq, int Hkv, int N, int d, int W,
+                               int stride, float scale, const swa_debug_t* dbg, void* stream);
+
+/* The key tiles each query tile visits, as the kernels enumerate them
+ * (host only; the kernels call the same function). kind 0 = window,
+ * 1 = window + stride, 2 = full causal. Query tiles are Bq rows, key tiles
+ * Bk keys (the kernels use 128 x 128). qtile_offsets [nq + 1] receives the
+ * start of each query tile's list in `tiles`; tiles receives up to cap
+ * entries in the encoding of swa_debug_t. Returns the total number of
+ * entries (which may exceed cap), or -1 on bad arguments. Either output
+ * may be NULL to just count. Source: "Learn: Sparse & Sliding-Window
+ * Attention", section 3 (cost proportional to ||M||_0);
+ * "Attention Variants Compared", glossary (zero blocks skipped in the
+ * kernel). */
+int64_t swa_schedule(int kind, int N, int W, int stride, int Bq, int Bk, int32_t* qtile_offsets,
+                     int32_t* tiles, int64_t cap);
+
+/* ||M||_0, the attended cells of one (b, head) N x N mask, in closed form
+ * (kind as swa_schedule; stride ignored unless kind == 1). -1 on bad
+ * arguments. Source: "Attention Variants Compared", count_nonmasked. */
+int64_t swa_count_nonmasked(int kind, int N, int W, int stride);
+
+/* Synchronises `stream`, then returns and clears the device error flag of
+ * the current device (SWA_OK if no kernel recorded an error). */
+swa_status_t swa_last_device_error(void* stream);
+
+/* A static, human-readable name for a status code. */
+const char* swa_status_string(swa_status_t status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SWA_ATTN_H */

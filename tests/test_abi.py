@@ -1,0 +1,134 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads and
+exports every function include/*.h declares; the schedule export matches the
+oracle's explicit-mask derivation bit for bit; the closed-form attended-cell
+count matches the oracle; bad arguments are rejected before any launch."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+from conftest import ROOT
+
+import differential_attention_swa_b200 as swa
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from differential_attention_swa_b200 import build
+
+    build.build()
+    return swa.library()
+
+
+def declared_functions():
+    names = []
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        for m in re.finditer(r"^\s*[A-Za-z_][\w\s\*]*?\b([a-z_][a-z0-9_]*)\s*\(", text, flags=re.M):
+            if m.group(1) not in ("if", "while", "for", "sizeof", "return"):
+                names.append(m.group(1))
+    return sorted(set(names))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for want in ("swa_attn_fwd", "strided_attn_fwd", "diff_attn_fwd", "swa_decode_step", "swa_schedule",
+                 "swa_count_nonmasked", "swa_last_device_error", "swa_status_string"):
+        assert want in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    out = os.popen(f"nm -D --defined-only {swa.LIB_PATH}").read()
+    for name in declared_functions():
+        assert re.search(rf"\bT {name}\b", out), name
+
+
+@pytest.mark.parametrize("kind,okind,N,W,S", [
+    (0, "swa", 256, 64, 0), (1, "strided", 256, 16, 8), (0, "swa", 1000, 130, 0), (1, "strided", 1000, 1, 1),
+    (1, "strided", 777, 200, 7), (0, "swa", 129, 5000, 0), (1, "strided", 300, 17, 400), (2, "causal", 513, 0, 0),
+    (0, "swa", 1, 1, 0), (1, "strided", 4000, 128, 128)])
+def test_schedule_export_bit_exact_vs_oracle(lib, orc, kind, okind, N, W, S):
+    got = swa.schedule(kind, N, W, S)
+    want, _ = orc.schedule(okind, N, W, S, 128, 128)
+    assert got == want
+
+
+def test_schedule_sampled_at_workload_sizes(lib, orc):
+    for (kind, okind, N, W, S, qts) in [(0, "swa", 8192, 4096, 0, (0, 1, 31, 32, 63)),
+                                        (1, "strided", 16384, 128, 128, (0, 1, 2, 64, 127)),
+                                        (0, "swa", 131072, 1024, 0, (0, 7, 8, 9, 1023))]:
+        got = swa.schedule(kind, N, W, S)
+        for qt in qts:
+            want, _ = orc.schedule_qtile(okind, N, W, S, 128, 128, qt)
+            assert got[qt] == want, (N, qt)
+    assert sum(len(x) for x in swa.schedule(0, 8192, 4096)) == 1584
+    assert sum(len(x) for x in swa.schedule(0, 131072, 1024)) == 9180
+    assert sum(len(x) for x in swa.schedule(1, 16384, 128, 128)) == 382
+
+
+@pytest.mark.parametrize("kind,okind,N,W,S", [
+    (0, "swa", 256, 64, 0), (1, "strided", 256, 16, 8), (1, "strided", 300, 17, 5), (0, "swa", 50, 50, 0),
+    (0, "swa", 50, 1, 0), (1, "strided", 97, 3, 1), (1, "strided", 97, 200, 3), (2, "causal", 70, 0, 0)])
+def test_count_nonmasked_closed_form_vs_oracle(lib, orc, kind, okind, N, W, S):
+    M = orc.mask(okind, N, W, S)
+    assert swa.count_nonmasked(kind, N, W, S) == orc.count_nonmasked(M)
+
+
+def test_count_nonmasked_workloads(lib):
+    assert swa.count_nonmasked(0, 8192, 4096) == 25167872
+    assert swa.count_nonmasked(1, 16384, 128, 128) == 3129408
+    assert swa.count_nonmasked(0, 131072, 1024) == 133693952
+    assert swa.count_nonmasked(0, 4096, 4096) == 8390656
+    assert swa.count_nonmasked(0, 256, 64) == 14368
+    assert swa.count_nonmasked(1, 256, 16, 8) == 7696
+
+
+def test_bad_arguments_rejected_before_launch(lib):
+    P = ctypes.c_void_p
+    good = P(0x10000)  # aligned, never dereferenced: validation fails first
+    nullp = None
+    st = lib.swa_attn_fwd(nullp, good, good, good, None, 1, 2, 2, 256, 64, 64, 0.125, None)
+    assert st == swa.ERR_INVALID_ARG
+    st = lib.swa_attn_fwd(P(0x10008), good, good, good, None, 1, 2, 2, 256, 64, 64, 0.125, None)
+    assert st == swa.ERR_INVALID_ARG  # misaligned
+    st = lib.swa_attn_fwd(good, good, good, good, None, 1, 3, 2, 256, 64, 64, 0.125, None)
+    assert st == swa.ERR_INVALID_ARG  # Hq % Hkv
+    st = lib.swa_attn_fwd(good, good, good, good, None, 1, 2, 2, 256, 64, 0, 0.125, None)
+    assert st == swa.ERR_INVALID_ARG  # W < 1
+    st = lib.swa_attn_fwd(good, good, good, good, None, 1, 2, 2, 0, 64, 4, 0.125, None)
+    assert st == swa.ERR_INVALID_ARG  # N < 1
+    st = lib.swa_attn_fwd(good, good, good, good, None, 1, 2, 2, 256, 64, 4, -1.0, None)
+    assert st == swa.ERR_INVALID_ARG  # scale
+    st = lib.swa_attn_fwd(good, good, good, good, None, 1, 2, 2, 256, 96, 4, 0.1, None)
+    assert st == swa.ERR_UNSUPPORTED  # head dim
+    st = lib.strided_attn_fwd(good, good, good, good, None, 1, 2, 2, 256, 64, 4, 0, 0.1, None)
+    assert st == swa.ERR_INVALID_ARG  # stride < 1
+    st = lib.diff_attn_fwd(good, good, good, good, good, good, None, 1, 2, 2, 64, 64, 128, 64, 0.1, None)
+    assert st == swa.ERR_INVALID_ARG  # lambda missing
+    st = lib.diff_attn_fwd(good, good, good, good, good, good, good, 1, 2, 2, 64, 128, 128, 64, 0.1, None)
+    assert st == swa.ERR_UNSUPPORTED  # d_qk 128 not built for the differential kernel
+    ws = lib.swa_decode_workspace_bytes(64, 16, 8, 128, 1024)
+    assert ws > 0
+    st = lib.swa_decode_step(good, good, good, good, good, good, good, 64, 16, 8, 128, 1024, 0.1, good, ws - 1,
+                             None)
+    assert st == swa.ERR_INVALID_ARG  # workspace too small
+    st = lib.swa_decode_step(good, good, good, good, good, good, good, 2, 6, 2, 128, 16, 0.1, good, 1 << 20,
+                             None)
+    assert st == swa.ERR_UNSUPPORTED  # group size 3
+    assert lib.swa_decode_workspace_bytes(1, 3, 2, 128, 16) == 0
+    assert lib.swa_schedule(0, 0, 4, 0, 128, 128, None, None, 0) == -1
+    assert lib.swa_count_nonmasked(1, 10, 4, 0) == -1
+    assert lib.swa_status_string(swa.ERR_TIMEOUT) == b"in-kernel wait timed out"
+
+
+def test_python_binding_refuses_cpu_tensors(lib):
+    import torch
+
+    q = torch.zeros(1, 2, 8, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        swa.swa_attn_fwd(q, q, q, 4)

@@ -1,0 +1,197 @@
+"""GPU parity: every C-ABI entry point against the fp64 oracle on the same
+seeded bf16 inputs.
+
+Bars: bf16 outputs (fp32 accumulate) within max|diff| <= 1e-2 and
+mean|diff| <= 2e-3 of the fp64 oracle; visited key-tile lists and attended
+cell counts bit-exact against the oracle's explicit-mask derivation."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import differential_attention_swa_b200 as swa
+from differential_attention_swa_b200.inputs import WORKLOADS, attn_inputs, decode_inputs, diff_inputs
+
+pytestmark = pytest.mark.gpu
+
+MAX_TOL = 1e-2
+MEAN_TOL = 2e-3
+KIND = {"swa": swa.MASK_WINDOW, "strided": swa.MASK_STRIDED}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from differential_attention_swa_b200 import build
+
+    build.build()
+    swa.library()
+    assert swa.last_device_error() == swa.OK
+
+
+def gpu(*ts):
+    return [t.cuda() for t in ts]
+
+
+def compare(got, want, what):
+    got = got.float().cpu().numpy().astype(np.float64).reshape(want.shape)
+    diff = np.abs(got - want)
+    assert np.isfinite(got).all(), f"{what}: non-finite output"
+    mx, mean = diff.max(), diff.mean()
+    assert mx <= MAX_TOL and mean <= MEAN_TOL, f"{what}: max {mx:.3e} mean {mean:.3e}"
+    return mx, mean
+
+
+def run_prefill(kind, q, k, v, W, S, lse=False):
+    qd, kd, vd = gpu(q, k, v)
+    if kind == "swa":
+        r = swa.swa_attn_fwd(qd, kd, vd, W, return_lse=lse)
+    else:
+        r = swa.strided_attn_fwd(qd, kd, vd, W, S, return_lse=lse)
+    assert swa.last_device_error() == swa.OK
+    return r
+
+
+# ------------------------------------------------------------ tiny, full --
+
+@pytest.mark.parametrize("name", ["tiny_swa", "tiny_strided"])
+def test_tiny_workloads_full(orc, name):
+    w = WORKLOADS[name]
+    q, k, v = attn_inputs(w.B, w.Hq, w.Hkv, w.N, w.d, seed=0)
+    out, lse = run_prefill(w.kind, q, k, v, w.W, w.S, lse=True)
+    ref, ref_lse = orc.attention(w.kind, q, k, v, W=w.W, S=w.S, scale=w.scale, with_lse=True)
+    compare(out, ref, name)
+    assert np.abs(lse.cpu().numpy() - ref_lse).max() < 2e-3
+
+
+EDGE = [
+    # kind, B, Hq, Hkv, N, d, W, S
+    ("swa", 1, 2, 2, 200, 64, 64, 0),       # ragged tail, odd tile count
+    ("swa", 1, 2, 2, 1, 64, 4, 0),          # a single row
+    ("swa", 1, 1, 1, 127, 64, 1, 0),        # window 1: out = V
+    ("swa", 2, 4, 4, 300, 64, 5000, 0),     # window beyond N: full causal
+    ("swa", 1, 8, 2, 384, 128, 100, 0),     # GQA group 4: head pairs
+    ("swa", 1, 6, 2, 257, 128, 129, 0),     # GQA group 3: tile pairs, ragged
+    ("swa", 2, 4, 2, 640, 128, 256, 0),     # group 2, several tiles
+    ("swa", 1, 2, 1, 130, 64, 128, 0),      # W equal to one tile
+    ("strided", 1, 2, 2, 300, 64, 17, 5),   # N not a multiple of S
+    ("strided", 1, 2, 2, 256, 64, 3, 1),    # stride 1: every key (full causal)
+    ("strided", 1, 2, 2, 333, 64, 20, 400), # stride beyond N: window + key 0
+    ("strided", 1, 4, 2, 1000, 128, 64, 7), # group 2 with stride tiles
+    ("strided", 1, 2, 2, 700, 64, 1, 3),    # window 1 + stride
+]
+
+
+@pytest.mark.parametrize("kind,B,Hq,Hkv,N,d,W,S", EDGE)
+def test_edge_cases_full(orc, kind, B, Hq, Hkv, N, d, W, S):
+    q, k, v = attn_inputs(B, Hq, Hkv, N, d, seed=N + W)
+    out = run_prefill(kind, q, k, v, W, S)
+    ref = orc.attention(kind, q, k, v, W=W, S=S, scale=1 / math.sqrt(d))
+    compare(out, ref, f"{kind} N{N} W{W} S{S}")
+
+
+@pytest.mark.parametrize("kind,N,W,S,Hq,Hkv,d", [
+    ("swa", 256, 64, 0, 2, 2, 64), ("strided", 256, 16, 8, 2, 2, 64), ("swa", 1000, 300, 0, 4, 2, 128),
+    ("strided", 1500, 100, 9, 2, 2, 64), ("swa", 385, 5000, 0, 3, 1, 64), ("strided", 2048, 128, 128, 2, 1, 64)])
+def test_visited_tiles_and_cells_bit_exact(orc, kind, N, W, S, Hq, Hkv, d):
+    q, k, v = attn_inputs(1, Hq, Hkv, N, d, seed=7)
+    qd, kd, vd = gpu(q, k, v)
+    out, cells, tiles, ntiles = swa.prefill_debug(KIND[kind], qd, kd, vd, W, S, tiles_cap=64)
+    assert swa.last_device_error() == swa.OK
+    lists, want_cells = orc.schedule(kind, N, W, S, 128, 128)
+    cells, tiles, ntiles = cells.cpu(), tiles.cpu(), ntiles.cpu()
+    for h in range(Hq):
+        for qt, (lst, c) in enumerate(zip(lists, want_cells)):
+            assert int(ntiles[0, h, qt]) == len(lst), (h, qt)
+            assert tiles[0, h, qt, :len(lst)].tolist() == lst, (h, qt)
+            assert int(cells[0, h, qt]) == c, (h, qt)
+    ref = orc.attention(kind, q, k, v, W=W, S=S, scale=1 / math.sqrt(d))
+    compare(out, ref, "debug path output")
+
+
+def test_timeout_is_reported_and_context_survives(orc):
+    q, k, v = attn_inputs(1, 2, 2, 256, 64, seed=1)
+    qd, kd, vd = gpu(q, k, v)
+    swa.prefill_debug(swa.MASK_WINDOW, qd, kd, vd, 64, inject_timeout=True)
+    assert swa.last_device_error() == swa.ERR_TIMEOUT
+    assert swa.last_device_error() == swa.OK  # cleared
+    out = swa.swa_attn_fwd(qd, kd, vd, 64)
+    assert swa.last_device_error() == swa.OK
+    compare(out, orc.attention("swa", q, k, v, W=64, scale=0.125), "after timeout")
+
+
+# ---------------------------------------------------------- differential --
+
+@pytest.mark.parametrize("N,W,dv,Hq,Hkv", [(256, None, 128, 2, 2), (300, 70, 128, 2, 1), (513, None, 64, 4, 2)])
+def test_diff_small_full(orc, N, W, dv, Hq, Hkv):
+    q1, k1, q2, k2, v = diff_inputs(1, Hq, Hkv, N, 64, dv, seed=3)
+    lam = torch.tensor([0.8, 0.5, 0.2, 1.0][:Hq], dtype=torch.float32)
+    out = swa.diff_attn_fwd(*gpu(q1, k1, q2, k2, v), lam.cuda(), window=W, scale=0.125)
+    assert swa.last_device_error() == swa.OK
+    ref = orc.diff_attention(q1, k1, q2, k2, v, lam, W=W, scale=0.125)
+    compare(out, ref, "diff")
+
+
+# ---------------------------------------------------------------- decode --
+
+@pytest.mark.parametrize("B,Hq,Hkv,d,W,pos0,T", [(2, 4, 2, 128, 64, 3, 70), (3, 16, 8, 128, 1024, 131072, 3),
+                                                  (2, 2, 2, 64, 100, 0, 5), (1, 8, 1, 128, 256, 250, 10)])
+def test_decode_steps_vs_oracle(orc, B, Hq, Hkv, d, W, pos0, T):
+    q, k_new, v_new, k_cache, v_cache = decode_inputs(T, B, Hq, Hkv, d, W, seed=5)
+    pos = np.array([[pos0 + t] * B for t in range(T)], dtype=np.int32)
+    ref, kc_ref, vc_ref = orc.decode(q, k_new, v_new, k_cache, v_cache, pos)
+    kc, vc = gpu(k_cache, v_cache)
+    posd = torch.from_numpy(pos).cuda()
+    qd, knd, vnd = gpu(q, k_new, v_new)
+    outs = []
+    for t in range(T):
+        outs.append(swa.swa_decode_step(qd[t], knd[t], vnd[t], kc, vc, posd[t]))
+    assert swa.last_device_error() == swa.OK
+    compare(torch.stack(outs), ref, "decode")
+    assert np.array_equal(kc.float().cpu().numpy(), kc_ref)
+    assert np.array_equal(vc.float().cpu().numpy(), vc_ref)
+
+
+# ------------------------------------------------------ workload sizes ----
+
+def sampled_rows(B, H, N, n, seed):
+    rng = np.random.default_rng(seed)
+    i = np.concatenate([rng.integers(0, N, n), [0, 1, 127, 128, N - 1, N - 2]])
+    bh = rng.integers(0, B * H, i.size)
+    return np.unique(bh.astype(np.int64) * N + i)
+
+
+@pytest.mark.parametrize("name", ["mistral_swa_prefill", "local_strided_prefill", "gemma_swa_prefill"])
+def test_workload_sampled_rows(orc, name):
+    w = WORKLOADS[name]
+    q, k, v = attn_inputs(w.B, w.Hq, w.Hkv, w.N, w.d, seed=0)
+    out = run_prefill(w.kind, q, k, v, w.W, w.S).reshape(-1, w.d)
+    rows = sampled_rows(w.B, w.Hq, w.N, 1500, 1)
+    ref = orc.attention(w.kind, q, k, v, W=w.W, S=w.S, scale=w.scale, rows=rows)
+    compare(out[torch.from_numpy(rows).cuda()], ref, name)
+    assert torch.isfinite(out.float()).all()
+
+
+def test_diff_workload_sampled_rows(orc):
+    w = WORKLOADS["diff_causal"]
+    q1, k1, q2, k2, v = diff_inputs(w.B, w.Hq, w.Hkv, w.N, w.d, w.dv, seed=0)
+    lam = torch.full((w.Hq,), w.lam, dtype=torch.float32)
+    out = swa.diff_attn_fwd(*gpu(q1, k1, q2, k2, v), lam.cuda(), window=w.W, scale=w.scale)
+    assert swa.last_device_error() == swa.OK
+    rows = sampled_rows(w.B, w.Hq, w.N, 1500, 2)
+    ref = orc.diff_attention(q1, k1, q2, k2, v, lam, W=w.W, scale=w.scale, rows=rows)
+    compare(out.reshape(-1, w.dv)[torch.from_numpy(rows).cuda()], ref, "diff workload")
+
+
+def test_decode_workload_first_steps(orc):
+    w = WORKLOADS["gemma_swa_decode"]
+    T = 3
+    q, k_new, v_new, k_cache, v_cache = decode_inputs(T, w.B, w.Hq, w.Hkv, w.d, w.W, seed=0)
+    pos = np.array([[w.pos0 + t] * w.B for t in range(T)], dtype=np.int32)
+    ref, _, _ = orc.decode(q, k_new, v_new, k_cache, v_cache, pos)
+    kc, vc = gpu(k_cache, v_cache)
+    posd = torch.from_numpy(pos).cuda()
+    qd, knd, vnd = gpu(q, k_new, v_new)
+    outs = [swa.swa_decode_step(qd[t], knd[t], vnd[t], kc, vc, posd[t]) for t in range(T)]
+    assert swa.last_device_error() == swa.OK
+    compare(torch.stack(outs), ref, "decode workload")
