@@ -153,7 +153,9 @@ def tiled_softmax_dot(q, K, V, mask_row_, scale: float, tile: int = 4) -> np.nda
 def _rows_arg(rows, total):
     if rows is None:
         return None, total
-    r = np.ascontiguousarray(rows, dtype=np.int64)
+    r = np.ascontiguousarray(rows, dtype=np.int64).reshape(-1)
+    if r.size and (r.min() < 0 or r.max() >= total):
+        raise ValueError(f"row ids must lie in [0, {total})")
     return r, r.size
 
 

@@ -207,6 +207,8 @@ def test_attention_row_subset_matches_full(orc):
     rows = np.array([0, 5, 89, 90, 179, 4 * 90 + 33, 8 * 90 - 1])
     part = orc.attention("strided", q, k, v, W=10, S=7, rows=rows)
     assert np.array_equal(part, full.reshape(-1, 16)[rows])
+    with pytest.raises(ValueError):
+        orc.attention("strided", q, k, v, W=10, S=7, rows=[2 * 4 * 90])
 
 
 # ------------------------------------------------------------ differential --
