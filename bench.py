@@ -94,6 +94,17 @@ def aggregate(per_rank_ms, units_per_rank):
     return n * units_per_rank / (t * 1e-3), t
 
 
+def max_over_ranks(ms: float, dist, device="cpu") -> float:
+    """The slowest rank's time (every rank takes part in the same all-reduce)."""
+    if dist is None:
+        return ms
+    import torch
+
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def shard_seed(base: int, rank: int) -> int:
     """Each rank draws its own batch (weak scaling over data)."""
     return base + 1000 * rank
@@ -274,11 +285,7 @@ def measure_ours(args, rank, world, peaks, peak_src, dist):
     if err != swa.OK:
         raise RuntimeError(f"kernel reported status {err}")
     mean_ms = sum(ms) / len(ms)
-    t_all = [mean_ms]
-    if dist:
-        t = torch.tensor([mean_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        t_all = [t.item()] * world
+    t_all = [max_over_ranks(mean_ms, dist, "cuda")] * world
     value, tmax = aggregate(t_all, flops)
     achieved = flops / (mean_ms * 1e-3) / 1e12
     peak = peaks["bf16_tflops"]
