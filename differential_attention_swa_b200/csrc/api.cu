@@ -246,6 +246,7 @@ const char* swa_status_string(swa_status_t s) {
     case SWA_ERR_UNSUPPORTED: return "unsupported head dimension or group size";
     case SWA_ERR_CUDA: return "CUDA error";
     case SWA_ERR_TIMEOUT: return "in-kernel wait timed out";
+    case SWA_ERR_SCRATCH_TOO_SMALL: return "sizes need more scratch than the static decode array holds";
   }
   return "unknown status";
 }

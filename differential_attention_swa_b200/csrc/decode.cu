@@ -20,8 +20,12 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <cmath>
 #include <cstdint>
+#include <cstring>
+#include <mutex>
 
+#include "../../include/swa_attn.h"
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -282,3 +286,65 @@ cudaError_t launch_decode(const DecodeParams& p0, cudaStream_t stream) {
 }
 
 }  // namespace swa
+
+// ---------------------------------------------------------------------------
+// Decode without a caller-provided workspace.
+//
+// Some callers cannot allocate device memory at all: a plugin host that hands
+// a library raw tensors but no allocator, or a serving loop that forbids
+// allocation on its hot path. For them the split partials live in one fixed
+// array compiled into this library. Every GPU that loads the library holds
+// these bytes until the process exits, and every call shares them.
+
+namespace swa {
+
+constexpr size_t kStaticDecodeScratchBytes = 4u << 20;  // SWA_DECODE_STATIC_SCRATCH_BYTES
+static_assert(kStaticDecodeScratchBytes == SWA_DECODE_STATIC_SCRATCH_BYTES, "header and library disagree");
+
+static __device__ __align__(256) unsigned char g_decode_scratch[kStaticDecodeScratchBytes];
+
+// In host code `g_decode_scratch` names a host-side stand-in, not device
+// memory, so the kernels receive the array's device address instead. It is
+// looked up once per device, with that device current, on the first call.
+static float* static_decode_scratch() {
+  static float* ptrs[64] = {nullptr};
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (ptrs[dev] == nullptr) {
+    void* a = nullptr;
+    if (cudaGetSymbolAddress(&a, g_decode_scratch) != cudaSuccess) return nullptr;
+    ptrs[dev] = static_cast<float*>(a);
+  }
+  return ptrs[dev];
+}
+
+}  // namespace swa
+
+extern "C" swa_status_t swa_decode_step_static(const void* q, const void* k_new, const void* v_new, void* k_cache,
+                                               void* v_cache, const int32_t* pos, void* o, int B, int Hq, int Hkv,
+                                               int d, int W, float scale, void* stream) {
+  using namespace swa;
+  auto a16 = [](const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
+  if (!a16(q) || !a16(k_new) || !a16(v_new) || !a16(k_cache) || !a16(v_cache) || !a16(o) || pos == nullptr ||
+      (reinterpret_cast<uintptr_t>(pos) & 3u))
+    return SWA_ERR_INVALID_ARG;
+  if (B < 1 || Hq < 1 || Hkv < 1 || W < 1 || Hq % Hkv != 0) return SWA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !isfinite(scale)) return SWA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return SWA_ERR_UNSUPPORTED;
+  const int G = Hq / Hkv;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return SWA_ERR_UNSUPPORTED;
+  if (decode_partial_bytes(B, Hq, Hkv, d, W) > kStaticDecodeScratchBytes) return SWA_ERR_SCRATCH_TOO_SMALL;
+  float* scratch = static_decode_scratch();
+  if (scratch == nullptr) return SWA_ERR_CUDA;
+  // Each split writes its whole record before the combine reads it, so the
+  // array needs no clearing between calls.
+  DecodeParams p;
+  memset(&p, 0, sizeof(p));
+  p.q = q; p.k_new = k_new; p.v_new = v_new; p.k_cache = k_cache; p.v_cache = v_cache; p.pos = pos; p.o = o;
+  p.partial = scratch;
+  p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.d = d; p.W = W; p.G = G;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  return launch_decode(p, static_cast<cudaStream_t>(stream)) == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
+}

@@ -42,7 +42,9 @@ typedef enum {
   SWA_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size or ratio  */
   SWA_ERR_UNSUPPORTED = 2, /* valid but not built: head dim outside {64,128} */
   SWA_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed           */
-  SWA_ERR_TIMEOUT = 4      /* a bounded in-kernel wait ran out            */
+  SWA_ERR_TIMEOUT = 4,     /* a bounded in-kernel wait ran out            */
+  SWA_ERR_SCRATCH_TOO_SMALL = 5 /* sizes need more scratch than the library's
+                                   static decode array holds               */
 } swa_status_t;
 
 /* Optional device-side debug outputs of the prefill kernels (pass NULL to
@@ -126,6 +128,31 @@ swa_status_t swa_decode_step(const void* q, const void* k_new, const void* v_new
 
 /* Scratch bytes swa_decode_step needs for these sizes (0 on bad sizes). */
 size_t swa_decode_workspace_bytes(int B, int Hq, int Hkv, int d, int W);
+
+/* Bytes of the scratch array compiled into the library for
+ * swa_decode_step_static (on every GPU that loads the library). */
+#define SWA_DECODE_STATIC_SCRATCH_BYTES (4u << 20)
+
+/* swa_decode_step for callers that cannot allocate device memory. The pages
+ * have no counterpart: this is a convenience of this library's ABI.
+ * Some callers cannot hand over a workspace: a plugin host that gives a
+ * library tensors but no allocator, or a serving loop whose hot path may not
+ * allocate. This entry point allocates nothing; its scratch (the per-split
+ * partial results) is a fixed array of SWA_DECODE_STATIC_SCRATCH_BYTES inside
+ * the library, which every GPU that loads the library holds until the process
+ * exits. Arguments, layout and results are those of swa_decode_step, minus
+ * the workspace. Sizes whose scratch (swa_decode_workspace_bytes) exceeds the
+ * array return SWA_ERR_SCRATCH_TOO_SMALL before anything is launched.
+ * The first call on a device looks up the array's device address (once per
+ * device, with that device current); make that first call before any stream
+ * capture. Every call shares the one array, which keeps the last call's
+ * contents (nothing in it needs to start at zero): calls whose work overlaps
+ * on the GPU -- on different streams, or from different threads -- race on
+ * it and must be serialised by the caller. */
+swa_status_t swa_decode_step_static(const void* q, const void* k_new, const void* v_new,
+                                    void* k_cache, void* v_cache, const int32_t* pos, void* o,
+                                    int B, int Hq, int Hkv, int d, int W, float scale,
+                                    void* stream);
 
 /* Prefill with debug outputs. kind 0 = sliding window (stride ignored),
  * kind 1 = local + strided. Same arithmetic as swa_attn_fwd /
