@@ -18,11 +18,15 @@
 // Warp roles (384 threads):
 //   warp 0      TMA producer: Q once, then K and V tiles through a ring of
 //               shared-memory slots.
-//   warp 1      TMEM owner and MMA issuer (one thread): S_t = Q_t K^T into
-//               TMEM, then O_t += P_t V once softmax t has written P_t.
+//   warp 1      TMEM owner and MMA issuer (one thread). Per key tile and
+//               sub: O_t += P_t(prev) V(prev) (A operand read from TMEM),
+//               then S_t = Q_t K^T into the same TMEM columns that held P_t;
+//               the tensor core runs MMAs in issue order, so P is read
+//               before S overwrites it, and the commit that signals S_t also
+//               covers the PV before it.
 //   warps 4-7   softmax of sub 0, warps 8-11 softmax of sub 1: one thread
 //               per query row (TMEM lane), fp32 online softmax in the log2
-//               domain, P as bf16 into shared memory (128-byte swizzle),
+//               domain, P as bf16 back into TMEM over the consumed scores,
 //               lazy rescaling of O, then the epilogue O / l -> bf16.
 // Every wait is bounded; on a timeout the CTA records SWA_ERR_TIMEOUT,
 // drains what it has in flight, frees TMEM and returns.
@@ -41,7 +45,6 @@ namespace swa {
 constexpr int BM = 128;  // query rows per sub (TMEM lanes)
 constexpr int BN = 128;  // keys per tile (S columns)
 constexpr int kThreads = 384;
-constexpr float kLog2e = 1.4426950408889634f;
 // Lazy rescale threshold (log2 units): O and l keep a stale row max until a
 // new score exceeds it by more than this, so P stays below 2^8.
 constexpr float kRescaleTau = 8.0f;
@@ -52,14 +55,12 @@ struct PrefillCfg {
   static constexpr int kKBytes = BN * DQK * 2 * (DIFF ? 2 : 1);
   static constexpr int kVBytes = BN * DV * 2;
   static constexpr int kSlot = kKBytes > kVBytes ? kKBytes : kVBytes;
-  static constexpr int kPBytes = BM * BN * 2;
-  static constexpr int kTiles = 2 * kQBytes + 2 * kPBytes;
+  static constexpr int kTiles = 2 * kQBytes;
   static constexpr int kBudget = 227 * 1024 - 1024 - 1024;  // minus alignment slack and barriers
   static constexpr int kSlotsRaw = (kBudget - kTiles) / kSlot;
   static constexpr int kSlots = kSlotsRaw > 8 ? 8 : kSlotsRaw;
   static_assert(kSlots >= 2, "shared memory too small for the K/V ring");
   static constexpr int kOffQ = 0;
-  static constexpr int kOffP = 2 * kQBytes;
   static constexpr int kOffSlots = kTiles;
   static constexpr int kOffBar = kTiles + kSlots * kSlot;
   static constexpr int kSmemBytes = kOffBar + 1024 + 1024;  // barriers area + alignment slack
@@ -303,8 +304,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t idesc_s = idesc_bf16_f32(BM, BN, false);
       const uint32_t idesc_pv = idesc_bf16_f32(BM, DV, true);
       const int zq = un.b * p.Hq;
-      int kcount[2] = {0, 0};
-      int pending_v[2] = {-1, -1};  // V slot of the item whose PV is still to issue
+      const int ntot[2] = {un.valid[0] ? qtile_nkeys(it.k[0]) : 0, un.valid[1] ? qtile_nkeys(it.k[1]) : 0};
+      int kcount[2] = {0, 0};   // S tiles issued per sub
+      int pv_done[2] = {0, 0};  // PV products issued per sub
+      bool pending[2] = {false, false};  // sub has a PV for the previous item to issue
       int64_t dbg_row[2] = {-1, -1};
       for (int t = 0; t < 2; ++t)
         if (un.valid[t] && p.dbg_tiles && !(DIFF && t == 1))
@@ -313,21 +316,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) record_timeout(abort_flag, p.err_flag);
       tc_fence_after();
       int L = 0;
-      int prev_vslot = -1;
-      auto issue_pv = [&](int t) -> bool {
-        const int vslot = pending_v[t];
-        const uint32_t vb = sbase + C::kOffSlots + vslot * C::kSlot;
-        const uint32_t pb = sbase + C::kOffP + t * C::kPBytes;
+      int prev_vslot = -1, prev_vuse = 0;
+      // O_t += P_t V(prev): P_t is the bf16 tile softmax t wrote over the
+      // first 64 columns of S_t (two keys per column)
+      auto issue_pv = [&](int t) {
+        const uint32_t vb = sbase + C::kOffSlots + prev_vslot * C::kSlot;
+        const uint32_t a0 = tmem + t * BN;
         const uint32_t dcol = tmem + (t == 0 ? C::kOCol0 : C::kOCol1);
-        const int first = (kcount[t] == 1);  // this PV is the sub's first
+        const bool first = (pv_done[t] == 0);
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint64_t a = sw128_desc(pb + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-          const uint64_t b = sw128_desc(vb + kk * 2048, 16384, 1024);
-          umma_bf16_ss(dcol, a, b, idesc_pv, (first && kk == 0) ? 0u : 1u);
-        }
-        umma_commit(bar(BarLayout::kO + t));
-        pending_v[t] = -1;
+        for (int kk = 0; kk < BN / 16; ++kk)
+          umma_bf16_ts(dcol, a0 + kk * 8, sw128_desc(vb + kk * 2048, 16384, 1024), idesc_pv,
+                       (first && kk == 0) ? 0u : 1u);
+        ++pv_done[t];
+        if (pv_done[t] == ntot[t]) umma_commit(bar(BarLayout::kO + t));
+        pending[t] = false;
+      };
+      auto wait_prev_v = [&]() -> bool {
+        if (!mbar_wait(bar(BarLayout::kFull + prev_vslot), prev_vuse & 1, abort_flag)) return false;
+        tc_fence_after();
         return true;
       };
       for (int u = 0; u < it.n && ok; ++u) {
@@ -341,16 +348,25 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc_fence_after();
+        bool v_ready = false;
         for (int t = 0; t < 2 && ok; ++t) {
           const bool in = item_in_sub(it, t, u);
-          if (!in && pending_v[t] < 0) continue;
-          if (kcount[t] > 0) {
+          if (!in && !pending[t]) continue;
+          if (kcount[t] > 0) {  // softmax t has consumed S_t and written P_t
             if (!mbar_wait(bar(BarLayout::kP + t), (kcount[t] - 1) & 1, abort_flag)) {
               record_timeout(abort_flag, p.err_flag);
               ok = false;
               break;
             }
             tc_fence_after();
+          }
+          if (pending[t]) {
+            if (!v_ready && !(v_ready = wait_prev_v())) {
+              record_timeout(abort_flag, p.err_flag);
+              ok = false;
+              break;
+            }
+            issue_pv(t);
           }
           if (in) {
             const uint32_t qb = sbase + C::kOffQ + t * C::kQBytes;
@@ -366,27 +382,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (dbg_row[t] >= 0 && kcount[t] < p.dbg_cap)
               p.dbg_tiles[dbg_row[t] * p.dbg_cap + kcount[t]] =
                   item_is_stride(it, u) ? (kStrideTag | item_tile(it, u)) : item_tile(it, u);
+            ++kcount[t];
           }
-          if (pending_v[t] >= 0) issue_pv(t);
-          if (in) ++kcount[t];
         }
         if (!ok) break;
-        umma_commit(bar(BarLayout::kEmpty + kslot));
-        if (prev_vslot >= 0) umma_commit(bar(BarLayout::kEmpty + prev_vslot));
-        // V of this item must be resident before its PVs (issued next round)
-        if (!mbar_wait(bar(BarLayout::kFull + vslot), vuse & 1, abort_flag)) {
-          record_timeout(abort_flag, p.err_flag);
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        for (int t = 0; t < 2; ++t)
-          if (item_in_sub(it, t, u)) pending_v[t] = vslot;
+        umma_commit(bar(BarLayout::kEmpty + kslot));                    // K(u) read by this step's S
+        if (prev_vslot >= 0) umma_commit(bar(BarLayout::kEmpty + prev_vslot));  // V(u-1) by its PVs
+        for (int t = 0; t < 2; ++t) pending[t] = item_in_sub(it, t, u);
         prev_vslot = vslot;
+        prev_vuse = vuse;
       }
+      bool v_ready = false;
       for (int t = 0; t < 2 && ok; ++t) {
-        if (pending_v[t] < 0) continue;
-        if (!mbar_wait(bar(BarLayout::kP + t), (kcount[t] - 1) & 1, abort_flag)) {
+        if (!pending[t]) continue;
+        if (!mbar_wait(bar(BarLayout::kP + t), (kcount[t] - 1) & 1, abort_flag) ||
+            (!v_ready && !(v_ready = wait_prev_v()))) {
           record_timeout(abort_flag, p.err_flag);
           ok = false;
           break;
@@ -409,7 +419,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_addr = static_cast<uint32_t>(qw * 32) << 16;
     const uint32_t s_tmem = tmem + lane_addr + t * BN;
     const uint32_t o_tmem = tmem + lane_addr + (t == 0 ? C::kOCol0 : C::kOCol1);
-    const uint32_t pbase = sbase + C::kOffP + t * C::kPBytes;
     const bool valid_sub = un.valid[t] != 0;
     const int i = un.qt[t] * BM + r;                 // query index
     const bool row_ok = valid_sub && i < p.N;
@@ -446,22 +455,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
 
         float s[BN];
-        tmem_ld64(s_tmem, s);
-        tmem_ld64(s_tmem + 64, s + 64);
+        tmem_ld128(s_tmem, s);
         if (!__all_sync(0xffffffffu, full)) {
 #pragma unroll
           for (int c = 0; c < BN; ++c)
             if (c < c0 || c > c1) s[c] = -INFINITY;
         }
-        float mx = -INFINITY;
+        // row max over 8 independent chains
+        float mx8[8];
 #pragma unroll
-        for (int c = 0; c < BN; ++c) mx = fmaxf(mx, s[c]);
+        for (int j = 0; j < 8; ++j) mx8[j] = s[j];
+#pragma unroll
+        for (int c = 8; c < BN; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], s[c]);
+        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
         const float m_tile = mx * cl2;  // -inf stays -inf
         float m_use = m_run, alpha = 1.f;
         bool rescale = false;
         if (m_tile > m_run) {
           if (m_run == -INFINITY) {
-            m_use = m_tile;  // nothing accumulated yet: O row is 0 (or not written)
+            m_use = m_tile;  // nothing accumulated yet: the O row is 0 (or not yet written)
             alpha = 0.f;
           } else if (m_tile - m_run > kRescaleTau) {
             m_use = m_tile;
@@ -470,43 +483,37 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         const float msub = (m_use == -INFINITY) ? 0.f : m_use;
-        float rs = 0.f;
+        float rs8[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) rs8[j] = 0.f;
         uint32_t pk[BN / 2];
 #pragma unroll
         for (int c = 0; c < BN; c += 2) {
           const float p0 = ex2_approx(fmaf(s[c], cl2, -msub));
           const float p1 = ex2_approx(fmaf(s[c + 1], cl2, -msub));
-          rs += p0 + p1;
+          rs8[(c >> 1) & 7] += p0 + p1;
           pk[c / 2] = pack_bf16(p0, p1);
         }
+        const float rs = ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
         l_run = l_run * alpha + rs;
         m_run = m_use;
 
-        if (k > 0) {
-          const bool go = mbar_wait(bar(BarLayout::kO + t), (k - 1) & 1, abort_flag);
-          if (!__all_sync(0xffffffffu, go)) { if (lane == 0) record_timeout(abort_flag, p.err_flag); ok = false; break; }
-          tc_fence_after();
-          if (__any_sync(0xffffffffu, rescale)) {
-            const float f = rescale ? alpha : 1.f;
+        // P over the consumed scores: bf16 pairs in the first 64 columns of S_t
+        tmem_st32_u(s_tmem, pk);
+        tmem_st32_u(s_tmem + 32, pk + 32);
+        // the S_t commit also covered PV_t of the previous tile, so O_t is
+        // complete here and may be rescaled before PV_t of this tile
+        if (k > 0 && __any_sync(0xffffffffu, rescale)) {
+          const float f = rescale ? alpha : 1.f;
 #pragma unroll 1
-            for (int c = 0; c < DV; c += 32) {
-              float o[32];
-              tmem_ld32(o_tmem + c, o);
+          for (int c = 0; c < DV; c += 32) {
+            float o[32];
+            tmem_ld32(o_tmem + c, o);
 #pragma unroll
-              for (int e = 0; e < 32; ++e) o[e] *= f;
-              tmem_st32(o_tmem + c, o);
-            }
+            for (int e = 0; e < 32; ++e) o[e] *= f;
+            tmem_st32(o_tmem + c, o);
           }
         }
-        // P row -> shared memory, 128-byte swizzle (16-byte chunk j of row r
-        // goes to chunk j ^ (r & 7) of the row's 128-byte line)
-#pragma unroll
-        for (int j = 0; j < BN / 8; ++j) {
-          const uint32_t box = j >> 3, cb = j & 7;
-          const uint32_t addr = pbase + box * 16384 + r * 128 + ((cb ^ (r & 7)) << 4);
-          st_shared_v4(addr, pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
-        }
-        fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(bar(BarLayout::kP + t));
         ++k;
@@ -515,7 +522,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // ---------------------------------------------------- epilogue ---
     if (ok && valid_sub && k > 0) {
-      const bool got = mbar_wait(bar(BarLayout::kO + t), (k - 1) & 1, abort_flag);
+      const bool got = mbar_wait(bar(BarLayout::kO + t), 0, abort_flag);  // the sub's last PV
       ok = __all_sync(0xffffffffu, got);
       if (!ok && lane == 0) record_timeout(abort_flag, p.err_flag);
     }
@@ -528,7 +535,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           f2s[r] = (l_run > 0.f) ? p.lambda[hq] / l_run : 0.f;
           mbar_arrive(bar(BarLayout::kX));
         } else {
-          const bool g1 = mbar_wait(bar(BarLayout::kO + 1), (k - 1) & 1, abort_flag);
+          const bool g1 = mbar_wait(bar(BarLayout::kO + 1), 0, abort_flag);
           const bool g2 = mbar_wait(bar(BarLayout::kX), 0, abort_flag);
           if (!__all_sync(0xffffffffu, g1 && g2)) {
             if (lane == 0) record_timeout(abort_flag, p.err_flag);
