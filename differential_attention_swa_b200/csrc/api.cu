@@ -49,6 +49,19 @@ bool encode_rows(CUtensorMap* m, const void* base, int d, int64_t rows, int64_t 
   return r == CUDA_SUCCESS;
 }
 
+// Streaming multiprocessors of the current device (cached per device).
+int sm_count() {
+  static int counts[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return -1;
+  if (counts[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+    counts[dev] = n;
+  }
+  return counts[dev];
+}
+
 bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 bool head_dim_ok(int d) { return d == 64 || d == 128; }
@@ -115,6 +128,9 @@ swa_status_t run_prefill(int kind, bool diff, const void* q, const void* k, cons
     nunits = nB * Hq * ((p.nq + 1) / 2);
   }
   if (nunits > 0x7fffffff) return SWA_ERR_INVALID_ARG;
+  p.nunits = (int)nunits;
+  p.num_ctas = sm_count();
+  if (p.num_ctas <= 0) return SWA_ERR_CUDA;
   p.err_flag = device_error_ptr();
   if (p.err_flag == nullptr) return SWA_ERR_CUDA;
   cudaError_t e = launch_prefill(maps, p, dqk, dv, diff, (int)nunits, static_cast<cudaStream_t>(stream));

@@ -23,6 +23,8 @@ struct PrefillParams {
   int kind;  // MaskKind
   int mode;  // UnitMode
   int nq;    // query tiles of 128 rows
+  int nunits;    // work units of two subs
+  int num_ctas;  // persistent CTAs (one per SM)
   float scale_log2;  // scale * log2(e)
   void* o;
   float* lse;

@@ -73,6 +73,8 @@ struct PrefillCfg {
 // Barrier block layout (8-byte mbarriers, then a few words).
 struct BarLayout {
   static constexpr int kQ = 0;
+  static constexpr int kQEmpty = 25;    // every S MMA of the unit done: Q may be replaced
+  static constexpr int kOFree = 26;     // + sub: epilogue done reading O_t
   static constexpr int kFull = 1;       // + slot
   static constexpr int kEmpty = 9;      // + slot
   static constexpr int kS = 17;         // + sub
@@ -80,7 +82,7 @@ struct BarLayout {
   static constexpr int kO = 21;         // + sub
   static constexpr int kX = 23;         // differential hand-off of 1/l2
   static constexpr int kFinal = 24;     // MMA drain on abort
-  static constexpr int kCount = 25;
+  static constexpr int kCount = 28;
   static constexpr int kWordsOff = 256; // bytes: tmem base, abort flag
   static constexpr int kF2Off = 512;    // bytes: 128 floats
 };
@@ -192,12 +194,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-
-  const Unit un = decode_unit(p, blockIdx.x);
-  const Items it = unit_items(p, un);
+  // persistent CTAs: round r gives CTA c unit r*P + c (r even) or
+  // r*P + P-1-c (r odd). Units come heaviest first, so the alternating
+  // direction evens out the per-CTA totals.
+  const int nunits = p.nunits, P = gridDim.x, c_id = blockIdx.x;
+  auto unit_of = [&](int rnd) -> int { return rnd * P + ((rnd & 1) ? (P - 1 - c_id) : c_id); };
 
   if (threadIdx.x == 0) {
     mbar_init(bar(BarLayout::kQ), 1);
+    mbar_init(bar(BarLayout::kQEmpty), 1);
     for (int s = 0; s < C::kSlots; ++s) {
       mbar_init(bar(BarLayout::kFull + s), 1);
       mbar_init(bar(BarLayout::kEmpty + s), 1);
@@ -206,6 +211,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(BarLayout::kS + t), 1);
       mbar_init(bar(BarLayout::kP + t), 128);
       mbar_init(bar(BarLayout::kO + t), 1);
+      mbar_init(bar(BarLayout::kOFree + t), 128);
     }
     mbar_init(bar(BarLayout::kX), 128);
     mbar_init(bar(BarLayout::kFinal), 1);
@@ -235,67 +241,78 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_prefetch_map(&tm_ks);
         tma_prefetch_map(&tm_vs);
       }
-      const int nvalid = un.valid[0] + un.valid[1];
-      mbar_arrive_expect_tx(bar(BarLayout::kQ), nvalid * C::kQBytes);
-      for (int t = 0; t < 2; ++t) {
-        if (!un.valid[t]) continue;
-        const CUtensorMap* m = (DIFF && t == 1) ? &tm_q2 : &tm_q;
-        for (int bx = 0; bx < DQK / 64; ++bx)
-          tma_load_3d(sbase + C::kOffQ + t * C::kQBytes + bx * 16384, m, bar(BarLayout::kQ), bx * 64,
-                      un.qt[t] * BM, un.b * p.Hq + un.hq[t]);
-      }
-      const int zkv = un.b * p.Hkv + un.hkv;
-      int L = 0;
+      int L = 0;      // K/V loads issued, across units
+      int nq_ld = 0;  // Q loads issued (one per unit)
       int issued[8];
       for (int s = 0; s < 8; ++s) issued[s] = 0;
       bool ok = true;
-      for (int u = 0; u < it.n && ok; ++u) {
-        const bool st = item_is_stride(it, u);
-        const int row = item_tile(it, u) * BN;
-        // K (or K1 and K2)
-        {
-          const int slot = L % C::kSlots, use = L / C::kSlots;
-          ++L;
-          if (use > 0 && !mbar_wait(bar(BarLayout::kEmpty + slot), (use - 1) & 1, abort_flag)) {
-            record_timeout(abort_flag, p.err_flag);
-            ok = false;
-            break;
-          }
-          if (!(p.inject_timeout && blockIdx.x == 0 && u == 0)) {
-            mbar_arrive_expect_tx(bar(BarLayout::kFull + slot), C::kKBytes);
-            const uint32_t dst = sbase + C::kOffSlots + slot * C::kSlot;
-            const CUtensorMap* m = st ? &tm_ks : &tm_k;
-            for (int bx = 0; bx < DQK / 64; ++bx)
-              tma_load_3d(dst + bx * 16384, m, bar(BarLayout::kFull + slot), bx * 64, row, zkv);
-            if (DIFF)
+      for (int rnd = 0; rnd * P < nunits && ok; ++rnd) {
+        const int ui = unit_of(rnd);
+        if (ui >= nunits) continue;
+        const Unit un = decode_unit(p, ui);
+        const Items it = unit_items(p, un);
+        // Q of this unit once every S MMA of the previous unit is done
+        if (nq_ld > 0 && !mbar_wait(bar(BarLayout::kQEmpty), (nq_ld - 1) & 1, abort_flag)) {
+          record_timeout(abort_flag, p.err_flag);
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(bar(BarLayout::kQ), (un.valid[0] + un.valid[1]) * C::kQBytes);
+        for (int t = 0; t < 2; ++t) {
+          if (!un.valid[t]) continue;
+          const CUtensorMap* m = (DIFF && t == 1) ? &tm_q2 : &tm_q;
+          for (int bx = 0; bx < DQK / 64; ++bx)
+            tma_load_3d(sbase + C::kOffQ + t * C::kQBytes + bx * 16384, m, bar(BarLayout::kQ), bx * 64,
+                        un.qt[t] * BM, un.b * p.Hq + un.hq[t]);
+        }
+        ++nq_ld;
+        const int zkv = un.b * p.Hkv + un.hkv;
+        for (int u = 0; u < it.n && ok; ++u) {
+          const bool st = item_is_stride(it, u);
+          const int row = item_tile(it, u) * BN;
+          {  // K (or K1 and K2)
+            const int slot = L % C::kSlots, use = L / C::kSlots;
+            ++L;
+            if (use > 0 && !mbar_wait(bar(BarLayout::kEmpty + slot), (use - 1) & 1, abort_flag)) {
+              record_timeout(abort_flag, p.err_flag);
+              ok = false;
+              break;
+            }
+            if (!(p.inject_timeout && ui == 0 && u == 0)) {
+              mbar_arrive_expect_tx(bar(BarLayout::kFull + slot), C::kKBytes);
+              const uint32_t dst = sbase + C::kOffSlots + slot * C::kSlot;
+              const CUtensorMap* m = st ? &tm_ks : &tm_k;
               for (int bx = 0; bx < DQK / 64; ++bx)
-                tma_load_3d(dst + BN * DQK * 2 + bx * 16384, &tm_k2, bar(BarLayout::kFull + slot),
-                            bx * 64, row, zkv);
+                tma_load_3d(dst + bx * 16384, m, bar(BarLayout::kFull + slot), bx * 64, row, zkv);
+              if (DIFF)
+                for (int bx = 0; bx < DQK / 64; ++bx)
+                  tma_load_3d(dst + BN * DQK * 2 + bx * 16384, &tm_k2, bar(BarLayout::kFull + slot), bx * 64,
+                              row, zkv);
+              issued[slot] = use + 1;
+            }
+          }
+          {  // V
+            const int slot = L % C::kSlots, use = L / C::kSlots;
+            ++L;
+            if (use > 0 && !mbar_wait(bar(BarLayout::kEmpty + slot), (use - 1) & 1, abort_flag)) {
+              record_timeout(abort_flag, p.err_flag);
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(bar(BarLayout::kFull + slot), C::kVBytes);
+            const uint32_t dst = sbase + C::kOffSlots + slot * C::kSlot;
+            const CUtensorMap* m = st ? &tm_vs : &tm_v;
+            for (int bx = 0; bx < DV / 64; ++bx)
+              tma_load_3d(dst + bx * 16384, m, bar(BarLayout::kFull + slot), bx * 64, row, zkv);
             issued[slot] = use + 1;
           }
-        }
-        // V
-        {
-          const int slot = L % C::kSlots, use = L / C::kSlots;
-          ++L;
-          if (use > 0 && !mbar_wait(bar(BarLayout::kEmpty + slot), (use - 1) & 1, abort_flag)) {
-            record_timeout(abort_flag, p.err_flag);
-            ok = false;
-            break;
-          }
-          mbar_arrive_expect_tx(bar(BarLayout::kFull + slot), C::kVBytes);
-          const uint32_t dst = sbase + C::kOffSlots + slot * C::kSlot;
-          const CUtensorMap* m = st ? &tm_vs : &tm_v;
-          for (int bx = 0; bx < DV / 64; ++bx)
-            tma_load_3d(dst + bx * 16384, m, bar(BarLayout::kFull + slot), bx * 64, row, zkv);
-          issued[slot] = use + 1;
         }
       }
       if (!ok || *abort_flag) {
         // drain: every load issued lands before the CTA may exit
         for (int s = 0; s < C::kSlots; ++s)
           if (issued[s] > 0) mbar_wait_timed(bar(BarLayout::kFull + s), (issued[s] - 1) & 1);
-        mbar_wait_timed(bar(BarLayout::kQ), 0);
+        if (nq_ld > 0) mbar_wait_timed(bar(BarLayout::kQ), (nq_ld - 1) & 1);
       }
     }
   } else if (warp == 1) {
@@ -303,109 +320,132 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       const uint32_t idesc_s = idesc_bf16_f32(BM, BN, false);
       const uint32_t idesc_pv = idesc_bf16_f32(BM, DV, true);
-      const int zq = un.b * p.Hq;
-      const int ntot[2] = {un.valid[0] ? qtile_nkeys(it.k[0]) : 0, un.valid[1] ? qtile_nkeys(it.k[1]) : 0};
-      int kcount[2] = {0, 0};   // S tiles issued per sub
-      int pv_done[2] = {0, 0};  // PV products issued per sub
-      bool pending[2] = {false, false};  // sub has a PV for the previous item to issue
-      int64_t dbg_row[2] = {-1, -1};
-      for (int t = 0; t < 2; ++t)
-        if (un.valid[t] && p.dbg_tiles && !(DIFF && t == 1))
-          dbg_row[t] = (int64_t)(zq + un.hq[t]) * p.nq + un.qt[t];
-      bool ok = mbar_wait(bar(BarLayout::kQ), 0, abort_flag);
-      if (!ok) record_timeout(abort_flag, p.err_flag);
-      tc_fence_after();
+      // descriptors of slice kk differ from slice 0 only in the start
+      // address field (bits 0-13, in 16-byte units)
+      const uint64_t q_desc0[2] = {sw128_desc(sbase + C::kOffQ, 16, 1024),
+                                   sw128_desc(sbase + C::kOffQ + C::kQBytes, 16, 1024)};
       int L = 0;
-      int prev_vslot = -1, prev_vuse = 0;
-      // O_t += P_t V(prev): P_t is the bf16 tile softmax t wrote over the
-      // first 64 columns of S_t (two keys per column)
-      auto issue_pv = [&](int t) {
-        const uint32_t vb = sbase + C::kOffSlots + prev_vslot * C::kSlot;
-        const uint32_t a0 = tmem + t * BN;
-        const uint32_t dcol = tmem + (t == 0 ? C::kOCol0 : C::kOCol1);
-        const bool first = (pv_done[t] == 0);
-#pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk)
-          umma_bf16_ts(dcol, a0 + kk * 8, sw128_desc(vb + kk * 2048, 16384, 1024), idesc_pv,
-                       (first && kk == 0) ? 0u : 1u);
-        ++pv_done[t];
-        if (pv_done[t] == ntot[t]) umma_commit(bar(BarLayout::kO + t));
-        pending[t] = false;
-      };
-      auto wait_prev_v = [&]() -> bool {
-        if (!mbar_wait(bar(BarLayout::kFull + prev_vslot), prev_vuse & 1, abort_flag)) return false;
-        tc_fence_after();
-        return true;
-      };
-      for (int u = 0; u < it.n && ok; ++u) {
-        const int kslot = L % C::kSlots, kuse = L / C::kSlots;
-        ++L;
-        const int vslot = L % C::kSlots, vuse = L / C::kSlots;
-        ++L;
-        if (!mbar_wait(bar(BarLayout::kFull + kslot), kuse & 1, abort_flag)) {
+      int ksteps[2] = {0, 0};  // S tiles issued per sub, across units (barrier phases)
+      int nunit[2] = {0, 0};   // units in which the sub took part (O / O-free phases)
+      int nq = 0;              // units started (Q phases)
+      bool ok = true;
+      for (int rnd = 0; rnd * P < nunits && ok; ++rnd) {
+        const int ui = unit_of(rnd);
+        if (ui >= nunits) continue;
+        const Unit un = decode_unit(p, ui);
+        const Items it = unit_items(p, un);
+        const int ntot[2] = {un.valid[0] ? qtile_nkeys(it.k[0]) : 0, un.valid[1] ? qtile_nkeys(it.k[1]) : 0};
+        int kcount[2] = {0, 0};   // S tiles of this unit per sub
+        int pv_done[2] = {0, 0};  // PV products of this unit per sub
+        bool pending[2] = {false, false};
+        int64_t dbg_row[2] = {-1, -1};
+        for (int t = 0; t < 2; ++t)
+          if (un.valid[t] && p.dbg_tiles && !(DIFF && t == 1))
+            dbg_row[t] = (int64_t)(un.b * p.Hq + un.hq[t]) * p.nq + un.qt[t];
+        if (!mbar_wait(bar(BarLayout::kQ), nq & 1, abort_flag)) {
           record_timeout(abort_flag, p.err_flag);
           ok = false;
           break;
         }
+        ++nq;
         tc_fence_after();
-        bool v_ready = false;
-        for (int t = 0; t < 2 && ok; ++t) {
-          const bool in = item_in_sub(it, t, u);
-          if (!in && !pending[t]) continue;
-          if (kcount[t] > 0) {  // softmax t has consumed S_t and written P_t
-            if (!mbar_wait(bar(BarLayout::kP + t), (kcount[t] - 1) & 1, abort_flag)) {
-              record_timeout(abort_flag, p.err_flag);
-              ok = false;
-              break;
-            }
+        int prev_vslot = -1, prev_vuse = 0;
+        // O_t += P_t V(prev): P_t is the bf16 tile softmax t wrote over the
+        // first 64 columns of S_t (two keys per column)
+        auto issue_pv = [&](int t) -> bool {
+          if (pv_done[t] == 0 && nunit[t] > 0) {
+            // the first PV overwrites O_t: the previous unit's epilogue must be done with it
+            if (!mbar_wait(bar(BarLayout::kOFree + t), (nunit[t] - 1) & 1, abort_flag)) return false;
             tc_fence_after();
           }
-          if (pending[t]) {
-            if (!v_ready && !(v_ready = wait_prev_v())) {
-              record_timeout(abort_flag, p.err_flag);
-              ok = false;
-              break;
-            }
-            issue_pv(t);
-          }
-          if (in) {
-            const uint32_t qb = sbase + C::kOffQ + t * C::kQBytes;
-            const uint32_t kb = sbase + C::kOffSlots + kslot * C::kSlot + ((DIFF && t == 1) ? BN * DQK * 2 : 0);
-            const uint32_t dcol = tmem + t * BN;
+          const uint64_t b0 = sw128_desc(sbase + C::kOffSlots + prev_vslot * C::kSlot, 16384, 1024);
+          const uint32_t a0 = tmem + t * BN;
+          const uint32_t dcol = tmem + (t == 0 ? C::kOCol0 : C::kOCol1);
+          const bool first = (pv_done[t] == 0);
 #pragma unroll
-            for (int kk = 0; kk < DQK / 16; ++kk) {
-              const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-              umma_bf16_ss(dcol, sw128_desc(qb + off, 16, 1024), sw128_desc(kb + off, 16, 1024), idesc_s,
-                           kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < BN / 16; ++kk)
+            umma_bf16_ts(dcol, a0 + kk * 8, b0 + (uint64_t)(kk * 2048 >> 4), idesc_pv, (first && kk == 0) ? 0u : 1u);
+          ++pv_done[t];
+          if (pv_done[t] == ntot[t]) umma_commit(bar(BarLayout::kO + t));
+          pending[t] = false;
+          return true;
+        };
+        auto wait_prev_v = [&]() -> bool {
+          if (!mbar_wait(bar(BarLayout::kFull + prev_vslot), prev_vuse & 1, abort_flag)) return false;
+          tc_fence_after();
+          return true;
+        };
+        for (int u = 0; u < it.n && ok; ++u) {
+          const int kslot = L % C::kSlots, kuse = L / C::kSlots;
+          ++L;
+          const int vslot = L % C::kSlots, vuse = L / C::kSlots;
+          ++L;
+          if (!mbar_wait(bar(BarLayout::kFull + kslot), kuse & 1, abort_flag)) {
+            record_timeout(abort_flag, p.err_flag);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          bool v_ready = false;
+          for (int t = 0; t < 2 && ok; ++t) {
+            const bool in = item_in_sub(it, t, u);
+            if (!in && !pending[t]) continue;
+            if (ksteps[t] > 0) {  // softmax t has consumed S_t and written P_t
+              if (!mbar_wait(bar(BarLayout::kP + t), (ksteps[t] - 1) & 1, abort_flag)) {
+                record_timeout(abort_flag, p.err_flag);
+                ok = false;
+                break;
+              }
+              tc_fence_after();
             }
-            umma_commit(bar(BarLayout::kS + t));
-            if (dbg_row[t] >= 0 && kcount[t] < p.dbg_cap)
-              p.dbg_tiles[dbg_row[t] * p.dbg_cap + kcount[t]] =
-                  item_is_stride(it, u) ? (kStrideTag | item_tile(it, u)) : item_tile(it, u);
-            ++kcount[t];
+            if (pending[t]) {
+              if ((!v_ready && !(v_ready = wait_prev_v())) || !issue_pv(t)) {
+                record_timeout(abort_flag, p.err_flag);
+                ok = false;
+                break;
+              }
+            }
+            if (in) {
+              const uint64_t kd0 = sw128_desc(sbase + C::kOffSlots + kslot * C::kSlot +
+                                                  ((DIFF && t == 1) ? BN * DQK * 2 : 0), 16, 1024);
+              const uint32_t dcol = tmem + t * BN;
+#pragma unroll
+              for (int kk = 0; kk < DQK / 16; ++kk) {
+                const uint64_t off = (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
+                umma_bf16_ss(dcol, q_desc0[t] + off, kd0 + off, idesc_s, kk > 0 ? 1u : 0u);
+              }
+              umma_commit(bar(BarLayout::kS + t));
+              if (dbg_row[t] >= 0 && kcount[t] < p.dbg_cap)
+                p.dbg_tiles[dbg_row[t] * p.dbg_cap + kcount[t]] =
+                    item_is_stride(it, u) ? (kStrideTag | item_tile(it, u)) : item_tile(it, u);
+              ++kcount[t];
+              ++ksteps[t];
+            }
+          }
+          if (!ok) break;
+          umma_commit(bar(BarLayout::kEmpty + kslot));                            // K(u) read by this step's S
+          if (prev_vslot >= 0) umma_commit(bar(BarLayout::kEmpty + prev_vslot));  // V(u-1) by its PVs
+          if (u == it.n - 1) umma_commit(bar(BarLayout::kQEmpty));                // last S of the unit: Q free
+          for (int t = 0; t < 2; ++t) pending[t] = item_in_sub(it, t, u);
+          prev_vslot = vslot;
+          prev_vuse = vuse;
+        }
+        bool v_ready = false;
+        for (int t = 0; t < 2 && ok; ++t) {
+          if (!pending[t]) continue;
+          if (!mbar_wait(bar(BarLayout::kP + t), (ksteps[t] - 1) & 1, abort_flag) ||
+              (!v_ready && !(v_ready = wait_prev_v())) || !issue_pv(t)) {
+            record_timeout(abort_flag, p.err_flag);
+            ok = false;
+            break;
           }
         }
-        if (!ok) break;
-        umma_commit(bar(BarLayout::kEmpty + kslot));                    // K(u) read by this step's S
-        if (prev_vslot >= 0) umma_commit(bar(BarLayout::kEmpty + prev_vslot));  // V(u-1) by its PVs
-        for (int t = 0; t < 2; ++t) pending[t] = item_in_sub(it, t, u);
-        prev_vslot = vslot;
-        prev_vuse = vuse;
-      }
-      bool v_ready = false;
-      for (int t = 0; t < 2 && ok; ++t) {
-        if (!pending[t]) continue;
-        if (!mbar_wait(bar(BarLayout::kP + t), (kcount[t] - 1) & 1, abort_flag) ||
-            (!v_ready && !(v_ready = wait_prev_v()))) {
-          record_timeout(abort_flag, p.err_flag);
-          ok = false;
-          break;
+        if (ok && prev_vslot >= 0) umma_commit(bar(BarLayout::kEmpty + prev_vslot));
+        for (int t = 0; t < 2; ++t) {
+          if (dbg_row[t] >= 0) p.dbg_ntiles[dbg_row[t]] = kcount[t];
+          if (un.valid[t]) ++nunit[t];
         }
-        tc_fence_after();
-        issue_pv(t);
       }
-      for (int t = 0; t < 2; ++t)
-        if (dbg_row[t] >= 0) p.dbg_ntiles[dbg_row[t]] = kcount[t];
       if (!ok || *abort_flag) {
         umma_commit(bar(BarLayout::kFinal));
         mbar_wait_timed(bar(BarLayout::kFinal), 0);
@@ -419,21 +459,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_addr = static_cast<uint32_t>(qw * 32) << 16;
     const uint32_t s_tmem = tmem + lane_addr + t * BN;
     const uint32_t o_tmem = tmem + lane_addr + (t == 0 ? C::kOCol0 : C::kOCol1);
-    const bool valid_sub = un.valid[t] != 0;
-    const int i = un.qt[t] * BM + r;                 // query index
-    const bool row_ok = valid_sub && i < p.N;
     const int Wc = (p.kind == kMaskCausal) ? p.N : p.W;
-    const int lo = window_lo(i, Wc);
-    const int mst = (p.kind == kMaskStrided) ? stride_rows_below(lo, p.S) : 0;
     const float cl2 = p.scale_log2;
-
-    float m_run = -INFINITY;  // running max, log2 units (scores * scale * log2 e)
-    float l_run = 0.f;
-    long long cells = 0;
-    int k = 0;
+    int kglob = 0;   // S tiles consumed, across units (barrier phases)
+    int nunit = 0;   // units this sub took part in
+    int nx = 0;      // differential hand-offs
     bool ok = true;
 
-    if (valid_sub) {
+    for (int rnd = 0; rnd * P < nunits && ok; ++rnd) {
+      const int ui = unit_of(rnd);
+      if (ui >= nunits) continue;
+      const Unit un = decode_unit(p, ui);
+      const Items it = unit_items(p, un);
+      if (!un.valid[t]) continue;
+      const int i = un.qt[t] * BM + r;  // query index
+      const bool row_ok = i < p.N;
+      const int lo = window_lo(i, Wc);
+      const int mst = (p.kind == kMaskStrided) ? stride_rows_below(lo, p.S) : 0;
+      float m_run = -INFINITY;  // running max, log2 units (scores * scale * log2 e)
+      float l_run = 0.f;
+      long long cells = 0;
+      int k = 0;  // tiles of this unit
+
       for (int u = 0; u < it.n; ++u) {
         if (!item_in_sub(it, t, u)) continue;
         // attended columns [c0, c1] of this row in this tile
@@ -450,7 +497,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (c1 >= c0) cells += c1 - c0 + 1;
         const bool full = (c0 == 0 && c1 == BN - 1);
 
-        const bool got = mbar_wait(bar(BarLayout::kS + t), k & 1, abort_flag);
+        const bool got = mbar_wait(bar(BarLayout::kS + t), kglob & 1, abort_flag);
         if (!__all_sync(0xffffffffu, got)) { if (lane == 0) record_timeout(abort_flag, p.err_flag); ok = false; break; }
         tc_fence_after();
 
@@ -517,50 +564,53 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         mbar_arrive(bar(BarLayout::kP + t));
         ++k;
+        ++kglob;
       }
-    }
+      if (!ok) break;
 
-    // ---------------------------------------------------- epilogue ---
-    if (ok && valid_sub && k > 0) {
-      const bool got = mbar_wait(bar(BarLayout::kO + t), 0, abort_flag);  // the sub's last PV
-      ok = __all_sync(0xffffffffu, got);
-      if (!ok && lane == 0) record_timeout(abort_flag, p.err_flag);
-    }
-    if (ok && valid_sub && k > 0) {
+      // -------------------------------------------------- epilogue ---
+      {
+        const bool got = mbar_wait(bar(BarLayout::kO + t), nunit & 1, abort_flag);  // the sub's last PV
+        if (!__all_sync(0xffffffffu, got)) { if (lane == 0) record_timeout(abort_flag, p.err_flag); ok = false; break; }
+      }
+      ++nunit;
       tc_fence_after();
       const int hq = un.hq[t];
       const int64_t orow = ((int64_t)(un.b * p.Hq + hq) * p.N + i);
       if (DIFF) {
         if (t == 1) {
+          // hands lambda / l2 to sub 0, which reads both accumulators
           f2s[r] = (l_run > 0.f) ? p.lambda[hq] / l_run : 0.f;
+          tc_fence_before();
           mbar_arrive(bar(BarLayout::kX));
         } else {
-          const bool g1 = mbar_wait(bar(BarLayout::kO + 1), 0, abort_flag);
-          const bool g2 = mbar_wait(bar(BarLayout::kX), 0, abort_flag);
-          if (!__all_sync(0xffffffffu, g1 && g2)) {
-            if (lane == 0) record_timeout(abort_flag, p.err_flag);
-          } else {
-            tc_fence_after();
-            const float inv1 = 1.f / l_run;
-            const float f2 = f2s[r];
-            const uint32_t o2_tmem = tmem + lane_addr + C::kOCol1;
-            __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.o) + orow * DV;
+          const bool g2 = mbar_wait(bar(BarLayout::kX), nx & 1, abort_flag);
+          if (!__all_sync(0xffffffffu, g2)) { if (lane == 0) record_timeout(abort_flag, p.err_flag); ok = false; break; }
+          ++nx;
+          tc_fence_after();
+          const float inv1 = 1.f / l_run;
+          const float f2 = f2s[r];
+          const uint32_t o2_tmem = tmem + lane_addr + C::kOCol1;
+          __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.o) + orow * DV;
 #pragma unroll 1
-            for (int c = 0; c < DV; c += 32) {
-              float a[32], b2[32];
-              tmem_ld32(o_tmem + c, a);
-              tmem_ld32(o2_tmem + c, b2);
-              if (row_ok) {
+          for (int c = 0; c < DV; c += 32) {
+            float a[32], b2[32];
+            tmem_ld32(o_tmem + c, a);
+            tmem_ld32(o2_tmem + c, b2);
+            if (row_ok) {
 #pragma unroll
-                for (int e = 0; e < 32; e += 8) {
-                  st_global_v4(dst + c + e, pack_bf16(a[e] * inv1 - b2[e] * f2, a[e + 1] * inv1 - b2[e + 1] * f2),
-                               pack_bf16(a[e + 2] * inv1 - b2[e + 2] * f2, a[e + 3] * inv1 - b2[e + 3] * f2),
-                               pack_bf16(a[e + 4] * inv1 - b2[e + 4] * f2, a[e + 5] * inv1 - b2[e + 5] * f2),
-                               pack_bf16(a[e + 6] * inv1 - b2[e + 6] * f2, a[e + 7] * inv1 - b2[e + 7] * f2));
-                }
+              for (int e = 0; e < 32; e += 8) {
+                st_global_v4(dst + c + e, pack_bf16(a[e] * inv1 - b2[e] * f2, a[e + 1] * inv1 - b2[e + 1] * f2),
+                             pack_bf16(a[e + 2] * inv1 - b2[e + 2] * f2, a[e + 3] * inv1 - b2[e + 3] * f2),
+                             pack_bf16(a[e + 4] * inv1 - b2[e + 4] * f2, a[e + 5] * inv1 - b2[e + 5] * f2),
+                             pack_bf16(a[e + 6] * inv1 - b2[e + 6] * f2, a[e + 7] * inv1 - b2[e + 7] * f2));
               }
             }
           }
+          // both accumulators read: the next unit's first PVs may overwrite them
+          tc_fence_before();
+          mbar_arrive(bar(BarLayout::kOFree + 0));
+          mbar_arrive(bar(BarLayout::kOFree + 1));
         }
       } else {
         const float inv = 1.f / l_run;
@@ -576,6 +626,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                            pack_bf16(a[e + 4] * inv, a[e + 5] * inv), pack_bf16(a[e + 6] * inv, a[e + 7] * inv));
           }
         }
+        tc_fence_before();
+        mbar_arrive(bar(BarLayout::kOFree + t));  // O_t read: the next unit may overwrite it
         if (p.lse && row_ok) p.lse[orow] = (m_run + __log2f(l_run)) * 0.6931471805599453f;
       }
       if (p.dbg_cells && !(DIFF && t == 1)) {
@@ -608,7 +660,8 @@ static cudaError_t launch_one(const PrefillMaps& maps, const PrefillParams& p, i
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  kern<<<nunits, kThreads, C::kSmemBytes, stream>>>(maps.q, maps.q2, maps.k, maps.k2, maps.v, maps.ks, maps.vs, p);
+  const int grid = nunits < p.num_ctas ? nunits : p.num_ctas;
+  kern<<<grid, kThreads, C::kSmemBytes, stream>>>(maps.q, maps.q2, maps.k, maps.k2, maps.v, maps.ks, maps.vs, p);
   return cudaGetLastError();
 }
 
