@@ -49,6 +49,7 @@ constexpr int kThreads = 384;
 // new score exceeds it by more than this, so P stays below 2^8.
 constexpr float kRescaleTau = 8.0f;
 
+
 template <int DQK, int DV, bool DIFF>
 struct PrefillCfg {
   static constexpr int kQBytes = BM * DQK * 2;
@@ -530,18 +531,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         const float msub = (m_use == -INFINITY) ? 0.f : m_use;
-        float rs8[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) rs8[j] = 0.f;
+        // p = 2^(s * scale * log2 e - m): packed fp32 pairs for the scaling
+        // and the row sum, MUFU ex2 for the exponential
+        const float2 cl2x2 = make_float2(cl2, cl2), negm = make_float2(-msub, -msub);
+        float2 rs2[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
         uint32_t pk[BN / 2];
 #pragma unroll
-        for (int c = 0; c < BN; c += 2) {
-          const float p0 = ex2_approx(fmaf(s[c], cl2, -msub));
-          const float p1 = ex2_approx(fmaf(s[c + 1], cl2, -msub));
-          rs8[(c >> 1) & 7] += p0 + p1;
-          pk[c / 2] = pack_bf16(p0, p1);
+        for (int j = 0; j < BN / 2; ++j) {
+          const float2 x = __ffma2_rn(make_float2(s[2 * j], s[2 * j + 1]), cl2x2, negm);
+          const float p0 = ex2_approx(x.x);
+          const float p1 = ex2_approx(x.y);
+          rs2[j & 3] = __fadd2_rn(rs2[j & 3], make_float2(p0, p1));
+          pk[j] = pack_bf16(p0, p1);
         }
-        const float rs = ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
+        const float2 rsum = __fadd2_rn(__fadd2_rn(rs2[0], rs2[1]), __fadd2_rn(rs2[2], rs2[3]));
+        const float rs = rsum.x + rsum.y;
         l_run = l_run * alpha + rs;
         m_run = m_use;
 
