@@ -38,10 +38,10 @@ bool get_encoder() {
 // 3-D bf16 view (inner = head dim, rows, outer = batch*heads) with a
 // 64 x 128 box and the 128-byte swizzle the MMA descriptors expect.
 bool encode_rows(CUtensorMap* m, const void* base, int d, int64_t rows, int64_t outer, int64_t row_stride_el,
-                 int64_t outer_stride_el) {
+                 int64_t outer_stride_el, uint32_t box_rows = 128) {
   cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)rows, (cuuint64_t)outer};
   cuuint64_t strides[2] = {(cuuint64_t)row_stride_el * 2, (cuuint64_t)outer_stride_el * 2};
-  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t box[3] = {64, box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -88,7 +88,8 @@ swa_status_t run_prefill(int kind, bool diff, const void* q, const void* k, cons
   const int64_t nB = (int64_t)B;
   bool ok = encode_rows(&maps.q, q, dqk, N, nB * Hq, dqk, (int64_t)N * dqk) &&
             encode_rows(&maps.k, k, dqk, N, nB * Hkv, dqk, (int64_t)N * dqk) &&
-            encode_rows(&maps.v, v, dv, N, nB * Hkv, dv, (int64_t)N * dv);
+            encode_rows(&maps.v, v, dv, N, nB * Hkv, dv, (int64_t)N * dv) &&
+            encode_rows(&maps.o, o, dv, N, nB * Hq, dv, (int64_t)N * dv, 32);
   if (ok && diff)
     ok = encode_rows(&maps.q2, q2, dqk, N, nB * Hq, dqk, (int64_t)N * dqk) &&
          encode_rows(&maps.k2, k2, dqk, N, nB * Hkv, dqk, (int64_t)N * dqk);

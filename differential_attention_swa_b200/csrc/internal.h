@@ -39,6 +39,7 @@ struct PrefillParams {
 
 struct PrefillMaps {
   CUtensorMap q, q2, k, k2, v, ks, vs;
+  CUtensorMap o;  // output, 64 x 32-row boxes (one warp's rows)
 };
 
 cudaError_t launch_prefill(const PrefillMaps& maps, const PrefillParams& p, int dqk, int dv, bool diff,

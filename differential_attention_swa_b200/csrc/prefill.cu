@@ -56,12 +56,14 @@ struct PrefillCfg {
   static constexpr int kKBytes = BN * DQK * 2 * (DIFF ? 2 : 1);
   static constexpr int kVBytes = BN * DV * 2;
   static constexpr int kSlot = kKBytes > kVBytes ? kKBytes : kVBytes;
-  static constexpr int kTiles = 2 * kQBytes;
+  static constexpr int kStageBytes = 8 * 32 * 64 * 2;  // per softmax warp: 32 rows x 64 columns of bf16
+  static constexpr int kTiles = 2 * kQBytes + kStageBytes;
   static constexpr int kBudget = 227 * 1024 - 1024 - 1024;  // minus alignment slack and barriers
   static constexpr int kSlotsRaw = (kBudget - kTiles) / kSlot;
   static constexpr int kSlots = kSlotsRaw > 8 ? 8 : kSlotsRaw;
   static_assert(kSlots >= 2, "shared memory too small for the K/V ring");
   static constexpr int kOffQ = 0;
+  static constexpr int kOffStage = 2 * kQBytes;
   static constexpr int kOffSlots = kTiles;
   static constexpr int kOffBar = kTiles + kSlots * kSlot;
   static constexpr int kSmemBytes = kOffBar + 1024 + 1024;  // barriers area + alignment slack
@@ -182,7 +184,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_q2,
                    const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_k2,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_ks,
-                   const __grid_constant__ CUtensorMap tm_vs, const PrefillParams p) {
+                   const __grid_constant__ CUtensorMap tm_vs, const __grid_constant__ CUtensorMap tm_o,
+                   const PrefillParams p) {
   using C = PrefillCfg<DQK, DV, DIFF>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -462,6 +465,37 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t o_tmem = tmem + lane_addr + (t == 0 ? C::kOCol0 : C::kOCol1);
     const int Wc = (p.kind == kMaskCausal) ? p.N : p.W;
     const float cl2 = p.scale_log2;
+    // Epilogue store: this warp's 32 output rows go through a 4 KB
+    // shared-memory box (128-byte swizzle), 64 columns at a time, and lane 0
+    // writes the box with one TMA store; rows past N are clipped by TMA.
+    const uint32_t stage = sbase + C::kOffStage + (warp - 4) * 4096;
+    bool stage_used = false;
+    auto store_rows = [&](bool& used, auto&& fetch, int zrow, int row0) {
+#pragma unroll 1
+      for (int h = 0; h < DV / 64; ++h) {
+        if (used && lane == 0) bulk_wait_read();  // the previous box has been read out
+        __syncwarp();
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          float v[32];
+          fetch(64 * h + 32 * half, v);
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            const uint32_t chunk = 4 * half + q4;  // 16-byte chunk of the 128-byte row
+            const uint32_t addr = stage + lane * 128 + ((chunk ^ (lane & 7)) << 4);
+            st_shared_v4(addr, pack_bf16(v[8 * q4], v[8 * q4 + 1]), pack_bf16(v[8 * q4 + 2], v[8 * q4 + 3]),
+                         pack_bf16(v[8 * q4 + 4], v[8 * q4 + 5]), pack_bf16(v[8 * q4 + 6], v[8 * q4 + 7]));
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_3d(&tm_o, stage, 64 * h, row0, zrow);
+          bulk_commit();
+        }
+        used = true;
+      }
+    };
     int kglob = 0;   // S tiles consumed, across units (barrier phases)
     int nunit = 0;   // units this sub took part in
     int nx = 0;      // differential hand-offs
@@ -505,9 +539,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         float s[BN];
         tmem_ld128(s_tmem, s);
         if (!__all_sync(0xffffffffu, full)) {
+          // Most partial tiles are cut on one side only (the window's start,
+          // or the diagonal): test only the side some row of the warp needs.
+          const bool cut_lo = __any_sync(0xffffffffu, c0 > 0), cut_hi = __any_sync(0xffffffffu, c1 < BN - 1);
+          if (cut_lo && cut_hi) {
 #pragma unroll
-          for (int c = 0; c < BN; ++c)
-            if (c < c0 || c > c1) s[c] = -INFINITY;
+            for (int c = 0; c < BN; ++c) s[c] = (c >= c0 && c <= c1) ? s[c] : -INFINITY;
+          } else if (cut_lo) {
+#pragma unroll
+            for (int c = 0; c < BN; ++c) s[c] = (c >= c0) ? s[c] : -INFINITY;
+          } else {
+#pragma unroll
+            for (int c = 0; c < BN; ++c) s[c] = (c <= c1) ? s[c] : -INFINITY;
+          }
         }
         // row max over 8 independent chains
         float mx8[8];
@@ -595,22 +639,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float inv1 = 1.f / l_run;
           const float f2 = f2s[r];
           const uint32_t o2_tmem = tmem + lane_addr + C::kOCol1;
-          __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.o) + orow * DV;
-#pragma unroll 1
-          for (int c = 0; c < DV; c += 32) {
-            float a[32], b2[32];
-            tmem_ld32(o_tmem + c, a);
+          store_rows(stage_used, [&](int c, float* v) {
+            float b2[32];
+            tmem_ld32(o_tmem + c, v);
             tmem_ld32(o2_tmem + c, b2);
-            if (row_ok) {
 #pragma unroll
-              for (int e = 0; e < 32; e += 8) {
-                st_global_v4(dst + c + e, pack_bf16(a[e] * inv1 - b2[e] * f2, a[e + 1] * inv1 - b2[e + 1] * f2),
-                             pack_bf16(a[e + 2] * inv1 - b2[e + 2] * f2, a[e + 3] * inv1 - b2[e + 3] * f2),
-                             pack_bf16(a[e + 4] * inv1 - b2[e + 4] * f2, a[e + 5] * inv1 - b2[e + 5] * f2),
-                             pack_bf16(a[e + 6] * inv1 - b2[e + 6] * f2, a[e + 7] * inv1 - b2[e + 7] * f2));
-              }
-            }
-          }
+            for (int e = 0; e < 32; ++e) v[e] = v[e] * inv1 - b2[e] * f2;
+          }, un.b * p.Hq + hq, un.qt[t] * BM + qw * 32);
           // both accumulators read: the next unit's first PVs may overwrite them
           tc_fence_before();
           mbar_arrive(bar(BarLayout::kOFree + 0));
@@ -618,18 +653,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       } else {
         const float inv = 1.f / l_run;
-        __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.o) + orow * DV;
-#pragma unroll 1
-        for (int c = 0; c < DV; c += 32) {
-          float a[32];
-          tmem_ld32(o_tmem + c, a);
-          if (row_ok) {
+        store_rows(stage_used, [&](int c, float* v) {
+          tmem_ld32(o_tmem + c, v);
 #pragma unroll
-            for (int e = 0; e < 32; e += 8)
-              st_global_v4(dst + c + e, pack_bf16(a[e] * inv, a[e + 1] * inv), pack_bf16(a[e + 2] * inv, a[e + 3] * inv),
-                           pack_bf16(a[e + 4] * inv, a[e + 5] * inv), pack_bf16(a[e + 6] * inv, a[e + 7] * inv));
-          }
-        }
+          for (int e = 0; e < 32; ++e) v[e] *= inv;
+        }, un.b * p.Hq + hq, un.qt[t] * BM + qw * 32);
         tc_fence_before();
         mbar_arrive(bar(BarLayout::kOFree + t));  // O_t read: the next unit may overwrite it
         if (p.lse && row_ok) p.lse[orow] = (m_run + __log2f(l_run)) * 0.6931471805599453f;
@@ -645,6 +673,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
+  if (warp >= 4 && lane == 0) bulk_wait_all();  // output stores complete before exit
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -665,7 +694,8 @@ static cudaError_t launch_one(const PrefillMaps& maps, const PrefillParams& p, i
     attr_set = true;
   }
   const int grid = nunits < p.num_ctas ? nunits : p.num_ctas;
-  kern<<<grid, kThreads, C::kSmemBytes, stream>>>(maps.q, maps.q2, maps.k, maps.k2, maps.v, maps.ks, maps.vs, p);
+  kern<<<grid, kThreads, C::kSmemBytes, stream>>>(maps.q, maps.q2, maps.k, maps.k2, maps.v, maps.ks, maps.vs,
+                                                  maps.o, p);
   return cudaGetLastError();
 }
 
