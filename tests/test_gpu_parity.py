@@ -135,7 +135,10 @@ def test_diff_small_full(orc, N, W, dv, Hq, Hkv):
 # ---------------------------------------------------------------- decode --
 
 @pytest.mark.parametrize("B,Hq,Hkv,d,W,pos0,T", [(2, 4, 2, 128, 64, 3, 70), (3, 16, 8, 128, 1024, 131072, 3),
-                                                  (2, 2, 2, 64, 100, 0, 5), (1, 8, 1, 128, 256, 250, 10)])
+                                                  (2, 2, 2, 64, 100, 0, 5), (1, 8, 1, 128, 256, 250, 10),
+                                                  (1, 2, 1, 128, 4096, 4090, 8),   # one group, long window
+                                                  (5, 8, 8, 64, 1500, 1400, 3),   # last split ragged
+                                                  (40, 8, 8, 128, 2048, 5000, 2)])  # many groups, 2048 slots
 def test_decode_steps_vs_oracle(orc, B, Hq, Hkv, d, W, pos0, T):
     q, k_new, v_new, k_cache, v_cache = decode_inputs(T, B, Hq, Hkv, d, W, seed=5)
     pos = np.array([[pos0 + t] * B for t in range(T)], dtype=np.int32)
