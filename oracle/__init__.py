@@ -69,6 +69,8 @@ def _L():
         lib.orc_diff_attention.restype = I
         lib.orc_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, D, P]
         lib.orc_decode.restype = I
+        lib.orc_sink_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, D, P]
+        lib.orc_sink_decode.restype = I
         lib.orc_schedule_qtile.argtypes = [I, I, I, I, I, I, I, P, I64, P]
         lib.orc_schedule_qtile.restype = I64
         _lib = lib
@@ -230,6 +232,30 @@ def decode(q, k_new, v_new, k_cache, v_cache, pos, scale: float | None = None):
     out = np.empty((T, B, Hq, d), dtype=np.float64)
     rc = _L().orc_decode(_p(q), _p(k_new), _p(v_new), _p(kc), _p(vc), _p(pos), T, B, Hq, Hkv, d, W,
                          float(scale), _p(out))
+    if rc != 0:
+        raise ValueError("oracle: bad arguments")
+    return out, kc, vc
+
+
+def sink_decode(q, k_new, v_new, k_cache, v_cache, pos, n_sink: int, scale: float | None = None):
+    """T decode steps with attention sinks over an (n_sink + W)-slot cache
+    (StreamingLLM): positions below n_sink stay in their own slot, later ones
+    rotate through the W window slots. Shapes as decode(); caches
+    [B,Hkv,n_sink+W,d]. Returns (out, k_cache_after, v_cache_after)."""
+    q, k_new, v_new = _f32(q), _f32(k_new), _f32(v_new)
+    kc = _f32(k_cache).copy()
+    vc = _f32(v_cache).copy()
+    pos = np.ascontiguousarray(pos, dtype=np.int32)
+    T, B, Hq, d = q.shape
+    Hkv = k_new.shape[2]
+    W = kc.shape[2] - n_sink
+    if W < 1:
+        raise ValueError("the cache needs at least one window slot")
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    out = np.empty((T, B, Hq, d), dtype=np.float64)
+    rc = _L().orc_sink_decode(_p(q), _p(k_new), _p(v_new), _p(kc), _p(vc), _p(pos), T, B, Hq, Hkv, d,
+                              int(n_sink), W, float(scale), _p(out))
     if rc != 0:
         raise ValueError("oracle: bad arguments")
     return out, kc, vc

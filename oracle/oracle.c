@@ -461,3 +461,73 @@ int64_t orc_schedule_qtile(int kind, int N, int W, int S, int Bq, int Bk, int qt
   if (bad) return -2;
   return n > cap ? -1 : n;
 }
+
+/* ---------------------------------------------------------------------- */
+/* Decode with attention sinks ("Learn: Sparse & Sliding-Window           */
+/* Attention", section 4, StreamingLLM: keep the first k tokens for good  */
+/* plus the most recent w tokens, drop the middle; section 6: O(k + w)).  */
+/* ---------------------------------------------------------------------- */
+
+/* Caches: [B,Hkv,n_sink+W,d]. Positions p < n_sink stay in slot p for good;
+ * a later position p takes slot n_sink + (p - n_sink) % W, overwriting the
+ * oldest non-sink token. Each step first stores its token, then attends over
+ * the sink positions 0 .. min(n_sink, pos+1)-1 and the recent positions
+ * max(n_sink, pos-W+1) .. pos, each read from its slot. Shapes as
+ * orc_decode; n_sink = 0 is the plain rolling window. */
+int orc_sink_decode(const float* q, const float* k_new, const float* v_new, float* k_cache,
+                    float* v_cache, const int32_t* pos, int T, int B, int Hq, int Hkv, int d,
+                    int n_sink, int W, double scale, double* out) {
+  if (Hkv <= 0 || Hq % Hkv != 0 || W <= 0 || n_sink < 0) return 1;
+  const int G = Hq / Hkv;
+  const int slots = n_sink + W;
+  int* key_slot = (int*)malloc(sizeof(int) * (size_t)slots);
+  double* s = (double*)malloc(sizeof(double) * (size_t)slots);
+  double* qd = (double*)malloc(sizeof(double) * (size_t)d);
+  for (int t = 0; t < T; ++t) {
+    for (int b = 0; b < B; ++b) {
+      const int p = pos[(int64_t)t * B + b];
+      const int slot = (p < n_sink) ? p : n_sink + (p - n_sink) % W;
+      for (int hk = 0; hk < Hkv; ++hk) {
+        const int64_t src = (((int64_t)t * B + b) * Hkv + hk) * d;
+        const int64_t dst = (((int64_t)b * Hkv + hk) * slots + slot) * d;
+        memcpy(k_cache + dst, k_new + src, sizeof(float) * (size_t)d);
+        memcpy(v_cache + dst, v_new + src, sizeof(float) * (size_t)d);
+      }
+      /* the attended positions, each mapped to its slot */
+      int cnt = 0;
+      for (int u = 0; u < n_sink && u <= p; ++u) key_slot[cnt++] = u;
+      int first = p - W + 1;
+      if (first < n_sink) first = n_sink;
+      for (int u = first; u <= p; ++u) key_slot[cnt++] = n_sink + (u - n_sink) % W;
+      for (int hq = 0; hq < Hq; ++hq) {
+        const int hk = hq / G;
+        const float* qrow = q + (((int64_t)t * B + b) * Hq + hq) * d;
+        for (int c = 0; c < d; ++c) qd[c] = (double)qrow[c];
+        const float* Kc = k_cache + ((int64_t)b * Hkv + hk) * (int64_t)slots * d;
+        const float* Vc = v_cache + ((int64_t)b * Hkv + hk) * (int64_t)slots * d;
+        double mx = -INFINITY;
+        for (int u = 0; u < cnt; ++u) {
+          double dot = 0.0;
+          for (int c = 0; c < d; ++c) dot += qd[c] * (double)Kc[(int64_t)key_slot[u] * d + c];
+          s[u] = scale * dot;
+          if (s[u] > mx) mx = s[u];
+        }
+        double denom = 0.0;
+        for (int u = 0; u < cnt; ++u) {
+          s[u] = exp(s[u] - mx);
+          denom += s[u];
+        }
+        double* o = out + (((int64_t)t * B + b) * Hq + hq) * d;
+        for (int c = 0; c < d; ++c) o[c] = 0.0;
+        for (int u = 0; u < cnt; ++u) {
+          const double w = s[u] / denom;
+          for (int c = 0; c < d; ++c) o[c] += w * (double)Vc[(int64_t)key_slot[u] * d + c];
+        }
+      }
+    }
+  }
+  free(key_slot);
+  free(s);
+  free(qd);
+  return 0;
+}

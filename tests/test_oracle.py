@@ -378,3 +378,64 @@ def test_core_flops_table(orc):
     # a two-sided window of exactly w keys per row: s*w entries -> 4bswd
     assert orc.core_flops(s * w, d, b) == 4 * b * s * w * d
     assert (32768 * 32768) // (32768 * 2048) == nums["score_flops_reduction_w2048_s32768"]
+
+
+# ------------------------------------------------------ attention sinks ---
+
+def _sink_history(B, Hkv, Hq, d, n_sink, W, pos0, T, seed):
+    """A K/V history of pos0 + T tokens, a cache holding what a sink cache
+    holds before step pos0, and the T new tokens."""
+    L = pos0 + T
+    Kh = randn_bf16((B, Hkv, L, d), seed).float()
+    Vh = randn_bf16((B, Hkv, L, d), seed + 1).float()
+    q = randn_bf16((T, B, Hq, d), seed + 2).float()
+    kc = torch.full((B, Hkv, n_sink + W, d), float("nan"))  # unfilled slots must never be read
+    vc = torch.full((B, Hkv, n_sink + W, d), float("nan"))
+    for p in range(pos0):
+        if p < n_sink:
+            slot = p
+        elif p >= pos0 - W:
+            slot = n_sink + (p - n_sink) % W
+        else:
+            continue
+        kc[:, :, slot] = Kh[:, :, p]
+        vc[:, :, slot] = Vh[:, :, p]
+    k_new = Kh[:, :, pos0:].permute(2, 0, 1, 3).contiguous()
+    v_new = Vh[:, :, pos0:].permute(2, 0, 1, 3).contiguous()
+    pos = np.array([[pos0 + t] * B for t in range(T)], dtype=np.int32)
+    return Kh, Vh, q, kc, vc, k_new, v_new, pos
+
+
+@pytest.mark.parametrize("n_sink,W,pos0,T", [(4, 8, 0, 20), (4, 8, 30, 9), (1, 5, 2, 12), (3, 16, 10, 4),
+                                             (4, 6, 9, 1)])
+def test_sink_decode_equals_softmax_over_sinks_and_window(orc, n_sink, W, pos0, T):
+    """Step at pos attends positions 0 .. n_sink-1 (those <= pos) and the W
+    most recent positions above the sinks, whatever slots hold them."""
+    B, Hq, Hkv, d = 2, 4, 2, 16
+    Kh, Vh, q, kc, vc, k_new, v_new, pos = _sink_history(B, Hkv, Hq, d, n_sink, W, pos0, T, 40)
+    out, kc2, vc2 = orc.sink_decode(q, k_new, v_new, kc, vc, pos, n_sink)
+    G = Hq // Hkv
+    for t in range(T):
+        p = pos0 + t
+        keys = sorted(set(range(min(n_sink, p + 1))) | set(range(max(n_sink, p - W + 1), p + 1)))
+        assert len(keys) <= n_sink + W  # bounded cache, O(k + w)
+        Kw = Kh[:, :, keys].double().repeat_interleave(G, dim=1)
+        Vw = Vh[:, :, keys].double().repeat_interleave(G, dim=1)
+        ref = F.scaled_dot_product_attention(q[t].double()[:, :, None], Kw, Vw, scale=1 / 4)[:, :, 0]
+        assert np.abs(out[t] - ref.numpy()).max() < 1e-12
+    last = pos0 + T - 1
+    for p in range(min(n_sink, last + 1)):  # sinks never leave
+        assert np.array_equal(kc2[:, :, p], Kh[:, :, p].numpy())
+    for p in range(max(n_sink, last - W + 1), last + 1):
+        assert np.array_equal(vc2[:, :, n_sink + (p - n_sink) % W], Vh[:, :, p].numpy())
+
+
+def test_sink_decode_without_sinks_is_the_rolling_window(orc):
+    T, B, Hq, Hkv, d, W = 6, 2, 4, 2, 16, 8
+    q = randn_bf16((T, B, Hq, d), 1)
+    k_new, v_new = randn_bf16((T, B, Hkv, d), 2), randn_bf16((T, B, Hkv, d), 3)
+    kc, vc = randn_bf16((B, Hkv, W, d), 4), randn_bf16((B, Hkv, W, d), 5)
+    pos = np.array([[20 + t, 3 + t] for t in range(T)], dtype=np.int32)
+    a, ka, va = orc.decode(q, k_new, v_new, kc, vc, pos)
+    b, kb, vb = orc.sink_decode(q, k_new, v_new, kc, vc, pos, 0)
+    assert np.array_equal(a, b) and np.array_equal(ka, kb) and np.array_equal(va, vb)
