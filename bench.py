@@ -219,25 +219,31 @@ def prefill_workload(name, rank):
     return w, fn, flops, ins, out
 
 
-def decode_workload(rank):
+def decode_workload(rank, name="gemma_swa_decode"):
     import torch
 
     import differential_attention_swa_b200 as swa
     from differential_attention_swa_b200.inputs import WORKLOADS, decode_inputs
 
-    w = WORKLOADS["gemma_swa_decode"]
+    w = WORKLOADS[name]
+    n_sink = int(w.extra.get("n_sink", 0))
     T = w.steps
-    q, kn, vn, kc, vc = decode_inputs(T, w.B, w.Hq, w.Hkv, w.d, w.W, seed=shard_seed(0, rank))
+    q, kn, vn, kc, vc = decode_inputs(T, w.B, w.Hq, w.Hkv, w.d, n_sink + w.W, seed=shard_seed(0, rank))
     q, kn, vn, kc, vc = (t.cuda() for t in (q, kn, vn, kc, vc))
     pos = torch.tensor([[w.pos0 + t] * w.B for t in range(T)], dtype=torch.int32, device="cuda")
     out = torch.empty_like(q)
-    ws = torch.empty(swa.decode_workspace_bytes(w.B, w.Hq, w.Hkv, w.d, w.W), dtype=torch.uint8, device="cuda")
+    ws = torch.empty(max(16, swa.sink_decode_workspace_bytes(w.B, w.Hq, w.Hkv, w.d, n_sink, w.W)),
+                     dtype=torch.uint8, device="cuda")
     stream = torch.cuda.Stream()
     torch.cuda.synchronize()
 
     def steps():
         for t in range(T):
-            swa.swa_decode_step(q[t], kn[t], vn[t], kc, vc, pos[t], out=out[t], workspace=ws, scale=w.scale)
+            if n_sink:
+                swa.swa_sink_decode_step(q[t], kn[t], vn[t], kc, vc, pos[t], n_sink, out=out[t], workspace=ws,
+                                         scale=w.scale)
+            else:
+                swa.swa_decode_step(q[t], kn[t], vn[t], kc, vc, pos[t], out=out[t], workspace=ws, scale=w.scale)
 
     with torch.cuda.stream(stream):
         steps()  # warm (also sets kernel attributes before capture)
@@ -247,7 +253,7 @@ def decode_workload(rank):
         steps()
     # bytes per step: K and V of every cached slot read once per KV head, the
     # query and output rows, the new token's K and V
-    kv = 2 * w.B * w.Hkv * w.W * w.d * 2
+    kv = 2 * w.B * w.Hkv * (n_sink + w.W) * w.d * 2
     qo = 2 * w.B * w.Hq * w.d * 2
     new = 2 * w.B * w.Hkv * w.d * 2
     bytes_per_step = kv + qo + new
@@ -268,8 +274,8 @@ def measure_ours(args, rank, world, peaks, peak_src, dist):
         bus = f"{getattr(props, 'pci_domain_id', 0):08X}:{props.pci_bus_id:02X}:{getattr(props, 'pci_device_id', 0):02X}.0"
 
     main_name = args.only or "mistral_swa_prefill"
-    if main_name == "gemma_swa_decode":
-        return measure_decode_only(args, rank, world, peaks, flush, stream)
+    if main_name.endswith("_decode"):
+        return measure_decode_only(args, rank, world, peaks, flush, stream, main_name)
     w, fn, flops, ins, out = prefill_workload(main_name, rank)
     clocks = ClockSampler(bus)
     if dist:
@@ -342,16 +348,16 @@ def measure_e2e(w, fn, ins, out, flops, stream, steps=5):
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
 
-def measure_decode_only(args, rank, world, peaks, flush, stream):
-    v = measure_decode(args, rank, peaks, flush, stream)
+def measure_decode_only(args, rank, world, peaks, flush, stream, name):
+    v = measure_decode(args, rank, peaks, flush, stream, name=name)
     return {"metric": "decode HBM GB/s", "value": v["value"], "unit": "GB/s", "n_gpus": world, "steps": v["steps"],
-            "ms_per_step": v["ms_per_step"], "roofline": v["roofline"], "config": {"workload": "gemma_swa_decode"}}
+            "ms_per_step": v["ms_per_step"], "roofline": v["roofline"], "config": {"workload": name}}
 
 
-def measure_decode(args, rank, peaks, flush, stream, reps=5):
+def measure_decode(args, rank, peaks, flush, stream, reps=5, name="gemma_swa_decode"):
     import torch
 
-    w, g, bytes_per_step, T = decode_workload(rank)
+    w, g, bytes_per_step, T = decode_workload(rank, name)
     ms = time_steps(lambda: g.replay(), reps, 3, flush, stream)
     mean_ms = sum(ms) / len(ms)
     gbs = bytes_per_step * T / (mean_ms * 1e-3) / 1e9
@@ -387,6 +393,7 @@ def measure_variants(args, rank, peaks, flush, stream):
         del ins, o, fn
         torch.cuda.empty_cache()
     out["gemma_swa_decode"] = measure_decode(args, rank, peaks, flush, stream)
+    out["gemma_sink_decode"] = measure_decode(args, rank, peaks, flush, stream, name="gemma_sink_decode")
     if swa.last_device_error() != swa.OK:
         raise RuntimeError("a variant kernel reported an error")
     return out

@@ -26,6 +26,7 @@ TILE = 128  # query rows and keys per tile in the prefill kernels
 
 __all__ = [
     "swa_attn_fwd", "strided_attn_fwd", "diff_attn_fwd", "swa_decode_step", "decode_workspace_bytes",
+    "swa_sink_decode_step", "sink_decode_workspace_bytes",
     "prefill_debug", "schedule", "count_nonmasked", "last_device_error", "SwaError", "library",
 ]
 
@@ -59,6 +60,10 @@ def library() -> ctypes.CDLL:
     lib.swa_decode_step.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, F, P, SZ, P]
     lib.swa_decode_workspace_bytes.argtypes = [I, I, I, I, I]
     lib.swa_decode_workspace_bytes.restype = SZ
+    lib.swa_sink_decode_step.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, F, P, SZ, P]
+    lib.swa_sink_decode_step.restype = I
+    lib.swa_sink_decode_workspace_bytes.argtypes = [I, I, I, I, I, I]
+    lib.swa_sink_decode_workspace_bytes.restype = SZ
     lib.swa_prefill_debug.argtypes = [I, P, P, P, P, P, I, I, I, I, I, I, I, F, ctypes.POINTER(_Debug), P]
     lib.swa_schedule.argtypes = [I, I, I, I, I, I, P, P, I64]
     lib.swa_schedule.restype = I64
@@ -187,6 +192,39 @@ def swa_decode_step(q, k_new, v_new, k_cache, v_cache, pos, out=None, workspace=
                                    _ptr(out), B, Hq, Hkv, d, W, float(scale), _ptr(workspace),
                                    workspace.numel() * workspace.element_size(), _stream(stream))
     _raise(st, "swa_decode_step")
+    return out
+
+
+def sink_decode_workspace_bytes(B: int, Hq: int, Hkv: int, d: int, n_sink: int, W: int) -> int:
+    return int(library().swa_sink_decode_workspace_bytes(B, Hq, Hkv, d, n_sink, W))
+
+
+def swa_sink_decode_step(q, k_new, v_new, k_cache, v_cache, pos, n_sink: int, out=None, workspace=None,
+                         scale: float | None = None, stream=None):
+    """One decode step with attention sinks: the cache holds n_sink sink
+    slots (positions 0 .. n_sink-1, kept for good) then W rolling slots."""
+    _check(q, "q", dim=3)
+    _check(k_new, "k_new", dim=3)
+    _check(v_new, "v_new", dim=3)
+    _check(k_cache, "k_cache", dim=4)
+    _check(v_cache, "v_cache", dim=4)
+    _check(pos, "pos", dtype=torch.int32, dim=1)
+    B, Hq, d = q.shape
+    Hkv = k_cache.shape[1]
+    W = k_cache.shape[2] - int(n_sink)
+    if W < 1:
+        raise ValueError("the cache needs at least one window slot after the sinks")
+    if out is None:
+        out = torch.empty_like(q)
+    need = sink_decode_workspace_bytes(B, Hq, Hkv, d, n_sink, W)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    st = library().swa_sink_decode_step(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache),
+                                        _ptr(pos), _ptr(out), B, Hq, Hkv, d, int(n_sink), W, float(scale),
+                                        _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                        _stream(stream))
+    _raise(st, "swa_sink_decode_step")
     return out
 
 

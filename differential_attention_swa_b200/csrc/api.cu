@@ -164,6 +164,34 @@ int read_and_clear_device_error(cudaStream_t stream, int* err) {
 
 }  // namespace swa
 
+namespace swa {
+namespace {
+swa_status_t run_decode(const void* q, const void* k_new, const void* v_new, void* k_cache, void* v_cache,
+                        const int32_t* pos, void* o, int B, int Hq, int Hkv, int d, int n_sink, int W, float scale,
+                        void* workspace, size_t ws_bytes, void* stream) {
+  if (!aligned16(q) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) || !aligned16(v_cache) ||
+      !aligned16(o) || pos == nullptr || (reinterpret_cast<uintptr_t>(pos) & 3u))
+    return SWA_ERR_INVALID_ARG;
+  if (B < 1 || Hq < 1 || Hkv < 1 || W < 1 || n_sink < 0 || Hq % Hkv != 0) return SWA_ERR_INVALID_ARG;
+  if ((int64_t)n_sink + W > (1 << 30)) return SWA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return SWA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return SWA_ERR_UNSUPPORTED;
+  const int G = Hq / Hkv;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return SWA_ERR_UNSUPPORTED;
+  const size_t need = decode_partial_bytes(B, Hq, Hkv, d, n_sink + W);
+  if (!aligned16(workspace) || ws_bytes < need) return SWA_ERR_INVALID_ARG;
+  DecodeParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.q = q; p.k_new = k_new; p.v_new = v_new; p.k_cache = k_cache; p.v_cache = v_cache; p.pos = pos; p.o = o;
+  p.partial = static_cast<float*>(workspace);
+  p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.d = d; p.W = W; p.G = G; p.n_sink = n_sink;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  cudaError_t e = launch_decode(p, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
+}
+}  // namespace
+}  // namespace swa
+
 using namespace swa;
 
 extern "C" {
@@ -204,24 +232,20 @@ size_t swa_decode_workspace_bytes(int B, int Hq, int Hkv, int d, int W) {
 swa_status_t swa_decode_step(const void* q, const void* k_new, const void* v_new, void* k_cache, void* v_cache,
                              const int32_t* pos, void* o, int B, int Hq, int Hkv, int d, int W, float scale,
                              void* workspace, size_t ws_bytes, void* stream) {
-  if (!aligned16(q) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) || !aligned16(v_cache) ||
-      !aligned16(o) || pos == nullptr || (reinterpret_cast<uintptr_t>(pos) & 3u))
-    return SWA_ERR_INVALID_ARG;
-  if (B < 1 || Hq < 1 || Hkv < 1 || W < 1 || Hq % Hkv != 0) return SWA_ERR_INVALID_ARG;
-  if (!(scale > 0.f) || !std::isfinite(scale)) return SWA_ERR_INVALID_ARG;
-  if (d != 64 && d != 128) return SWA_ERR_UNSUPPORTED;
-  const int G = Hq / Hkv;
-  if (G != 1 && G != 2 && G != 4 && G != 8) return SWA_ERR_UNSUPPORTED;
-  const size_t need = decode_partial_bytes(B, Hq, Hkv, d, W);
-  if (!aligned16(workspace) || ws_bytes < need) return SWA_ERR_INVALID_ARG;
-  DecodeParams p;
-  std::memset(&p, 0, sizeof(p));
-  p.q = q; p.k_new = k_new; p.v_new = v_new; p.k_cache = k_cache; p.v_cache = v_cache; p.pos = pos; p.o = o;
-  p.partial = static_cast<float*>(workspace);
-  p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.d = d; p.W = W; p.G = G;
-  p.scale_log2 = scale * 1.4426950408889634f;
-  cudaError_t e = launch_decode(p, static_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
+  return run_decode(q, k_new, v_new, k_cache, v_cache, pos, o, B, Hq, Hkv, d, 0, W, scale, workspace, ws_bytes,
+                    stream);
+}
+
+swa_status_t swa_sink_decode_step(const void* q, const void* k_new, const void* v_new, void* k_cache,
+                                  void* v_cache, const int32_t* pos, void* o, int B, int Hq, int Hkv, int d,
+                                  int n_sink, int W, float scale, void* workspace, size_t ws_bytes, void* stream) {
+  return run_decode(q, k_new, v_new, k_cache, v_cache, pos, o, B, Hq, Hkv, d, n_sink, W, scale, workspace,
+                    ws_bytes, stream);
+}
+
+size_t swa_sink_decode_workspace_bytes(int B, int Hq, int Hkv, int d, int n_sink, int W) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || W < 1 || n_sink < 0 || Hq % Hkv != 0 || (d != 64 && d != 128)) return 0;
+  return decode_partial_bytes(B, Hq, Hkv, d, n_sink + W);
 }
 
 int64_t swa_schedule(int kind, int N, int W, int stride, int Bq, int Bk, int32_t* qtile_offsets, int32_t* tiles,

@@ -51,6 +51,8 @@ __device__ __forceinline__ void bf16x8_to_float(const uint4& u, float* f) {
   }
 }
 
+__device__ __forceinline__ int imin_dec(int a, int b) { return a < b ? a : b; }
+
 // Record of one split's partial result: m, l, two pad words, then d floats.
 __host__ __device__ constexpr int partial_stride(int d) { return d + 4; }
 
@@ -69,9 +71,12 @@ __global__ void __launch_bounds__(kDecThreads)
   const int rr = lane / LPR;   // row within the warp's load
   const int e = lane % LPR;    // 8-element column group
 
+  // Slots 0 .. n_sink-1 hold positions 0 .. n_sink-1 for good (attention
+  // sinks); a later position p rotates through slot n_sink + (p-n_sink) % W.
+  // The slots in use are always a prefix [0, nvalid) of the n_sink + W.
   const int pos = p.pos[b];
-  const int nvalid = pos + 1 < p.W ? pos + 1 : p.W;
-  const int new_slot = pos % p.W;
+  const int nvalid = pos < p.n_sink ? pos + 1 : p.n_sink + imin_dec(p.W, pos + 1 - p.n_sink);
+  const int new_slot = pos < p.n_sink ? pos : p.n_sink + (pos - p.n_sink) % p.W;
   const int s0 = split * p.chunk;
   const int s1 = (s0 + p.chunk) < nvalid ? (s0 + p.chunk) : nvalid;
 
@@ -94,7 +99,7 @@ __global__ void __launch_bounds__(kDecThreads)
     for (int c = 0; c < 8; ++c) acc[g][c] = 0.f;
   }
 
-  const int64_t cache_base = (int64_t)bk * p.W * D;
+  const int64_t cache_base = (int64_t)bk * (p.n_sink + p.W) * D;
   const __nv_bfloat16* kc = reinterpret_cast<const __nv_bfloat16*>(p.k_cache) + cache_base;
   const __nv_bfloat16* vc = reinterpret_cast<const __nv_bfloat16*>(p.v_cache) + cache_base;
   const __nv_bfloat16* kn = reinterpret_cast<const __nv_bfloat16*>(p.k_new) + (int64_t)bk * D;
@@ -249,8 +254,8 @@ static int decode_chunk(int B, int Hkv, int W) {
   return ((chunk + 63) / 64) * 64;
 }
 
-size_t decode_partial_bytes(int B, int Hq, int Hkv, int d, int W) {
-  return (size_t)B * Hq * decode_nsplit(B, Hkv, W) * partial_stride(d) * sizeof(float);
+size_t decode_partial_bytes(int B, int Hq, int Hkv, int d, int slots) {
+  return (size_t)B * Hq * decode_nsplit(B, Hkv, slots) * partial_stride(d) * sizeof(float);
 }
 
 template <int D, int G>
@@ -265,8 +270,8 @@ static cudaError_t launch_g(DecodeParams p, cudaStream_t stream) {
 
 cudaError_t launch_decode(const DecodeParams& p0, cudaStream_t stream) {
   DecodeParams p = p0;
-  p.nsplit = decode_nsplit(p.B, p.Hkv, p.W);
-  p.chunk = decode_chunk(p.B, p.Hkv, p.W);
+  p.nsplit = decode_nsplit(p.B, p.Hkv, p.n_sink + p.W);
+  p.chunk = decode_chunk(p.B, p.Hkv, p.n_sink + p.W);
   if (p.d == 128) {
     switch (p.G) {
       case 1: return launch_g<128, 1>(p, stream);
@@ -345,6 +350,7 @@ extern "C" swa_status_t swa_decode_step_static(const void* q, const void* k_new,
   p.q = q; p.k_new = k_new; p.v_new = v_new; p.k_cache = k_cache; p.v_cache = v_cache; p.pos = pos; p.o = o;
   p.partial = scratch;
   p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.d = d; p.W = W; p.G = G;
+  p.n_sink = 0;
   p.scale_log2 = scale * 1.4426950408889634f;
   return launch_decode(p, static_cast<cudaStream_t>(stream)) == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
 }

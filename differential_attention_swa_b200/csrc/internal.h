@@ -56,12 +56,13 @@ struct DecodeParams {
   void* o;
   float* partial;  // [B*Hq][nsplit][d + 2]
   int B, Hq, Hkv, d, W, G;
+  int n_sink;  // attention-sink slots ahead of the W window slots (0: none)
   int nsplit, chunk;
   float scale_log2;
 };
 
 int decode_nsplit(int B, int Hkv, int W);
-size_t decode_partial_bytes(int B, int Hq, int Hkv, int d, int W);
+size_t decode_partial_bytes(int B, int Hq, int Hkv, int d, int slots);
 cudaError_t launch_decode(const DecodeParams& p, cudaStream_t stream);
 
 int* device_error_ptr();

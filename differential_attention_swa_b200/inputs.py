@@ -85,4 +85,7 @@ WORKLOADS = {
     "gemma_swa_prefill": Workload("gemma_swa_prefill", "swa", 1, 16, 8, 131072, 128, 1024),
     "gemma_swa_decode": Workload("gemma_swa_decode", "decode", 64, 16, 8, 0, 128, 1024, steps=256,
                                  pos0=131072),
+    # the same decode with 4 attention-sink slots ahead of the window
+    "gemma_sink_decode": Workload("gemma_sink_decode", "decode", 64, 16, 8, 0, 128, 1024, steps=256,
+                                  pos0=131072, extra={"n_sink": 4}),
 }

@@ -129,6 +129,27 @@ swa_status_t swa_decode_step(const void* q, const void* k_new, const void* v_new
 /* Scratch bytes swa_decode_step needs for these sizes (0 on bad sizes). */
 size_t swa_decode_workspace_bytes(int B, int Hq, int Hkv, int d, int W);
 
+/* One decode step with attention sinks over an (n_sink + W)-slot cache.
+ * Source: "Learn: Sparse & Sliding-Window Attention", section 4
+ * (StreamingLLM: keep the first k tokens -- the attention sinks -- for good
+ * plus the most recent w tokens, drop the middle) and section 6 (the cache
+ * stays O(k + w)).
+ *   k_cache, v_cache [B,Hkv,n_sink+W,d] bf16 (device, updated): positions
+ *     p < n_sink live in slot p for good; a later position p takes slot
+ *     n_sink + (p - n_sink) % W, replacing the oldest non-sink token;
+ *   the step stores its token, then attends over the sink positions
+ *     0 .. min(n_sink, pos+1)-1 and the positions max(n_sink, pos-W+1) .. pos;
+ *   n_sink >= 0 (0 is swa_decode_step); workspace of at least
+ *     swa_sink_decode_workspace_bytes(...) bytes; other arguments as
+ *     swa_decode_step. */
+swa_status_t swa_sink_decode_step(const void* q, const void* k_new, const void* v_new,
+                                  void* k_cache, void* v_cache, const int32_t* pos, void* o,
+                                  int B, int Hq, int Hkv, int d, int n_sink, int W, float scale,
+                                  void* workspace, size_t ws_bytes, void* stream);
+
+/* Scratch bytes swa_sink_decode_step needs (0 on bad sizes). */
+size_t swa_sink_decode_workspace_bytes(int B, int Hq, int Hkv, int d, int n_sink, int W);
+
 /* Bytes of the scratch array compiled into the library for
  * swa_decode_step_static (on every GPU that loads the library). */
 #define SWA_DECODE_STATIC_SCRATCH_BYTES (4u << 20)

@@ -155,6 +155,23 @@ def test_decode_steps_vs_oracle(orc, B, Hq, Hkv, d, W, pos0, T):
     assert np.array_equal(vc.float().cpu().numpy(), vc_ref)
 
 
+@pytest.mark.parametrize("B,Hq,Hkv,d,n_sink,W,pos0,T", [(2, 4, 2, 128, 4, 64, 0, 70), (2, 4, 2, 128, 4, 64, 200, 3),
+                                                         (3, 16, 8, 128, 4, 1024, 131072, 2),
+                                                         (1, 8, 1, 64, 2, 100, 5, 20), (2, 2, 2, 128, 1, 1, 0, 6)])
+def test_sink_decode_vs_oracle(orc, B, Hq, Hkv, d, n_sink, W, pos0, T):
+    q, k_new, v_new, k_cache, v_cache = decode_inputs(T, B, Hq, Hkv, d, n_sink + W, seed=9)
+    pos = np.array([[pos0 + t] * B for t in range(T)], dtype=np.int32)
+    ref, kc_ref, vc_ref = orc.sink_decode(q, k_new, v_new, k_cache, v_cache, pos, n_sink)
+    kc, vc = gpu(k_cache, v_cache)
+    posd = torch.from_numpy(pos).cuda()
+    qd, knd, vnd = gpu(q, k_new, v_new)
+    outs = [swa.swa_sink_decode_step(qd[t], knd[t], vnd[t], kc, vc, posd[t], n_sink) for t in range(T)]
+    assert swa.last_device_error() == swa.OK
+    compare(torch.stack(outs), ref, "sink decode")
+    assert np.array_equal(kc.float().cpu().numpy(), kc_ref)
+    assert np.array_equal(vc.float().cpu().numpy(), vc_ref)
+
+
 # ------------------------------------------------------ workload sizes ----
 
 def sampled_rows(B, H, N, n, seed):
