@@ -71,6 +71,8 @@ def _L():
         lib.orc_decode.restype = I
         lib.orc_sink_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, D, P]
         lib.orc_sink_decode.restype = I
+        lib.orc_diff_decode.argtypes = [P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, D, P]
+        lib.orc_diff_decode.restype = I
         lib.orc_schedule_qtile.argtypes = [I, I, I, I, I, I, I, P, I64, P]
         lib.orc_schedule_qtile.restype = I64
         _lib = lib
@@ -259,6 +261,30 @@ def sink_decode(q, k_new, v_new, k_cache, v_cache, pos, n_sink: int, scale: floa
     if rc != 0:
         raise ValueError("oracle: bad arguments")
     return out, kc, vc
+
+
+def diff_decode(q1, q2, k1_new, k2_new, v_new, k1_cache, k2_cache, v_cache, lam, pos,
+                scale: float | None = None):
+    """T differential decode steps over a rolling W-slot cache: both maps
+    attend over the window, one V cache is shared.
+
+    q1, q2: [T,B,Hq,dk]; k1_new, k2_new: [T,B,Hkv,dk]; v_new: [T,B,Hkv,dv];
+    caches [B,Hkv,W,dk] / [B,Hkv,W,dv] (copied); lam: [Hq]; pos: [T,B].
+    Returns (out [T,B,Hq,dv] fp64, k1_cache, k2_cache, v_cache after)."""
+    q1, q2, k1_new, k2_new, v_new = _f32(q1), _f32(q2), _f32(k1_new), _f32(k2_new), _f32(v_new)
+    k1c, k2c, vc = _f32(k1_cache).copy(), _f32(k2_cache).copy(), _f32(v_cache).copy()
+    lam = _f32(lam).reshape(-1)
+    pos = np.ascontiguousarray(pos, dtype=np.int32)
+    T, B, Hq, dk = q1.shape
+    Hkv, W, dv = vc.shape[1], vc.shape[2], vc.shape[3]
+    if scale is None:
+        scale = 1.0 / np.sqrt(dk)
+    out = np.empty((T, B, Hq, dv), dtype=np.float64)
+    rc = _L().orc_diff_decode(_p(q1), _p(q2), _p(k1_new), _p(k2_new), _p(v_new), _p(k1c), _p(k2c), _p(vc),
+                              _p(lam), _p(pos), T, B, Hq, Hkv, dk, dv, W, float(scale), _p(out))
+    if rc != 0:
+        raise ValueError("oracle: bad arguments")
+    return out, k1c, k2c, vc
 
 
 # ------------------------------------------------------------- schedule ---

@@ -531,3 +531,75 @@ int orc_sink_decode(const float* q, const float* k_new, const float* v_new, floa
   free(qd);
   return 0;
 }
+
+/* Differential attention, one decode step per (t, b), over a rolling W-slot
+ * cache ("Differential Transformer" reading: two softmax maps over the same
+ * keys, combined as w1 - lambda_h w2 and applied to one shared V).
+ * q1, q2: [T,B,Hq,dk]; k1_new, k2_new: [T,B,Hkv,dk]; v_new: [T,B,Hkv,dv];
+ * caches k1c, k2c: [B,Hkv,W,dk], vc: [B,Hkv,W,dv], updated in place; lambda:
+ * [Hq]. Each step writes its token into slot pos % W, then attends over the
+ * positions max(0, pos-W+1) .. pos. out: [T,B,Hq,dv] doubles. */
+int orc_diff_decode(const float* q1, const float* q2, const float* k1_new, const float* k2_new,
+                    const float* v_new, float* k1c, float* k2c, float* vc, const float* lambda,
+                    const int32_t* pos, int T, int B, int Hq, int Hkv, int dk, int dv, int W,
+                    double scale, double* out) {
+  if (Hkv <= 0 || Hq % Hkv != 0 || W <= 0) return 1;
+  const int G = Hq / Hkv;
+  double* s1 = (double*)malloc(sizeof(double) * (size_t)W);
+  double* s2 = (double*)malloc(sizeof(double) * (size_t)W);
+  int* key_slot = (int*)malloc(sizeof(int) * (size_t)W);
+  for (int t = 0; t < T; ++t) {
+    for (int b = 0; b < B; ++b) {
+      const int p = pos[(int64_t)t * B + b];
+      const int slot = p % W;
+      for (int hk = 0; hk < Hkv; ++hk) {
+        const int64_t src = ((int64_t)t * B + b) * Hkv + hk;
+        const int64_t dst = ((int64_t)b * Hkv + hk) * W + slot;
+        memcpy(k1c + dst * dk, k1_new + src * dk, sizeof(float) * (size_t)dk);
+        memcpy(k2c + dst * dk, k2_new + src * dk, sizeof(float) * (size_t)dk);
+        memcpy(vc + dst * dv, v_new + src * dv, sizeof(float) * (size_t)dv);
+      }
+      int cnt = 0;
+      for (int u = (p - W + 1 > 0 ? p - W + 1 : 0); u <= p; ++u) key_slot[cnt++] = u % W;
+      for (int hq = 0; hq < Hq; ++hq) {
+        const int hk = hq / G;
+        const float* a1 = q1 + (((int64_t)t * B + b) * Hq + hq) * dk;
+        const float* a2 = q2 + (((int64_t)t * B + b) * Hq + hq) * dk;
+        const int64_t cb = ((int64_t)b * Hkv + hk) * W;
+        double m1 = -INFINITY, m2 = -INFINITY;
+        for (int u = 0; u < cnt; ++u) {
+          double d1 = 0.0, d2 = 0.0;
+          const float* r1 = k1c + (cb + key_slot[u]) * dk;
+          const float* r2 = k2c + (cb + key_slot[u]) * dk;
+          for (int c = 0; c < dk; ++c) {
+            d1 += (double)a1[c] * (double)r1[c];
+            d2 += (double)a2[c] * (double)r2[c];
+          }
+          s1[u] = scale * d1;
+          s2[u] = scale * d2;
+          if (s1[u] > m1) m1 = s1[u];
+          if (s2[u] > m2) m2 = s2[u];
+        }
+        double z1 = 0.0, z2 = 0.0;
+        for (int u = 0; u < cnt; ++u) {
+          s1[u] = exp(s1[u] - m1);
+          s2[u] = exp(s2[u] - m2);
+          z1 += s1[u];
+          z2 += s2[u];
+        }
+        const double lam = (double)lambda[hq];
+        double* o = out + (((int64_t)t * B + b) * Hq + hq) * dv;
+        for (int c = 0; c < dv; ++c) o[c] = 0.0;
+        for (int u = 0; u < cnt; ++u) {
+          const double w = s1[u] / z1 - lam * (s2[u] / z2);
+          const float* vr = vc + (cb + key_slot[u]) * dv;
+          for (int c = 0; c < dv; ++c) o[c] += w * (double)vr[c];
+        }
+      }
+    }
+  }
+  free(s1);
+  free(s2);
+  free(key_slot);
+  return 0;
+}

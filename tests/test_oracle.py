@@ -439,3 +439,56 @@ def test_sink_decode_without_sinks_is_the_rolling_window(orc):
     a, ka, va = orc.decode(q, k_new, v_new, kc, vc, pos)
     b, kb, vb = orc.sink_decode(q, k_new, v_new, kc, vc, pos, 0)
     assert np.array_equal(a, b) and np.array_equal(ka, kb) and np.array_equal(va, vb)
+
+
+# ------------------------------------------------------ differential decode --
+
+def _diff_history(B, Hkv, Hq, dk, dv, W, pos0, T, seed):
+    """Histories of K1, K2, V over pos0 + T tokens, caches holding what a
+    W-slot rolling cache holds before step pos0, and the T new tokens."""
+    L = pos0 + T
+    K1h = randn_bf16((B, Hkv, L, dk), seed).float()
+    K2h = randn_bf16((B, Hkv, L, dk), seed + 1).float()
+    Vh = randn_bf16((B, Hkv, L, dv), seed + 2).float()
+    q1 = randn_bf16((T, B, Hq, dk), seed + 3).float()
+    q2 = randn_bf16((T, B, Hq, dk), seed + 4).float()
+    caches = [torch.full((B, Hkv, W, x), float("nan")) for x in (dk, dk, dv)]  # unfilled slots never read
+    for p in range(max(0, pos0 - W), pos0):
+        for c, h in zip(caches, (K1h, K2h, Vh)):
+            c[:, :, p % W] = h[:, :, p]
+    new = [h[:, :, pos0:].permute(2, 0, 1, 3).contiguous() for h in (K1h, K2h, Vh)]
+    pos = np.array([[pos0 + t] * B for t in range(T)], dtype=np.int32)
+    return (K1h, K2h, Vh), (q1, q2), caches, new, pos
+
+
+@pytest.mark.parametrize("W,pos0,T,G", [(8, 0, 12, 2), (8, 30, 9, 1), (5, 2, 10, 4), (16, 40, 3, 2)])
+def test_diff_decode_is_difference_of_two_window_softmaxes(orc, W, pos0, T, G):
+    """Each step equals SDPA(q1, K1w, Vw) - lambda_h SDPA(q2, K2w, Vw) over
+    the window positions max(0, p-W+1) .. p, whatever slots hold them; V is
+    the same for both maps."""
+    B, Hkv, dk, dv = 2, 2, 16, 24
+    Hq = Hkv * G
+    (K1h, K2h, Vh), (q1, q2), (k1c, k2c, vc), (k1n, k2n, vn), pos = _diff_history(B, Hkv, Hq, dk, dv, W, pos0, T, 60)
+    lam = torch.linspace(-0.5, 0.9, Hq)
+    out, k1a, k2a, va = orc.diff_decode(q1, q2, k1n, k2n, vn, k1c, k2c, vc, lam, pos)
+    for t in range(T):
+        p = pos0 + t
+        keys = list(range(max(0, p - W + 1), p + 1))
+        K1w, K2w, Vw = (h[:, :, keys].double().repeat_interleave(G, dim=1) for h in (K1h, K2h, Vh))
+        a1 = F.scaled_dot_product_attention(q1[t].double()[:, :, None], K1w, Vw, scale=1 / 4)[:, :, 0]
+        a2 = F.scaled_dot_product_attention(q2[t].double()[:, :, None], K2w, Vw, scale=1 / 4)[:, :, 0]
+        ref = a1 - lam.double()[None, :, None] * a2
+        assert np.abs(out[t] - ref.numpy()).max() < 1e-12
+    last = pos0 + T - 1
+    for p in range(max(0, last - W + 1), last + 1):  # the window's tokens sit in slot p % W
+        assert np.array_equal(k2a[:, :, p % W], K2h[:, :, p].numpy())
+        assert np.array_equal(va[:, :, p % W], Vh[:, :, p].numpy())
+
+
+def test_diff_decode_with_lambda_zero_is_the_plain_decode(orc):
+    T, B, Hq, Hkv, d, W = 5, 2, 4, 2, 16, 8
+    (K1h, K2h, Vh), (q1, q2), (k1c, k2c, vc), (k1n, k2n, vn), pos = _diff_history(B, Hkv, Hq, d, d, W, 20, T, 70)
+    out, k1a, _, va = orc.diff_decode(q1, q2, k1n, k2n, vn, k1c, k2c, vc, np.zeros(Hq), pos)
+    ref, kr, vr = orc.decode(q1, k1n, vn, k1c, vc, pos)
+    assert np.abs(out - ref).max() < 1e-12
+    assert np.array_equal(k1a, kr) and np.array_equal(va, vr)
