@@ -226,6 +226,8 @@ def decode_workload(rank, name="gemma_swa_decode"):
     from differential_attention_swa_b200.inputs import WORKLOADS, decode_inputs
 
     w = WORKLOADS[name]
+    if w.kind == "diff_decode":
+        return diff_decode_workload(rank, w)
     n_sink = int(w.extra.get("n_sink", 0))
     T = w.steps
     q, kn, vn, kc, vc = decode_inputs(T, w.B, w.Hq, w.Hkv, w.d, n_sink + w.W, seed=shard_seed(0, rank))
@@ -258,6 +260,43 @@ def decode_workload(rank, name="gemma_swa_decode"):
     new = 2 * w.B * w.Hkv * w.d * 2
     bytes_per_step = kv + qo + new
     return w, g, bytes_per_step, T
+
+
+def diff_decode_workload(rank, w):
+    import torch
+
+    import differential_attention_swa_b200 as swa
+    from differential_attention_swa_b200.inputs import diff_decode_inputs
+
+    T, dk, dv = w.steps, w.d, w.dv_
+    ins = diff_decode_inputs(T, w.B, w.Hq, w.Hkv, dk, dv, w.W, seed=shard_seed(0, rank))
+    q1, q2, k1n, k2n, vn, k1c, k2c, vc = (t.cuda() for t in ins)
+    lam = torch.full((w.Hq,), w.lam, dtype=torch.float32, device="cuda")
+    pos = torch.tensor([[w.pos0 + t] * w.B for t in range(T)], dtype=torch.int32, device="cuda")
+    out = torch.empty((T, w.B, w.Hq, dv), dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(max(16, swa.diff_decode_workspace_bytes(w.B, w.Hq, w.Hkv, dk, dv, w.W)), dtype=torch.uint8,
+                     device="cuda")
+    stream = torch.cuda.Stream()
+    torch.cuda.synchronize()
+
+    def steps():
+        for t in range(T):
+            swa.swa_diff_decode_step(q1[t], q2[t], k1n[t], k2n[t], vn[t], k1c, k2c, vc, pos[t], lam, out=out[t],
+                                     workspace=ws, scale=w.scale)
+
+    with torch.cuda.stream(stream):
+        steps()
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        steps()
+    # bytes per step: K1, K2 and V of every cached slot read once per KV head
+    # (V once for both maps), both maps' query rows, the output row, the new
+    # token's K1, K2 and V, and lambda
+    kv = w.B * w.Hkv * w.W * (2 * dk + dv) * 2
+    qo = w.B * w.Hq * (2 * dk + dv) * 2
+    new = w.B * w.Hkv * (2 * dk + dv) * 2
+    return w, g, kv + qo + new + 4 * w.Hq, T
 
 
 def measure_ours(args, rank, world, peaks, peak_src, dist):
@@ -358,6 +397,7 @@ def measure_decode(args, rank, peaks, flush, stream, reps=5, name="gemma_swa_dec
     import torch
 
     w, g, bytes_per_step, T = decode_workload(rank, name)
+    diff = w.kind == "diff_decode"
     ms = time_steps(lambda: g.replay(), reps, 3, flush, stream)
     mean_ms = sum(ms) / len(ms)
     gbs = bytes_per_step * T / (mean_ms * 1e-3) / 1e9
@@ -368,8 +408,9 @@ def measure_decode(args, rank, peaks, flush, stream, reps=5, name="gemma_swa_dec
             "decode_steps_per_graph": T, "bytes_per_decode_step": bytes_per_step,
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
                          "frac": round(gbs / peak, 4),
-                         "traffic": profiled_traffic("decode_gemma.md", DECODE_SOURCES),
-                         "kernel": "decode_split_kernel<128,2> + decode_combine_kernel<128>"},
+                         "traffic": None if diff else profiled_traffic("decode_gemma.md", DECODE_SOURCES),
+                         "kernel": ("diff_decode_split_kernel<2> + diff_decode_combine_kernel" if diff else
+                                    "decode_split_kernel<128,2> + decode_combine_kernel<128>")},
             "launches": reps * T * 2}
 
 
@@ -394,6 +435,7 @@ def measure_variants(args, rank, peaks, flush, stream):
         torch.cuda.empty_cache()
     out["gemma_swa_decode"] = measure_decode(args, rank, peaks, flush, stream)
     out["gemma_sink_decode"] = measure_decode(args, rank, peaks, flush, stream, name="gemma_sink_decode")
+    out["diff_gqa_decode"] = measure_decode(args, rank, peaks, flush, stream, name="diff_gqa_decode")
     if swa.last_device_error() != swa.OK:
         raise RuntimeError("a variant kernel reported an error")
     return out

@@ -26,7 +26,7 @@ TILE = 128  # query rows and keys per tile in the prefill kernels
 
 __all__ = [
     "swa_attn_fwd", "strided_attn_fwd", "diff_attn_fwd", "swa_decode_step", "decode_workspace_bytes",
-    "swa_sink_decode_step", "sink_decode_workspace_bytes",
+    "swa_sink_decode_step", "sink_decode_workspace_bytes", "swa_diff_decode_step", "diff_decode_workspace_bytes",
     "prefill_debug", "schedule", "count_nonmasked", "last_device_error", "SwaError", "library",
 ]
 
@@ -64,6 +64,10 @@ def library() -> ctypes.CDLL:
     lib.swa_sink_decode_step.restype = I
     lib.swa_sink_decode_workspace_bytes.argtypes = [I, I, I, I, I, I]
     lib.swa_sink_decode_workspace_bytes.restype = SZ
+    lib.swa_diff_decode_step.argtypes = [P, P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, P, SZ, P]
+    lib.swa_diff_decode_step.restype = I
+    lib.swa_diff_decode_workspace_bytes.argtypes = [I, I, I, I, I, I]
+    lib.swa_diff_decode_workspace_bytes.restype = SZ
     lib.swa_prefill_debug.argtypes = [I, P, P, P, P, P, I, I, I, I, I, I, I, F, ctypes.POINTER(_Debug), P]
     lib.swa_schedule.argtypes = [I, I, I, I, I, I, P, P, I64]
     lib.swa_schedule.restype = I64
@@ -225,6 +229,37 @@ def swa_sink_decode_step(q, k_new, v_new, k_cache, v_cache, pos, n_sink: int, ou
                                         _ptr(workspace), workspace.numel() * workspace.element_size(),
                                         _stream(stream))
     _raise(st, "swa_sink_decode_step")
+    return out
+
+
+def diff_decode_workspace_bytes(B: int, Hq: int, Hkv: int, d_qk: int, d_v: int, W: int) -> int:
+    return int(library().swa_diff_decode_workspace_bytes(B, Hq, Hkv, d_qk, d_v, W))
+
+
+def swa_diff_decode_step(q1, q2, k1_new, k2_new, v_new, k1_cache, k2_cache, v_cache, pos, lam, out=None,
+                         workspace=None, scale: float | None = None, stream=None):
+    """One differential decode step: two maps over the same rolling window,
+    V cache shared. q1, q2 [B,Hq,64]; k*_new [B,Hkv,64]; v_new [B,Hkv,128];
+    k*_cache [B,Hkv,W,64]; v_cache [B,Hkv,W,128]; lam fp32 [Hq]."""
+    for t, n in ((q1, "q1"), (q2, "q2"), (k1_new, "k1_new"), (k2_new, "k2_new"), (v_new, "v_new")):
+        _check(t, n, dim=3)
+    for t, n in ((k1_cache, "k1_cache"), (k2_cache, "k2_cache"), (v_cache, "v_cache")):
+        _check(t, n, dim=4)
+    _check(pos, "pos", dtype=torch.int32, dim=1)
+    _check(lam, "lambda", dtype=torch.float32, dim=1)
+    B, Hq, dqk = q1.shape
+    Hkv, W, dv = v_cache.shape[1], v_cache.shape[2], v_cache.shape[3]
+    if out is None:
+        out = torch.empty((B, Hq, dv), dtype=q1.dtype, device=q1.device)
+    need = diff_decode_workspace_bytes(B, Hq, Hkv, dqk, dv, W)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q1.device)
+    scale = 1.0 / math.sqrt(dqk) if scale is None else scale
+    st = library().swa_diff_decode_step(_ptr(q1), _ptr(q2), _ptr(k1_new), _ptr(k2_new), _ptr(v_new), _ptr(k1_cache),
+                                        _ptr(k2_cache), _ptr(v_cache), _ptr(pos), _ptr(lam), _ptr(out), B, Hq, Hkv,
+                                        dqk, dv, W, float(scale), _ptr(workspace),
+                                        workspace.numel() * workspace.element_size(), _stream(stream))
+    _raise(st, "swa_diff_decode_step")
     return out
 
 

@@ -248,6 +248,36 @@ size_t swa_sink_decode_workspace_bytes(int B, int Hq, int Hkv, int d, int n_sink
   return decode_partial_bytes(B, Hq, Hkv, d, n_sink + W);
 }
 
+size_t swa_diff_decode_workspace_bytes(int B, int Hq, int Hkv, int d_qk, int d_v, int W) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || W < 1 || Hq % Hkv != 0 || d_qk != 64 || d_v != 128) return 0;
+  return diff_decode_partial_bytes(B, Hq, Hkv, W);
+}
+
+swa_status_t swa_diff_decode_step(const void* q1, const void* q2, const void* k1_new, const void* k2_new,
+                                  const void* v_new, void* k1_cache, void* k2_cache, void* v_cache,
+                                  const int32_t* pos, const float* lambda, void* o, int B, int Hq, int Hkv, int d_qk,
+                                  int d_v, int W, float scale, void* workspace, size_t ws_bytes, void* stream) {
+  if (!aligned16(q1) || !aligned16(q2) || !aligned16(k1_new) || !aligned16(k2_new) || !aligned16(v_new) ||
+      !aligned16(k1_cache) || !aligned16(k2_cache) || !aligned16(v_cache) || !aligned16(o) || pos == nullptr ||
+      (reinterpret_cast<uintptr_t>(pos) & 3u) || lambda == nullptr || (reinterpret_cast<uintptr_t>(lambda) & 3u))
+    return SWA_ERR_INVALID_ARG;
+  if (B < 1 || Hq < 1 || Hkv < 1 || W < 1 || Hq % Hkv != 0 || W > (1 << 30)) return SWA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return SWA_ERR_INVALID_ARG;
+  if (d_qk != 64 || d_v != 128) return SWA_ERR_UNSUPPORTED;
+  const int G = Hq / Hkv;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return SWA_ERR_UNSUPPORTED;
+  if (!aligned16(workspace) || ws_bytes < diff_decode_partial_bytes(B, Hq, Hkv, W)) return SWA_ERR_INVALID_ARG;
+  DiffDecodeParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.q1 = q1; p.q2 = q2; p.k1_new = k1_new; p.k2_new = k2_new; p.v_new = v_new;
+  p.k1_cache = k1_cache; p.k2_cache = k2_cache; p.v_cache = v_cache; p.o = o;
+  p.pos = pos; p.lambda = lambda; p.partial = static_cast<float*>(workspace);
+  p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.W = W; p.G = G;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  cudaError_t e = launch_diff_decode(p, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
+}
+
 int64_t swa_schedule(int kind, int N, int W, int stride, int Bq, int Bk, int32_t* qtile_offsets, int32_t* tiles,
                      int64_t cap) {
   if (N < 1 || Bq < 1 || Bk < 1 || kind < 0 || kind > 2) return -1;

@@ -61,6 +61,21 @@ struct DecodeParams {
   float scale_log2;
 };
 
+// Differential decode: two maps (q1/K1, q2/K2) over one rolling window and
+// one shared V cache; d_qk = 64, d_v = 128.
+struct DiffDecodeParams {
+  const void *q1, *q2, *k1_new, *k2_new, *v_new;
+  void *k1_cache, *k2_cache, *v_cache, *o;
+  const int32_t* pos;
+  const float* lambda;
+  float* partial;
+  int B, Hq, Hkv, W, G;
+  int nsplit, chunk;
+  float scale_log2;
+};
+size_t diff_decode_partial_bytes(int B, int Hq, int Hkv, int W);
+cudaError_t launch_diff_decode(const DiffDecodeParams& p, cudaStream_t stream);
+
 int decode_nsplit(int B, int Hkv, int W);
 size_t decode_partial_bytes(int B, int Hq, int Hkv, int d, int slots);
 cudaError_t launch_decode(const DecodeParams& p, cudaStream_t stream);

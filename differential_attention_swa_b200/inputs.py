@@ -48,10 +48,24 @@ def decode_inputs(T, B, Hq, Hkv, d, W, seed: int = 0):
     return q, k_new, v_new, k_cache, v_cache
 
 
+def diff_decode_inputs(T, B, Hq, Hkv, dk, dv, W, seed: int = 0):
+    """Caches pre-filled with W tokens (K1, K2, V), then T steps of new
+    tokens and both maps' queries."""
+    k1_cache = randn_bf16((B, Hkv, W, dk), seed + 0)
+    k2_cache = randn_bf16((B, Hkv, W, dk), seed + 1)
+    v_cache = randn_bf16((B, Hkv, W, dv), seed + 2)
+    q1 = randn_bf16((T, B, Hq, dk), seed + 3)
+    q2 = randn_bf16((T, B, Hq, dk), seed + 4)
+    k1_new = randn_bf16((T, B, Hkv, dk), seed + 5)
+    k2_new = randn_bf16((T, B, Hkv, dk), seed + 6)
+    v_new = randn_bf16((T, B, Hkv, dv), seed + 7)
+    return q1, q2, k1_new, k2_new, v_new, k1_cache, k2_cache, v_cache
+
+
 @dataclass(frozen=True)
 class Workload:
     name: str
-    kind: str  # "swa", "strided", "diff", "decode"
+    kind: str  # "swa", "strided", "diff", "decode", "diff_decode"
     B: int
     Hq: int
     Hkv: int
@@ -88,4 +102,8 @@ WORKLOADS = {
     # the same decode with 4 attention-sink slots ahead of the window
     "gemma_sink_decode": Workload("gemma_sink_decode", "decode", 64, 16, 8, 0, 128, 1024, steps=256,
                                   pos0=131072, extra={"n_sink": 4}),
+    # differential decode with the differential prefill's head dims and
+    # context (4096-token window), GQA groups of 2: both maps share V
+    "diff_gqa_decode": Workload("diff_gqa_decode", "diff_decode", 64, 16, 8, 0, 64, 4096, dv=128, lam=0.8,
+                                steps=256, pos0=4096),
 }

@@ -150,6 +150,37 @@ swa_status_t swa_sink_decode_step(const void* q, const void* k_new, const void* 
 /* Scratch bytes swa_sink_decode_step needs (0 on bad sizes). */
 size_t swa_sink_decode_workspace_bytes(int B, int Hq, int Hkv, int d, int n_sink, int W);
 
+/* One differential-attention decode step over a rolling W-slot cache.
+ * ("Differential Transformer": out = sum_j (w1_j - lambda_h w2_j) v_j with
+ * w1 = softmax(scale q1 K1^T), w2 = softmax(scale q2 K2^T) over the same
+ * window; "Differential Transformer V2" names the first version's double
+ * read of the value cache, which this step avoids: every slot's K1, K2 and
+ * V bytes are read once. Window as swa_decode_step: "Learn: Sparse &
+ * Sliding-Window Attention", section 4.)
+ *   q1, q2            device bf16 [B, Hq, d_qk]
+ *   k1_new, k2_new    device bf16 [B, Hkv, d_qk]; v_new [B, Hkv, d_v]
+ *   k1_cache, k2_cache device bf16 [B, Hkv, W, d_qk]; v_cache [B, Hkv, W, d_v];
+ *                     position p lives in slot p % W; the step first stores
+ *                     its token in slot pos % W, then attends over the
+ *                     positions max(0, pos-W+1) .. pos
+ *   pos               device int32 [B], absolute position of the new token
+ *   lambda            device fp32 [Hq]
+ *   o                 device bf16 [B, Hq, d_v]
+ *   d_qk = 64 and d_v = 128 only (SWA_ERR_UNSUPPORTED otherwise); Hq/Hkv in
+ *   {1, 2, 4, 8}; workspace: device, 16-byte aligned, at least
+ *   swa_diff_decode_workspace_bytes(...) bytes, owned by the caller.
+ * Pointers not 16-byte aligned (pos and lambda: 4), a null pointer, a short
+ * workspace or a bad size return SWA_ERR_INVALID_ARG before any launch. */
+swa_status_t swa_diff_decode_step(const void* q1, const void* q2, const void* k1_new,
+                                  const void* k2_new, const void* v_new, void* k1_cache,
+                                  void* k2_cache, void* v_cache, const int32_t* pos,
+                                  const float* lambda, void* o, int B, int Hq, int Hkv,
+                                  int d_qk, int d_v, int W, float scale, void* workspace,
+                                  size_t ws_bytes, void* stream);
+
+/* Scratch bytes swa_diff_decode_step needs (0 on bad or unsupported sizes). */
+size_t swa_diff_decode_workspace_bytes(int B, int Hq, int Hkv, int d_qk, int d_v, int W);
+
 /* Bytes of the scratch array compiled into the library for
  * swa_decode_step_static (on every GPU that loads the library). */
 #define SWA_DECODE_STATIC_SCRATCH_BYTES (4u << 20)

@@ -132,3 +132,24 @@ def test_python_binding_refuses_cpu_tensors(lib):
     q = torch.zeros(1, 2, 8, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         swa.swa_attn_fwd(q, q, q, 4)
+
+
+def test_diff_decode_bad_arguments_rejected_before_launch(lib):
+    P, I, F, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    g = P(0x10000)  # aligned, never dereferenced: validation fails first
+    ws = lib.swa_diff_decode_workspace_bytes(64, 16, 8, 64, 128, 4096)
+    assert ws > 0
+    assert lib.swa_diff_decode_workspace_bytes(64, 16, 8, 128, 128, 4096) == 0  # d_qk 128 not built
+    assert lib.swa_diff_decode_workspace_bytes(64, 16, 6, 64, 128, 4096) == 0  # Hq % Hkv
+
+    def call(B=64, Hq=16, Hkv=8, dqk=64, dv=128, W=4096, scale=0.125, wsb=ws, lam=g, q1=g):
+        return lib.swa_diff_decode_step(q1, g, g, g, g, g, g, g, g, lam, g, I(B), I(Hq), I(Hkv), I(dqk), I(dv),
+                                        I(W), F(scale), g, SZ(wsb), None)
+
+    assert call(wsb=ws - 1) == swa.ERR_INVALID_ARG  # workspace too small
+    assert call(lam=None) == swa.ERR_INVALID_ARG  # lambda missing
+    assert call(q1=P(0x10008)) == swa.ERR_INVALID_ARG  # misaligned
+    assert call(W=0) == swa.ERR_INVALID_ARG
+    assert call(scale=0.0) == swa.ERR_INVALID_ARG
+    assert call(dqk=128) == swa.ERR_UNSUPPORTED
+    assert call(Hq=24, Hkv=8) == swa.ERR_UNSUPPORTED  # group of 3

@@ -11,7 +11,7 @@ import pytest
 import torch
 
 import differential_attention_swa_b200 as swa
-from differential_attention_swa_b200.inputs import WORKLOADS, attn_inputs, decode_inputs, diff_inputs
+from differential_attention_swa_b200.inputs import WORKLOADS, attn_inputs, decode_inputs, diff_decode_inputs, diff_inputs
 
 pytestmark = pytest.mark.gpu
 
@@ -172,6 +172,36 @@ def test_sink_decode_vs_oracle(orc, B, Hq, Hkv, d, n_sink, W, pos0, T):
     assert np.array_equal(vc.float().cpu().numpy(), vc_ref)
 
 
+def run_diff_decode(orc, B, Hq, Hkv, W, pos0, T, seed, lam=None):
+    dk, dv = 64, 128
+    ins = diff_decode_inputs(T, B, Hq, Hkv, dk, dv, W, seed=seed)
+    q1, q2, k1n, k2n, vn, k1c, k2c, vc = ins
+    # lambda in the range the method uses (0 < lambda < 1): with it the
+    # outputs stay below 4, where bf16's half-ulp (1.56e-2 from 4 up) would
+    # exceed the bar by itself; the oracle's pins cover negative lambda
+    lam = torch.linspace(0.2, 0.8, Hq) if lam is None else lam
+    pos = np.array([[pos0 + t] * B for t in range(T)], dtype=np.int32)
+    ref, k1r, k2r, vr = orc.diff_decode(q1, q2, k1n, k2n, vn, k1c, k2c, vc, lam, pos)
+    k1d, k2d, vd = gpu(k1c, k2c, vc)
+    q1d, q2d, k1nd, k2nd, vnd = gpu(q1, q2, k1n, k2n, vn)
+    posd, lamd = torch.from_numpy(pos).cuda(), lam.float().cuda()
+    outs = [swa.swa_diff_decode_step(q1d[t], q2d[t], k1nd[t], k2nd[t], vnd[t], k1d, k2d, vd, posd[t], lamd)
+            for t in range(T)]
+    assert swa.last_device_error() == swa.OK
+    return torch.stack(outs), ref, (k1d, k2d, vd), (k1r, k2r, vr)
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,W,pos0,T", [(2, 4, 2, 64, 0, 70), (3, 16, 8, 4096, 4096, 2), (1, 8, 1, 100, 5, 20),
+                                               (2, 2, 2, 1, 0, 4), (5, 4, 1, 1500, 1400, 3), (2, 16, 16, 300, 900, 2)])
+def test_diff_decode_vs_oracle(orc, B, Hq, Hkv, W, pos0, T):
+    """Both maps over the rolling window, V read once: early positions,
+    wrap-around, GQA groups 1-8, W = 1 and a ragged last split."""
+    out, ref, caches, caches_ref = run_diff_decode(orc, B, Hq, Hkv, W, pos0, T, seed=31)
+    compare(out, ref, "diff decode")
+    for c, r in zip(caches, caches_ref):  # each new token stored in slot pos % W, nothing else touched
+        assert np.array_equal(c.float().cpu().numpy(), r)
+
+
 # ------------------------------------------------------ workload sizes ----
 
 def sampled_rows(B, H, N, n, seed):
@@ -201,6 +231,13 @@ def test_diff_workload_sampled_rows(orc):
     rows = sampled_rows(w.B, w.Hq, w.N, 1500, 2)
     ref = orc.diff_attention(q1, k1, q2, k2, v, lam, W=w.W, scale=w.scale, rows=rows)
     compare(out.reshape(-1, w.dv)[torch.from_numpy(rows).cuda()], ref, "diff workload")
+
+
+def test_diff_decode_workload_first_step(orc):
+    w = WORKLOADS["diff_gqa_decode"]
+    lam = torch.full((w.Hq,), w.lam)
+    out, ref, _, _ = run_diff_decode(orc, w.B, w.Hq, w.Hkv, w.W, w.pos0, 1, seed=0, lam=lam)
+    compare(out, ref, "diff decode workload")
 
 
 def test_decode_workload_first_steps(orc):
