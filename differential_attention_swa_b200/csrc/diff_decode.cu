@@ -1,11 +1,12 @@
 // diff_decode.cu -- one differential-attention decode step over a rolling
 // W-slot cache on sm_100a.
 //
-// "Differential Transformer": two softmax maps, softmax(q1 K1^T s) and
-// softmax(q2 K2^T s), over the same keys, combined as w1 - lambda_h w2 and
-// applied to one V. "Differential Transformer V2" notes that the first
-// version loads the value cache twice per step; here one pass reads every
-// slot's K1, K2 and V bytes exactly once and feeds both maps from them.
+// "Attention Variants -- Sliding Window, Sparse, Differential", The Problem:
+// two softmax maps, softmax(q1 K1^T s) and softmax(q2 K2^T s), over the same
+// keys, one subtracted from the other (w1 - lambda_h w2) and applied to one
+// V. "Attention Variants Compared", symptom table: the first differential
+// version's decode loads the value cache twice per step; here one pass reads
+// every slot's K1, K2 and V bytes exactly once and feeds both maps.
 // The window is the sliding one of "Learn: Sparse & Sliding-Window
 // Attention", section 4: position p lives in slot p % W.
 //

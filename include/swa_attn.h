@@ -151,12 +151,14 @@ swa_status_t swa_sink_decode_step(const void* q, const void* k_new, const void* 
 size_t swa_sink_decode_workspace_bytes(int B, int Hq, int Hkv, int d, int n_sink, int W);
 
 /* One differential-attention decode step over a rolling W-slot cache.
- * ("Differential Transformer": out = sum_j (w1_j - lambda_h w2_j) v_j with
- * w1 = softmax(scale q1 K1^T), w2 = softmax(scale q2 K2^T) over the same
- * window; "Differential Transformer V2" names the first version's double
- * read of the value cache, which this step avoids: every slot's K1, K2 and
- * V bytes are read once. Window as swa_decode_step: "Learn: Sparse &
- * Sliding-Window Attention", section 4.)
+ * ("Attention Variants -- Sliding Window, Sparse, Differential", The Problem:
+ * two attention maps from separate Q/K projections, one subtracted from the
+ * other: out = sum_j (w1_j - lambda_h w2_j) v_j with w1 = softmax(scale q1
+ * K1^T), w2 = softmax(scale q2 K2^T) over the same window. "Attention
+ * Variants Compared", symptom table: the first differential version's
+ * decode loads the value cache twice; here every slot's K1, K2 and V bytes
+ * are read once. Window as swa_decode_step: "Learn: Sparse & Sliding-Window
+ * Attention", section 4.)
  *   q1, q2            device bf16 [B, Hq, d_qk]
  *   k1_new, k2_new    device bf16 [B, Hkv, d_qk]; v_new [B, Hkv, d_v]
  *   k1_cache, k2_cache device bf16 [B, Hkv, W, d_qk]; v_cache [B, Hkv, W, d_v];

@@ -533,8 +533,9 @@ int orc_sink_decode(const float* q, const float* k_new, const float* v_new, floa
 }
 
 /* Differential attention, one decode step per (t, b), over a rolling W-slot
- * cache ("Differential Transformer" reading: two softmax maps over the same
- * keys, combined as w1 - lambda_h w2 and applied to one shared V).
+ * cache ("Attention Variants -- Sliding Window, Sparse, Differential", The
+ * Problem: two softmax maps over the same keys, combined as w1 - lambda_h w2
+ * and applied to one shared V; window as orc_decode).
  * q1, q2: [T,B,Hq,dk]; k1_new, k2_new: [T,B,Hkv,dk]; v_new: [T,B,Hkv,dv];
  * caches k1c, k2c: [B,Hkv,W,dk], vc: [B,Hkv,W,dv], updated in place; lambda:
  * [Hq]. Each step writes its token into slot pos % W, then attends over the
