@@ -33,8 +33,9 @@ _LIB = os.path.join(_HERE, "liboracle.so")
 MASK_SWA = 0
 MASK_STRIDED = 1
 MASK_CAUSAL = 2
+MASK_GLOBAL = 3  # window + global tokens 0 .. g-1; the `stride` argument carries g
 
-_KIND = {"swa": MASK_SWA, "strided": MASK_STRIDED, "causal": MASK_CAUSAL}
+_KIND = {"swa": MASK_SWA, "strided": MASK_STRIDED, "causal": MASK_CAUSAL, "global": MASK_GLOBAL}
 
 
 def build(force: bool = False) -> str:
@@ -294,7 +295,7 @@ STRIDE_TAG = 0x40000000
 
 def schedule_qtile(kind: str, N: int, W: int, S: int, Bq: int, Bk: int, qt: int):
     """(tiles, cells) for one query tile, read off the explicit mask."""
-    cap = (N + Bk - 1) // Bk + ((N + max(S, 1) - 1) // max(S, 1) + Bk - 1) // Bk + 1
+    cap = 2 * ((N + Bk - 1) // Bk) + ((N + max(S, 1) - 1) // max(S, 1) + Bk - 1) // Bk + 1
     tiles = np.empty(cap, dtype=np.int32)
     cells = np.zeros(1, dtype=np.int64)
     n = _L().orc_schedule_qtile(_KIND[kind], N, W, S, Bq, Bk, qt, _p(tiles), cap, _p(cells))

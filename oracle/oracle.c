@@ -11,7 +11,8 @@
  *        strided_mask, the task table (count_nonmasked, tiled_softmax_dot).
  *   [SW] "Learn: Sparse & Sliding-Window Attention": section 3 "The math"
  *        (A = softmax(QK^T/sqrt(d_k) + log M) V, log M in {0, -inf}, dense
- *        causal M_ij = 1[j <= i], band M_ij = 1[i-w < j <= i]); section 4
+ *        causal M_ij = 1[j <= i], band M_ij = 1[i-w < j <= i]); section 3b
+ *        (Longformer: window plus global tokens); section 4
  *        (rolling KV window at decode: keep the last w tokens, evict the
  *        oldest).
  *   [IG] "Exploring Attention Variants: Flash Attention, Sliding-Window, and
@@ -42,6 +43,7 @@
 #define ORC_MASK_SWA 0
 #define ORC_MASK_STRIDED 1
 #define ORC_MASK_CAUSAL 2
+#define ORC_MASK_GLOBAL 3
 
 /* ---------------------------------------------------------------------- */
 /* Masks, one row at a time, in the pages' additive form: 0.0 = attends,  */
@@ -70,9 +72,26 @@ void orc_causal_mask_row(int n, int i, double* row) {
   for (int j = 0; j < n; ++j) row[j] = (j <= i) ? 0.0 : -INFINITY;
 }
 
+/* [SW] section 3b (Longformer): the sliding window plus g global tokens
+ * that attend to everything and are attended to by everything, each adding
+ * a full row and a full column to M. Reading for this causal path: the
+ * global tokens are positions 0 .. g-1 (a [CLS] or question prefix), and
+ * "everything" is every position the causal mask allows. Row i of the
+ * window is taken first, then global column j (j < g, j <= i), then, when
+ * i itself is global, its whole causal row. */
+void orc_global_mask_row(int n, int window, int g, int i, double* row) {
+  orc_swa_mask_row(n, window, i, row);
+  for (int j = 0; j < g && j <= i; ++j) row[j] = 0.0;
+  if (i < g)
+    for (int j = 0; j <= i; ++j) row[j] = 0.0;
+}
+
+/* kind: swa / strided / causal / global; `stride` carries S for strided
+ * and the number of global tokens g for global. */
 void orc_mask_row(int kind, int n, int window, int stride, int i, double* row) {
   if (kind == ORC_MASK_SWA) orc_swa_mask_row(n, window, i, row);
   else if (kind == ORC_MASK_STRIDED) orc_strided_mask_row(n, window, stride, i, row);
+  else if (kind == ORC_MASK_GLOBAL) orc_global_mask_row(n, window, stride, i, row);
   else orc_causal_mask_row(n, i, row);
 }
 
@@ -416,7 +435,11 @@ int orc_decode(const float* q, const float* k_new, const float* v_new, float* k_
 int64_t orc_schedule_qtile(int kind, int N, int W, int S, int Bq, int Bk, int qt, int32_t* tiles,
                            int64_t cap, int64_t* cells) {
   int nkt = (N + Bk - 1) / Bk;
-  int nst = (S > 0) ? ((N + S - 1) / S + Bk - 1) / Bk : 0;
+  /* extra key tiles: stride keys m*S (tile m / Bk) or global keys j < g
+   * (tile j / Bk), tagged 0x40000000 | tile */
+  int nst = 0;
+  if (kind == ORC_MASK_STRIDED && S > 0) nst = ((N + S - 1) / S + Bk - 1) / Bk;
+  if (kind == ORC_MASK_GLOBAL && S > 0) nst = ((S < N ? S : N) + Bk - 1) / Bk;
   uint8_t* band = (uint8_t*)calloc((size_t)nkt + 1, 1);
   uint8_t* strd = (uint8_t*)calloc((size_t)nst + 1, 1);
   double* row = (double*)malloc(sizeof(double) * (size_t)N);
@@ -427,18 +450,23 @@ int64_t orc_schedule_qtile(int kind, int N, int W, int S, int Bq, int Bk, int qt
   if (r1 > N) r1 = N;
   for (int i = r0; i < r1; ++i) {
     orc_mask_row(kind, N, W, S, i, row);
-    /* the window part of the same row: for the strided mask the band is the
-     * swa_mask row (its first loop); for swa/causal the whole row is band */
-    if (kind == ORC_MASK_STRIDED) orc_swa_mask_row(N, W, i, wrow);
+    /* the window part of the same row: for the strided and global masks
+     * the band is the swa_mask row (their first loop); for swa/causal the
+     * whole row is band */
+    const int split = (kind == ORC_MASK_STRIDED || kind == ORC_MASK_GLOBAL);
+    if (split) orc_swa_mask_row(N, W, i, wrow);
     for (int j = 0; j < N; ++j) {
       if (row[j] != 0.0) continue;
       ++c;
-      int in_band = (kind == ORC_MASK_STRIDED) ? (wrow[j] == 0.0) : 1;
+      int in_band = split ? (wrow[j] == 0.0) : 1;
       if (in_band) {
         band[j / Bk] = 1;
-      } else {
+      } else if (kind == ORC_MASK_STRIDED) {
         if (j % S != 0) bad = 1;
         strd[(j / S) / Bk] = 1;
+      } else {
+        if (j >= S) bad = 1; /* outside the window only global keys may be attended */
+        strd[j / Bk] = 1;
       }
     }
   }

@@ -177,6 +177,8 @@ def sdpa_ref(q, k, v, allowed, scale):
     ("strided", 1, 2, 1, 150, 16, 16, 7, 11),
     ("strided", 2, 4, 4, 97, 8, 8, 3, 1),
     ("causal", 1, 3, 1, 55, 16, 16, 0, 0),
+    ("global", 1, 4, 2, 140, 16, 16, 9, 5),
+    ("global", 2, 2, 2, 70, 8, 24, 3, 40),
 ])
 def test_attention_matches_torch_sdpa_fp64(orc, kind, B, Hq, Hkv, N, d, dv, W, S):
     q, k, v = attn_inputs(B, Hq, Hkv, N, d, dv, seed=11)
@@ -189,6 +191,8 @@ def test_attention_matches_torch_sdpa_fp64(orc, kind, B, Hq, Hkv, N, d, dv, W, S
         allowed = (ii - W < jj) & (jj <= ii)
         if kind == "strided":
             allowed |= (jj % S == 0) & (jj <= ii)
+        if kind == "global":  # S carries the number of global tokens
+            allowed |= ((jj < S) | (ii < S)) & (jj <= ii)
     ref = sdpa_ref(q, k, v, allowed, scale)
     assert np.abs(out - ref).max() < 1e-12
     # natural-log sum of exp over the attended scores
@@ -282,7 +286,7 @@ def test_decode_equals_window_softmax_over_history(orc, W, pos0, T):
 
 # --------------------------------------------------------------- schedule --
 
-def tiles_touched_from_mask(allowed, band_allowed, Bq, Bk, S):
+def tiles_touched_from_mask(allowed, band_allowed, Bq, Bk, S, global_keys=False):
     """Block-reduce boolean masks: which key tiles / stride tiles hold an
     attended cell for each query tile."""
     N = allowed.shape[0]
@@ -291,7 +295,8 @@ def tiles_touched_from_mask(allowed, band_allowed, Bq, Bk, S):
         rows = slice(qt * Bq, min(N, qt * Bq + Bq))
         a, b = allowed[rows], band_allowed[rows]
         extra = a & ~b
-        st = sorted({(j // S) // Bk for j in np.nonzero(extra.any(0))[0]}) if S else []
+        unit = 1 if global_keys else S  # global keys are tiled as they are; stride keys m*S compacted
+        st = sorted({(j // unit) // Bk for j in np.nonzero(extra.any(0))[0]}) if S else []
         kt = sorted({j // Bk for j in np.nonzero(b.any(0))[0]})
         out.append(([0x40000000 | t for t in st] + kt, int(a.sum())))
     return out
@@ -300,7 +305,8 @@ def tiles_touched_from_mask(allowed, band_allowed, Bq, Bk, S):
 @pytest.mark.parametrize("kind,N,W,S,Bq,Bk", [
     ("swa", 256, 64, 0, 128, 128), ("strided", 256, 16, 8, 128, 128), ("swa", 300, 50, 0, 64, 32),
     ("strided", 517, 33, 5, 128, 16), ("swa", 100, 1000, 0, 32, 32), ("strided", 130, 1, 1, 64, 64),
-    ("causal", 200, 0, 0, 64, 32)])
+    ("causal", 200, 0, 0, 64, 32), ("global", 256, 16, 8, 128, 128), ("global", 517, 33, 200, 128, 16),
+    ("global", 300, 64, 300, 64, 32), ("global", 130, 1, 1, 64, 64)])
 def test_schedule_matches_block_reduction(orc, kind, N, W, S, Bq, Bk):
     ii, jj = np.meshgrid(np.arange(N), np.arange(N), indexing="ij")
     if kind == "causal":
@@ -308,9 +314,13 @@ def test_schedule_matches_block_reduction(orc, kind, N, W, S, Bq, Bk):
         band = allowed
     else:
         band = (ii - W < jj) & (jj <= ii)
-        allowed = band | ((jj % S == 0) & (jj <= ii)) if kind == "strided" else band
+        allowed = band
+        if kind == "strided":
+            allowed = band | ((jj % S == 0) & (jj <= ii))
+        if kind == "global":
+            allowed = band | (((jj < S) | (ii < S)) & (jj <= ii))
     lists, cells = orc.schedule(kind, N, W, S, Bq, Bk)
-    want = tiles_touched_from_mask(allowed, band, Bq, Bk, S)
+    want = tiles_touched_from_mask(allowed, band, Bq, Bk, S, global_keys=(kind == "global"))
     assert lists == [w[0] for w in want]
     assert cells == [w[1] for w in want]
     assert sum(cells) == int(allowed.sum())
@@ -492,3 +502,56 @@ def test_diff_decode_with_lambda_zero_is_the_plain_decode(orc):
     ref, kr, vr = orc.decode(q1, k1n, vn, k1c, vc, pos)
     assert np.abs(out - ref).max() < 1e-12
     assert np.array_equal(k1a, kr) and np.array_equal(va, vr)
+
+
+
+# ------------------------------------------------------- global tokens -----
+
+def global_closed(N, W, g):
+    # per row: min(i+1, W) window keys plus the global keys below the window
+    i = np.arange(N, dtype=np.int64)
+    lo = np.maximum(0, i - W + 1)
+    return int(np.minimum(i + 1, W).sum() + np.minimum(g, lo).sum())
+
+
+def test_global_mask_8_2_3_matches_hand_derived_grid(orc):
+    M = orc.mask("global", 8, 2, 3)
+    assert grid_of(M) == read_grid("global_mask_n8_w2_g3.txt")
+    assert orc.count_nonmasked(M) == 30 == global_closed(8, 2, 3)
+
+
+def test_global_mask_brute_force_all_small(orc):
+    """Against the predicate j <= i and (i - W < j or j < g or i < g), for
+    every n <= 20, every window and every number of global tokens; the
+    count against the closed form."""
+    for n in range(1, 21):
+        ii, jj = np.meshgrid(np.arange(n), np.arange(n), indexing="ij")
+        for W in range(1, n + 2):
+            for g in range(0, n + 2):
+                want = (jj <= ii) & ((ii - W < jj) | (jj < g) | (ii < g))
+                M = orc.mask("global", n, W, g)
+                assert np.array_equal(M == 0.0, want), (n, W, g)
+                assert orc.count_nonmasked(M) == global_closed(n, W, g), (n, W, g)
+
+
+def test_global_mask_special_cases(orc):
+    n, W = 40, 6
+    assert np.array_equal(orc.mask("global", n, W, 0), orc.swa_mask(n, W))  # no global token
+    assert np.array_equal(orc.mask("global", n, W, 1), orc.strided_mask(n, W, n + 5))  # only key 0
+    for g in (n, n + 3):
+        assert np.array_equal(orc.mask("global", n, W, g), orc.causal_mask(n))
+    assert np.array_equal(orc.mask("global", n, n, 7), orc.causal_mask(n))
+
+
+@pytest.mark.parametrize("n_sink,W,pos", [(4, 8, 3), (4, 8, 9), (4, 8, 40), (2, 16, 17), (1, 5, 30)])
+def test_global_prefill_row_equals_sink_decode_step(orc, n_sink, W, pos):
+    """A decode step with n_sink attention sinks and a W-token window sees
+    exactly row pos of the window + global-token mask with g = n_sink: the
+    two oracle functions are written separately and must agree."""
+    B, Hq, Hkv, d = 1, 4, 2, 16
+    Kh, Vh, q, kc, vc, k_new, v_new, posarr = _sink_history(B, Hkv, Hq, d, n_sink, W, pos, 1, 90)
+    dec, _, _ = orc.sink_decode(q, k_new, v_new, kc, vc, posarr, n_sink)
+    Q = torch.zeros(B, Hq, pos + 1, d)
+    Q[:, :, pos] = q[0]
+    pre = orc.attention("global", Q, Kh, Vh, W=W, S=n_sink, scale=0.25)
+    assert np.abs(pre[:, :, pos] - dec[0]).max() < 1e-12
