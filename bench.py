@@ -211,6 +211,9 @@ def prefill_workload(name, rank):
         if w.kind == "swa":
             fn = lambda: swa.swa_attn_fwd(q, k, v, w.W, out=out)
             nnz = swa.count_nonmasked(swa.MASK_WINDOW, w.N, w.W)
+        elif w.kind == "global":  # S carries the number of global tokens
+            fn = lambda: swa.global_attn_fwd(q, k, v, w.W, w.S, out=out)
+            nnz = swa.count_nonmasked(swa.MASK_GLOBAL, w.N, w.W, w.S)
         else:
             fn = lambda: swa.strided_attn_fwd(q, k, v, w.W, w.S, out=out)
             nnz = swa.count_nonmasked(swa.MASK_STRIDED, w.N, w.W, w.S)
@@ -421,7 +424,7 @@ def measure_variants(args, rank, peaks, flush, stream):
 
     out = {}
     reps = max(5, min(args.steps, 10))
-    for name in ("local_strided_prefill", "diff_causal", "gemma_swa_prefill"):
+    for name in ("local_strided_prefill", "diff_causal", "gemma_swa_prefill", "longformer_global_prefill"):
         w, fn, flops, ins, o = prefill_workload(name, rank)
         ms = time_steps(fn, reps, 3, flush, stream)
         mean_ms = sum(ms) / len(ms)

@@ -20,12 +20,12 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libswa_attn.so")
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT = range(5)
-MASK_WINDOW, MASK_STRIDED, MASK_CAUSAL = 0, 1, 2
+MASK_WINDOW, MASK_STRIDED, MASK_CAUSAL, MASK_GLOBAL = 0, 1, 2, 3
 STRIDE_TAG = 0x40000000
 TILE = 128  # query rows and keys per tile in the prefill kernels
 
 __all__ = [
-    "swa_attn_fwd", "strided_attn_fwd", "diff_attn_fwd", "swa_decode_step", "decode_workspace_bytes",
+    "swa_attn_fwd", "strided_attn_fwd", "global_attn_fwd", "diff_attn_fwd", "swa_decode_step", "decode_workspace_bytes",
     "swa_sink_decode_step", "sink_decode_workspace_bytes", "swa_diff_decode_step", "diff_decode_workspace_bytes",
     "prefill_debug", "schedule", "count_nonmasked", "last_device_error", "SwaError", "library",
 ]
@@ -56,6 +56,8 @@ def library() -> ctypes.CDLL:
     P, I, F, I64, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_int64, ctypes.c_size_t
     lib.swa_attn_fwd.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, P]
     lib.strided_attn_fwd.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, F, P]
+    lib.global_attn_fwd.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, F, P]
+    lib.global_attn_fwd.restype = I
     lib.diff_attn_fwd.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, F, P]
     lib.swa_decode_step.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, F, P, SZ, P]
     lib.swa_decode_workspace_bytes.argtypes = [I, I, I, I, I]
@@ -144,6 +146,18 @@ def strided_attn_fwd(q, k, v, window: int, stride: int, scale: float | None = No
     st = library().strided_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, N, d,
                                     int(window), int(stride), float(scale), _stream(stream))
     _raise(st, "strided_attn_fwd")
+    return (out, lse) if return_lse else out
+
+
+def global_attn_fwd(q, k, v, window: int, n_global: int, scale: float | None = None, out=None,
+                    return_lse: bool = False, stream=None):
+    """Window + global tokens: the window OR keys j < n_global (positions
+    0 .. n_global-1 are the global tokens), j <= i."""
+    B, Hq, Hkv, N, d, out, lse = _prefill_common(q, k, v, out, return_lse)
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    st = library().global_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, N, d,
+                                   int(window), int(n_global), float(scale), _stream(stream))
+    _raise(st, "global_attn_fwd")
     return (out, lse) if return_lse else out
 
 

@@ -74,6 +74,7 @@ swa_status_t run_prefill(int kind, bool diff, const void* q, const void* k, cons
   if (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)) return SWA_ERR_INVALID_ARG;
   if (B < 1 || Hq < 1 || Hkv < 1 || N < 1 || W < 1 || Hq % Hkv != 0) return SWA_ERR_INVALID_ARG;
   if (kind == kMaskStrided && S < 1) return SWA_ERR_INVALID_ARG;
+  if (kind == kMaskGlobal && S < 0) return SWA_ERR_INVALID_ARG;
   if (!(scale > 0.f) || !std::isfinite(scale)) return SWA_ERR_INVALID_ARG;
   if ((int64_t)B * Hq > (1 << 30) / 8) return SWA_ERR_INVALID_ARG;
   if (!head_dim_ok(dqk) || !head_dim_ok(dv)) return SWA_ERR_UNSUPPORTED;
@@ -101,11 +102,13 @@ swa_status_t run_prefill(int kind, bool diff, const void* q, const void* k, cons
   }
   if (!ok) return SWA_ERR_INVALID_ARG;
   if (!diff) maps.q2 = maps.q, maps.k2 = maps.k;
+  // global keys are the first rows of K/V themselves: the extra view is K/V
   if (kind != kMaskStrided) maps.ks = maps.k, maps.vs = maps.v;
 
   PrefillParams p;
   std::memset(&p, 0, sizeof(p));
-  p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.N = N; p.W = W; p.S = (kind == kMaskStrided) ? S : 0;
+  p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.N = N; p.W = W;
+  p.S = (kind == kMaskStrided || kind == kMaskGlobal) ? S : 0;  // stride, or number of global tokens
   p.G = G; p.kind = kind;
   p.nq = (N + 127) / 128;
   p.scale_log2 = scale * 1.4426950408889634f;
@@ -209,6 +212,13 @@ swa_status_t strided_attn_fwd(const void* q, const void* k, const void* v, void*
                      stride, scale, nullptr, stream);
 }
 
+swa_status_t global_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                             int Hkv, int N, int d, int W, int n_global, float scale, void* stream) {
+  if (n_global < 0) return SWA_ERR_INVALID_ARG;
+  return run_prefill(kMaskGlobal, false, q, k, nullptr, nullptr, v, o, lse, nullptr, B, Hq, Hkv, N, d, d, W,
+                     n_global, scale, nullptr, stream);
+}
+
 swa_status_t diff_attn_fwd(const void* q1, const void* k1, const void* q2, const void* k2, const void* v, void* o,
                            const float* lambda, int B, int Hq, int Hkv, int N, int d_qk, int d_v, int W, float scale,
                            void* stream) {
@@ -219,7 +229,7 @@ swa_status_t diff_attn_fwd(const void* q1, const void* k1, const void* q2, const
 swa_status_t swa_prefill_debug(int kind, const void* q, const void* k, const void* v, void* o, float* lse, int B,
                                int Hq, int Hkv, int N, int d, int W, int stride, float scale, const swa_debug_t* dbg,
                                void* stream) {
-  if (kind != kMaskWindow && kind != kMaskStrided) return SWA_ERR_INVALID_ARG;
+  if (kind != kMaskWindow && kind != kMaskStrided && kind != kMaskGlobal) return SWA_ERR_INVALID_ARG;
   return run_prefill(kind, false, q, k, nullptr, nullptr, v, o, lse, nullptr, B, Hq, Hkv, N, d, d, W, stride, scale,
                      dbg, stream);
 }
@@ -280,9 +290,10 @@ swa_status_t swa_diff_decode_step(const void* q1, const void* q2, const void* k1
 
 int64_t swa_schedule(int kind, int N, int W, int stride, int Bq, int Bk, int32_t* qtile_offsets, int32_t* tiles,
                      int64_t cap) {
-  if (N < 1 || Bq < 1 || Bk < 1 || kind < 0 || kind > 2) return -1;
+  if (N < 1 || Bq < 1 || Bk < 1 || kind < 0 || kind > 3) return -1;
   if (kind != kMaskCausal && W < 1) return -1;
   if (kind == kMaskStrided && stride < 1) return -1;
+  if (kind == kMaskGlobal && stride < 0) return -1;
   const int nq = (N + Bq - 1) / Bq;
   int64_t n = 0;
   for (int qt = 0; qt < nq; ++qt) {
@@ -297,9 +308,10 @@ int64_t swa_schedule(int kind, int N, int W, int stride, int Bq, int Bk, int32_t
 }
 
 int64_t swa_count_nonmasked(int kind, int N, int W, int stride) {
-  if (N < 0 || kind < 0 || kind > 2) return -1;
+  if (N < 0 || kind < 0 || kind > 3) return -1;
   if (kind != kMaskCausal && W < 1) return -1;
   if (kind == kMaskStrided && stride < 1) return -1;
+  if (kind == kMaskGlobal && stride < 0) return -1;
   if (N == 0) return 0;
   return count_attended(kind, N, W, stride);
 }

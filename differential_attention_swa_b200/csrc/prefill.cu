@@ -510,7 +510,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int i = un.qt[t] * BM + r;  // query index
       const bool row_ok = i < p.N;
       const int lo = window_lo(i, Wc);
-      const int mst = (p.kind == kMaskStrided) ? stride_rows_below(lo, p.S) : 0;
+      const int mst = extra_rows_below(p.kind, lo, p.S);  // extra-view rows (stride or global keys) below lo
       float m_run = -INFINITY;  // running max, log2 units (scores * scale * log2 e)
       float l_run = 0.f;
       long long cells = 0;

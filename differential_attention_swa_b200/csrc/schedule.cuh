@@ -9,12 +9,18 @@
 // Variants Compared", swa_mask / strided_mask code):
 //   window:  key j attended by row i iff  lo_i <= j <= i,  lo_i = max(0, i-W+1)
 //   strided: window OR (j % S == 0 and j <= i).
-// A cell outside the window is a stride cell iff j % S == 0 and j < lo_i, so
-// the union splits into disjoint window cells and stride cells, and each
-// attended cell is visited exactly once.
+//   global:  window OR j < g OR i < g, with j <= i ("Learn: Sparse &
+//            Sliding-Window Attention", section 3b, Longformer's global
+//            tokens, here positions 0 .. g-1; a global row i < g attends
+//            keys j <= i < g, all of them global, so it needs no own term).
+// A cell outside the window is an "extra" cell iff it is a stride key
+// (j % S == 0) or a global key (j < g) below lo_i, so the union splits into
+// disjoint window cells and extra cells, and each attended cell is visited
+// exactly once.
 //
-// Stride cells are gathered by a strided view of K/V: stride row m holds key
-// m*S. A "stride tile" ct holds stride rows ct*Bk .. ct*Bk+Bk-1.
+// Extra cells are read through a second view of K/V whose row m holds key
+// m*S (strided) or key m (global: the global keys are the first g rows). An
+// "extra tile" ct holds rows ct*Bk .. ct*Bk+Bk-1 of that view.
 #pragma once
 
 #ifdef __CUDACC__
@@ -27,7 +33,7 @@ namespace swa {
 
 constexpr int kStrideTag = 0x40000000;
 
-enum MaskKind { kMaskWindow = 0, kMaskStrided = 1, kMaskCausal = 2 };
+enum MaskKind { kMaskWindow = 0, kMaskStrided = 1, kMaskCausal = 2, kMaskGlobal = 3 };
 
 SWA_HD int imin(int a, int b) { return a < b ? a : b; }
 SWA_HD int imax(int a, int b) { return a > b ? a : b; }
@@ -39,6 +45,14 @@ SWA_HD int window_lo(int i, int W) { return imax(0, i - W + 1); }
 // whose window starts at lo).
 SWA_HD int stride_rows_below(int lo, int S) { return (lo + S - 1) / S; }
 
+// Extra-view rows attended by a row whose window starts at lo: stride rows
+// below lo (strided), the global keys below lo (global; S carries g).
+SWA_HD int extra_rows_below(int kind, int lo, int S) {
+  if (kind == kMaskStrided && S > 0) return stride_rows_below(lo, S);
+  if (kind == kMaskGlobal && S > 0) return imin(S, lo);
+  return 0;
+}
+
 struct QTileKeys {
   int band_lo;   // first window key tile
   int band_hi;   // last window key tile
@@ -49,8 +63,8 @@ struct QTileKeys {
 // (or kind == causal) is full causal. The window part is the contiguous
 // range from the tile holding the first row's lo to the tile holding the
 // last row; every tile in it has an attended cell because consecutive rows'
-// windows overlap or abut. Stride tiles are those with a stride row below
-// the last row's lo (the largest lo in the tile).
+// windows overlap or abut. Extra tiles are those with an extra-view row
+// below the last row's lo (the largest lo in the tile).
 SWA_HD QTileKeys qtile_keys(int kind, int N, int W, int S, int Bq, int Bk, int qt) {
   QTileKeys r;
   const int r0 = qt * Bq;
@@ -58,11 +72,8 @@ SWA_HD QTileKeys qtile_keys(int kind, int N, int W, int S, int Bq, int Bk, int q
   const int Wc = (kind == kMaskCausal) ? N : W;
   r.band_lo = window_lo(r0, Wc) / Bk;
   r.band_hi = r1 / Bk;
-  r.n_stride = 0;
-  if (kind == kMaskStrided && S > 0) {
-    const int m = stride_rows_below(window_lo(r1, Wc), S);
-    r.n_stride = (m + Bk - 1) / Bk;
-  }
+  const int m = extra_rows_below(kind, window_lo(r1, Wc), S);
+  r.n_stride = (m + Bk - 1) / Bk;
   return r;
 }
 
@@ -83,6 +94,12 @@ SWA_HD long long count_attended(int kind, int N, int W, int S) {
   }
   long long n = N, w = W;
   long long band = n * w - w * (w - 1) / 2;
+  if (kind == kMaskGlobal && S > 0) {
+    // rows i >= W have lo_i = t for t = 1 .. N-W and add min(g, t) keys
+    const long long T = n - w, g = S;
+    if (T <= g) return band + T * (T + 1) / 2;
+    return band + g * (g + 1) / 2 + (T - g) * g;
+  }
   if (kind != kMaskStrided || S <= 0) return band;
   // stride cells: sum over rows i >= W of ceil((i - W + 1) / S)
   // = sum over t = 1 .. N-W of ceil(t / S)

@@ -92,6 +92,21 @@ swa_status_t strided_attn_fwd(const void* q, const void* k, const void* v, void*
                               int B, int Hq, int Hkv, int N, int d, int W, int stride,
                               float scale, void* stream);
 
+/* Window + global-token attention forward: row i attends key j <= i when
+ * i - W < j (the window) or j < n_global (a global token) or i < n_global
+ * (a global row). Source: "Learn: Sparse & Sliding-Window Attention",
+ * section 3b (Longformer: global tokens attend to everything and are
+ * attended to by everything, a full row and column of M each; cost
+ * O(s w + s g)) and section 6 (window + global FLOPs). The pages do not
+ * place the global tokens; this library takes positions 0 .. n_global-1
+ * (a [CLS] or question prefix), where a global row's causal keys are all
+ * global. Extra (global) keys below a row's window are visited as whole
+ * 128-key tiles of K/V, before the window tiles; every cell counts once.
+ *   Arguments as swa_attn_fwd, plus n_global >= 0 (0 is swa_attn_fwd). */
+swa_status_t global_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                             int B, int Hq, int Hkv, int N, int d, int W, int n_global,
+                             float scale, void* stream);
+
 /* Differential attention forward:
  *     o = softmax(Q1 K1^T * scale + log M) V - lambda[h] * softmax(Q2 K2^T * scale + log M) V
  * over one shared V, both maps under the same window mask (W >= N: causal).
@@ -209,15 +224,17 @@ swa_status_t swa_decode_step_static(const void* q, const void* k_new, const void
                                     void* stream);
 
 /* Prefill with debug outputs. kind 0 = sliding window (stride ignored),
- * kind 1 = local + strided. Same arithmetic as swa_attn_fwd /
- * strided_attn_fwd; dbg may be NULL. */
+ * kind 1 = local + strided, kind 3 = window + global tokens (stride carries
+ * n_global). Same arithmetic as swa_attn_fwd / strided_attn_fwd /
+ * global_attn_fwd; dbg may be NULL. */
 swa_status_t swa_prefill_debug(int kind, const void* q, const void* k, const void* v, void* o,
                                float* lse, int B, int Hq, int Hkv, int N, int d, int W,
                                int stride, float scale, const swa_debug_t* dbg, void* stream);
 
 /* The key tiles each query tile visits, as the kernels enumerate them
  * (host only; the kernels call the same function). kind 0 = window,
- * 1 = window + stride, 2 = full causal. Query tiles are Bq rows, key tiles
+ * 1 = window + stride, 2 = full causal, 3 = window + global tokens (stride
+ * carries n_global >= 0; extra tiles hold keys ct*Bk .. ct*Bk+Bk-1). Query tiles are Bq rows, key tiles
  * Bk keys (the kernels use 128 x 128). qtile_offsets [nq + 1] receives the
  * start of each query tile's list in `tiles`; tiles receives up to cap
  * entries in the encoding of swa_debug_t. Returns the total number of
@@ -230,7 +247,7 @@ int64_t swa_schedule(int kind, int N, int W, int stride, int Bq, int Bk, int32_t
                      int32_t* tiles, int64_t cap);
 
 /* ||M||_0, the attended cells of one (b, head) N x N mask, in closed form
- * (kind as swa_schedule; stride ignored unless kind == 1). -1 on bad
+ * (kind as swa_schedule; stride ignored unless kind is 1 or 3). -1 on bad
  * arguments. Source: "Attention Variants Compared", count_nonmasked. */
 int64_t swa_count_nonmasked(int kind, int N, int W, int stride);
 

@@ -51,7 +51,8 @@ def test_library_exports_every_declared_symbol(lib):
 @pytest.mark.parametrize("kind,okind,N,W,S", [
     (0, "swa", 256, 64, 0), (1, "strided", 256, 16, 8), (0, "swa", 1000, 130, 0), (1, "strided", 1000, 1, 1),
     (1, "strided", 777, 200, 7), (0, "swa", 129, 5000, 0), (1, "strided", 300, 17, 400), (2, "causal", 513, 0, 0),
-    (0, "swa", 1, 1, 0), (1, "strided", 4000, 128, 128)])
+    (0, "swa", 1, 1, 0), (1, "strided", 4000, 128, 128), (3, "global", 256, 16, 8), (3, "global", 1000, 130, 300),
+    (3, "global", 777, 64, 0), (3, "global", 500, 600, 40), (3, "global", 4000, 512, 64), (3, "global", 300, 1, 1)])
 def test_schedule_export_bit_exact_vs_oracle(lib, orc, kind, okind, N, W, S):
     got = swa.schedule(kind, N, W, S)
     want, _ = orc.schedule(okind, N, W, S, 128, 128)
@@ -73,7 +74,9 @@ def test_schedule_sampled_at_workload_sizes(lib, orc):
 
 @pytest.mark.parametrize("kind,okind,N,W,S", [
     (0, "swa", 256, 64, 0), (1, "strided", 256, 16, 8), (1, "strided", 300, 17, 5), (0, "swa", 50, 50, 0),
-    (0, "swa", 50, 1, 0), (1, "strided", 97, 3, 1), (1, "strided", 97, 200, 3), (2, "causal", 70, 0, 0)])
+    (0, "swa", 50, 1, 0), (1, "strided", 97, 3, 1), (1, "strided", 97, 200, 3), (2, "causal", 70, 0, 0),
+    (3, "global", 256, 16, 8), (3, "global", 300, 17, 200), (3, "global", 97, 3, 0), (3, "global", 97, 200, 5),
+    (3, "global", 130, 9, 130)])
 def test_count_nonmasked_closed_form_vs_oracle(lib, orc, kind, okind, N, W, S):
     M = orc.mask(okind, N, W, S)
     assert swa.count_nonmasked(kind, N, W, S) == orc.count_nonmasked(M)

@@ -17,7 +17,7 @@ pytestmark = pytest.mark.gpu
 
 MAX_TOL = 1e-2
 MEAN_TOL = 2e-3
-KIND = {"swa": swa.MASK_WINDOW, "strided": swa.MASK_STRIDED}
+KIND = {"swa": swa.MASK_WINDOW, "strided": swa.MASK_STRIDED, "global": swa.MASK_GLOBAL}
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -46,6 +46,8 @@ def run_prefill(kind, q, k, v, W, S, lse=False):
     qd, kd, vd = gpu(q, k, v)
     if kind == "swa":
         r = swa.swa_attn_fwd(qd, kd, vd, W, return_lse=lse)
+    elif kind == "global":  # S carries the number of global tokens
+        r = swa.global_attn_fwd(qd, kd, vd, W, S, return_lse=lse)
     else:
         r = swa.strided_attn_fwd(qd, kd, vd, W, S, return_lse=lse)
     assert swa.last_device_error() == swa.OK
@@ -79,6 +81,13 @@ EDGE = [
     ("strided", 1, 2, 2, 333, 64, 20, 400), # stride beyond N: window + key 0
     ("strided", 1, 4, 2, 1000, 128, 64, 7), # group 2 with stride tiles
     ("strided", 1, 2, 2, 700, 64, 1, 3),    # window 1 + stride
+    ("global", 1, 2, 2, 700, 64, 64, 50),   # global keys in a partial tile
+    ("global", 1, 2, 2, 900, 64, 100, 300), # global tokens span several tiles and the window
+    ("global", 1, 4, 2, 1000, 128, 64, 128),# group 2, one whole global tile
+    ("global", 1, 6, 2, 513, 128, 40, 7),   # group 3 (tile pairs), ragged
+    ("global", 1, 2, 2, 300, 64, 5000, 9),  # window beyond N: full causal
+    ("global", 1, 2, 2, 400, 64, 16, 0),    # no global token: the window
+    ("global", 1, 2, 2, 333, 64, 1, 1000),  # every token global: full causal
 ]
 
 
@@ -92,7 +101,8 @@ def test_edge_cases_full(orc, kind, B, Hq, Hkv, N, d, W, S):
 
 @pytest.mark.parametrize("kind,N,W,S,Hq,Hkv,d", [
     ("swa", 256, 64, 0, 2, 2, 64), ("strided", 256, 16, 8, 2, 2, 64), ("swa", 1000, 300, 0, 4, 2, 128),
-    ("strided", 1500, 100, 9, 2, 2, 64), ("swa", 385, 5000, 0, 3, 1, 64), ("strided", 2048, 128, 128, 2, 1, 64)])
+    ("strided", 1500, 100, 9, 2, 2, 64), ("swa", 385, 5000, 0, 3, 1, 64), ("strided", 2048, 128, 128, 2, 1, 64),
+    ("global", 1500, 100, 300, 2, 2, 64), ("global", 1000, 512, 64, 4, 2, 128), ("global", 777, 64, 0, 3, 1, 64)])
 def test_visited_tiles_and_cells_bit_exact(orc, kind, N, W, S, Hq, Hkv, d):
     q, k, v = attn_inputs(1, Hq, Hkv, N, d, seed=7)
     qd, kd, vd = gpu(q, k, v)
@@ -211,7 +221,8 @@ def sampled_rows(B, H, N, n, seed):
     return np.unique(bh.astype(np.int64) * N + i)
 
 
-@pytest.mark.parametrize("name", ["mistral_swa_prefill", "local_strided_prefill", "gemma_swa_prefill"])
+@pytest.mark.parametrize("name", ["mistral_swa_prefill", "local_strided_prefill", "gemma_swa_prefill",
+                                  "longformer_global_prefill"])
 def test_workload_sampled_rows(orc, name):
     w = WORKLOADS[name]
     q, k, v = attn_inputs(w.B, w.Hq, w.Hkv, w.N, w.d, seed=0)
