@@ -34,8 +34,10 @@ MASK_SWA = 0
 MASK_STRIDED = 1
 MASK_CAUSAL = 2
 MASK_GLOBAL = 3  # window + global tokens 0 .. g-1; the `stride` argument carries g
+MASK_DILATED = 4  # window of W keys spaced by the dilation; the `stride` argument carries it
 
-_KIND = {"swa": MASK_SWA, "strided": MASK_STRIDED, "causal": MASK_CAUSAL, "global": MASK_GLOBAL}
+_KIND = {"swa": MASK_SWA, "strided": MASK_STRIDED, "causal": MASK_CAUSAL, "global": MASK_GLOBAL,
+         "dilated": MASK_DILATED}
 
 
 def build(force: bool = False) -> str:

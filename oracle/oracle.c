@@ -44,6 +44,7 @@
 #define ORC_MASK_STRIDED 1
 #define ORC_MASK_CAUSAL 2
 #define ORC_MASK_GLOBAL 3
+#define ORC_MASK_DILATED 4
 
 /* ---------------------------------------------------------------------- */
 /* Masks, one row at a time, in the pages' additive form: 0.0 = attends,  */
@@ -86,12 +87,27 @@ void orc_global_mask_row(int n, int window, int g, int i, double* row) {
     for (int j = 0; j <= i; ++j) row[j] = 0.0;
 }
 
-/* kind: swa / strided / causal / global; `stride` carries S for strided
- * and the number of global tokens g for global. */
+/* [SW] section 3b (Longformer): dilation puts gaps of size d_dil inside
+ * the window, so the same budget of allowed keys reaches d_dil times
+ * further. Reading: the W keys i, i - dil, i - 2 dil, ..., i - (W-1) dil
+ * (those >= 0); dil = 1 is the plain window. */
+void orc_dilated_mask_row(int n, int window, int dil, int i, double* row) {
+  for (int j = 0; j < n; ++j) row[j] = -INFINITY;
+  for (int k = 0; k < window; ++k) {
+    const int64_t j = (int64_t)i - (int64_t)k * dil;
+    if (j < 0) break;
+    row[j] = 0.0;
+  }
+}
+
+/* kind: swa / strided / causal / global / dilated; `stride` carries S for
+ * strided, the number of global tokens g for global, the dilation for
+ * dilated. */
 void orc_mask_row(int kind, int n, int window, int stride, int i, double* row) {
   if (kind == ORC_MASK_SWA) orc_swa_mask_row(n, window, i, row);
   else if (kind == ORC_MASK_STRIDED) orc_strided_mask_row(n, window, stride, i, row);
   else if (kind == ORC_MASK_GLOBAL) orc_global_mask_row(n, window, stride, i, row);
+  else if (kind == ORC_MASK_DILATED) orc_dilated_mask_row(n, window, stride, i, row);
   else orc_causal_mask_row(n, i, row);
 }
 
@@ -434,6 +450,7 @@ int orc_decode(const float* q, const float* k_new, const float* v_new, float* k_
  * -2 if an outside-window cell is not a multiple of S. */
 int64_t orc_schedule_qtile(int kind, int N, int W, int S, int Bq, int Bk, int qt, int32_t* tiles,
                            int64_t cap, int64_t* cells) {
+  if (kind == ORC_MASK_DILATED) return -3; /* visited per residue class, as window masks */
   int nkt = (N + Bk - 1) / Bk;
   /* extra key tiles: stride keys m*S (tile m / Bk) or global keys j < g
    * (tile j / Bk), tagged 0x40000000 | tile */

@@ -555,3 +555,51 @@ def test_global_prefill_row_equals_sink_decode_step(orc, n_sink, W, pos):
     Q[:, :, pos] = q[0]
     pre = orc.attention("global", Q, Kh, Vh, W=W, S=n_sink, scale=0.25)
     assert np.abs(pre[:, :, pos] - dec[0]).max() < 1e-12
+
+
+# ------------------------------------------------------ dilated window -----
+
+def dilated_closed(N, W, dil):
+    # row i attends min(W, floor(i / dil) + 1) keys
+    i = np.arange(N, dtype=np.int64)
+    return int(np.minimum(W, i // dil + 1).sum())
+
+
+def test_dilated_mask_brute_force_all_small(orc):
+    """Against the predicate j <= i, (i - j) % dil == 0, (i - j) / dil < W,
+    for every n <= 20, window and dilation; count against the closed form."""
+    for n in range(1, 21):
+        ii, jj = np.meshgrid(np.arange(n), np.arange(n), indexing="ij")
+        for W in range(1, n + 2):
+            for dil in range(1, n + 2):
+                want = (jj <= ii) & ((ii - jj) % dil == 0) & ((ii - jj) // dil < W)
+                M = orc.mask("dilated", n, W, dil)
+                assert np.array_equal(M == 0.0, want), (n, W, dil)
+                assert orc.count_nonmasked(M) == dilated_closed(n, W, dil)
+
+
+def test_dilation_one_is_the_window(orc):
+    for n, W in ((40, 6), (17, 17), (9, 30)):
+        assert np.array_equal(orc.mask("dilated", n, W, 1), orc.swa_mask(n, W))
+
+
+@pytest.mark.parametrize("n,W,dil", [(50, 4, 3), (64, 7, 2), (33, 5, 4), (20, 30, 6)])
+def test_dilated_mask_is_dil_interleaved_windows(orc, n, W, dil):
+    """Rows and keys of one residue class mod dil form a plain window mask of
+    W keys on that subsequence; keys of other classes are never attended.
+    The kernels rest on this decomposition."""
+    M = orc.mask("dilated", n, W, dil)
+    ii, jj = np.meshgrid(np.arange(n), np.arange(n), indexing="ij")
+    assert np.all(M[(ii - jj) % dil != 0] == -np.inf)
+    for r in range(dil):
+        idx = np.arange(r, n, dil)
+        assert np.array_equal(M[np.ix_(idx, idx)], orc.swa_mask(idx.size, W))
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,N,d,W,dil", [(1, 2, 1, 90, 16, 5, 3), (2, 4, 4, 64, 8, 9, 2)])
+def test_dilated_attention_matches_torch_sdpa_fp64(orc, B, Hq, Hkv, N, d, W, dil):
+    q, k, v = attn_inputs(B, Hq, Hkv, N, d, seed=13)
+    out = orc.attention("dilated", q, k, v, W=W, S=dil, scale=0.25)
+    ii, jj = np.meshgrid(np.arange(N), np.arange(N), indexing="ij")
+    allowed = (jj <= ii) & ((ii - jj) % dil == 0) & ((ii - jj) // dil < W)
+    assert np.abs(out - sdpa_ref(q, k, v, allowed, 0.25)).max() < 1e-12
