@@ -214,6 +214,9 @@ def prefill_workload(name, rank):
         elif w.kind == "global":  # S carries the number of global tokens
             fn = lambda: swa.global_attn_fwd(q, k, v, w.W, w.S, out=out)
             nnz = swa.count_nonmasked(swa.MASK_GLOBAL, w.N, w.W, w.S)
+        elif w.kind == "dilated":  # S carries the dilation; each row sees min(W, i // S + 1) keys
+            fn = lambda: swa.dilated_attn_fwd(q, k, v, w.W, w.S, out=out)
+            nnz = sum(min(w.W, i // w.S + 1) for i in range(w.N))
         else:
             fn = lambda: swa.strided_attn_fwd(q, k, v, w.W, w.S, out=out)
             nnz = swa.count_nonmasked(swa.MASK_STRIDED, w.N, w.W, w.S)
@@ -424,7 +427,8 @@ def measure_variants(args, rank, peaks, flush, stream):
 
     out = {}
     reps = max(5, min(args.steps, 10))
-    for name in ("local_strided_prefill", "diff_causal", "gemma_swa_prefill", "longformer_global_prefill"):
+    for name in ("local_strided_prefill", "diff_causal", "gemma_swa_prefill", "longformer_global_prefill",
+                 "longformer_dilated_prefill"):
         w, fn, flops, ins, o = prefill_workload(name, rank)
         ms = time_steps(fn, reps, 3, flush, stream)
         mean_ms = sum(ms) / len(ms)

@@ -25,7 +25,7 @@ STRIDE_TAG = 0x40000000
 TILE = 128  # query rows and keys per tile in the prefill kernels
 
 __all__ = [
-    "swa_attn_fwd", "strided_attn_fwd", "global_attn_fwd", "diff_attn_fwd", "swa_decode_step", "decode_workspace_bytes",
+    "swa_attn_fwd", "strided_attn_fwd", "global_attn_fwd", "dilated_attn_fwd", "diff_attn_fwd", "swa_decode_step", "decode_workspace_bytes",
     "swa_sink_decode_step", "sink_decode_workspace_bytes", "swa_diff_decode_step", "diff_decode_workspace_bytes",
     "prefill_debug", "schedule", "count_nonmasked", "last_device_error", "SwaError", "library",
 ]
@@ -58,6 +58,8 @@ def library() -> ctypes.CDLL:
     lib.strided_attn_fwd.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, F, P]
     lib.global_attn_fwd.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, F, P]
     lib.global_attn_fwd.restype = I
+    lib.dilated_attn_fwd.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, F, P]
+    lib.dilated_attn_fwd.restype = I
     lib.diff_attn_fwd.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, F, P]
     lib.swa_decode_step.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, F, P, SZ, P]
     lib.swa_decode_workspace_bytes.argtypes = [I, I, I, I, I]
@@ -158,6 +160,17 @@ def global_attn_fwd(q, k, v, window: int, n_global: int, scale: float | None = N
     st = library().global_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, N, d,
                                    int(window), int(n_global), float(scale), _stream(stream))
     _raise(st, "global_attn_fwd")
+    return (out, lse) if return_lse else out
+
+
+def dilated_attn_fwd(q, k, v, window: int, dilation: int, scale: float | None = None, out=None,
+                     return_lse: bool = False, stream=None):
+    """Dilated window: row i attends keys i, i - dilation, ..., i - (window-1)*dilation."""
+    B, Hq, Hkv, N, d, out, lse = _prefill_common(q, k, v, out, return_lse)
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    st = library().dilated_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, N, d,
+                                    int(window), int(dilation), float(scale), _stream(stream))
+    _raise(st, "dilated_attn_fwd")
     return (out, lse) if return_lse else out
 
 

@@ -66,9 +66,15 @@ bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr
 
 bool head_dim_ok(int d) { return d == 64 || d == 128; }
 
+// Row r of the attention problem (r < N) is row row_off + r*row_mul of each
+// (b, head) in memory, whose heads hold N_full rows each (N_full < 0: N).
+// The dilated window runs one such strided view per residue class.
 swa_status_t run_prefill(int kind, bool diff, const void* q, const void* k, const void* q2, const void* k2,
                          const void* v, void* o, float* lse, const float* lambda, int B, int Hq, int Hkv, int N,
-                         int dqk, int dv, int W, int S, float scale, const swa_debug_t* dbg, void* stream) {
+                         int dqk, int dv, int W, int S, float scale, const swa_debug_t* dbg, void* stream,
+                         int N_full = -1, int row_mul = 1, int row_off = 0) {
+  if (N_full < 0) N_full = N;
+  if (row_mul < 1 || row_off < 0 || (int64_t)row_off + (int64_t)(N - 1) * row_mul >= N_full) return SWA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return SWA_ERR_INVALID_ARG;
   if (diff && (!aligned16(q2) || !aligned16(k2) || lambda == nullptr)) return SWA_ERR_INVALID_ARG;
   if (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)) return SWA_ERR_INVALID_ARG;
@@ -87,13 +93,17 @@ swa_status_t run_prefill(int kind, bool diff, const void* q, const void* k, cons
   PrefillMaps maps;
   std::memset(&maps, 0, sizeof(maps));
   const int64_t nB = (int64_t)B;
-  bool ok = encode_rows(&maps.q, q, dqk, N, nB * Hq, dqk, (int64_t)N * dqk) &&
-            encode_rows(&maps.k, k, dqk, N, nB * Hkv, dqk, (int64_t)N * dqk) &&
-            encode_rows(&maps.v, v, dv, N, nB * Hkv, dv, (int64_t)N * dv) &&
-            encode_rows(&maps.o, o, dv, N, nB * Hq, dv, (int64_t)N * dv, 32);
+  auto at = [&](const void* base, int d) {  // first row of the view
+    return static_cast<const void*>(static_cast<const uint16_t*>(base) + (int64_t)row_off * d);
+  };
+  const int64_t nf = N_full;
+  bool ok = encode_rows(&maps.q, at(q, dqk), dqk, N, nB * Hq, (int64_t)row_mul * dqk, nf * dqk) &&
+            encode_rows(&maps.k, at(k, dqk), dqk, N, nB * Hkv, (int64_t)row_mul * dqk, nf * dqk) &&
+            encode_rows(&maps.v, at(v, dv), dv, N, nB * Hkv, (int64_t)row_mul * dv, nf * dv) &&
+            encode_rows(&maps.o, at(o, dv), dv, N, nB * Hq, (int64_t)row_mul * dv, nf * dv, 32);
   if (ok && diff)
-    ok = encode_rows(&maps.q2, q2, dqk, N, nB * Hq, dqk, (int64_t)N * dqk) &&
-         encode_rows(&maps.k2, k2, dqk, N, nB * Hkv, dqk, (int64_t)N * dqk);
+    ok = encode_rows(&maps.q2, at(q2, dqk), dqk, N, nB * Hq, (int64_t)row_mul * dqk, nf * dqk) &&
+         encode_rows(&maps.k2, at(k2, dqk), dqk, N, nB * Hkv, (int64_t)row_mul * dqk, nf * dqk);
   if (ok && kind == kMaskStrided) {
     // stride row m is key m*S: a view whose row stride is S rows of K/V
     const int64_t rows = (N + (int64_t)S - 1) / S;
@@ -113,6 +123,7 @@ swa_status_t run_prefill(int kind, bool diff, const void* q, const void* k, cons
   p.nq = (N + 127) / 128;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.o = o; p.lse = lse; p.lambda = lambda;
+  p.lse_n = N_full; p.lse_off = row_off; p.lse_mul = row_mul;
   if (dbg) {
     p.dbg_cells = dbg->cells;
     p.dbg_tiles = dbg->tiles;
@@ -217,6 +228,20 @@ swa_status_t global_attn_fwd(const void* q, const void* k, const void* v, void* 
   if (n_global < 0) return SWA_ERR_INVALID_ARG;
   return run_prefill(kMaskGlobal, false, q, k, nullptr, nullptr, v, o, lse, nullptr, B, Hq, Hkv, N, d, d, W,
                      n_global, scale, nullptr, stream);
+}
+
+swa_status_t dilated_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                              int Hkv, int N, int d, int W, int dilation, float scale, void* stream) {
+  if (dilation < 1 || N < 1) return SWA_ERR_INVALID_ARG;
+  // residue class r (rows r, r + dilation, ...) is a plain window of W keys
+  // over the same class of keys: one strided view each
+  for (int r = 0; r < dilation && r < N; ++r) {
+    const int rows = (N - r + dilation - 1) / dilation;
+    const swa_status_t st = run_prefill(kMaskWindow, false, q, k, nullptr, nullptr, v, o, lse, nullptr, B, Hq, Hkv,
+                                        rows, d, d, W, 0, scale, nullptr, stream, N, dilation, r);
+    if (st != SWA_OK) return st;
+  }
+  return SWA_OK;
 }
 
 swa_status_t diff_attn_fwd(const void* q1, const void* k1, const void* q2, const void* k2, const void* v, void* o,

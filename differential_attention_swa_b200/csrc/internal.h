@@ -28,6 +28,7 @@ struct PrefillParams {
   float scale_log2;  // scale * log2(e)
   void* o;
   float* lse;
+  int lse_n, lse_off, lse_mul;  // lse row of (b, hq, i): (b*Hq + hq)*lse_n + lse_off + i*lse_mul
   const float* lambda;
   int64_t* dbg_cells;
   int32_t* dbg_tiles;

@@ -624,7 +624,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ++nunit;
       tc_fence_after();
       const int hq = un.hq[t];
-      const int64_t orow = ((int64_t)(un.b * p.Hq + hq) * p.N + i);
+      const int64_t orow = (int64_t)(un.b * p.Hq + hq) * p.lse_n + p.lse_off + (int64_t)i * p.lse_mul;
       if (DIFF) {
         if (t == 1) {
           // hands lambda / l2 to sub 0, which reads both accumulators

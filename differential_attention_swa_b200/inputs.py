@@ -65,7 +65,7 @@ def diff_decode_inputs(T, B, Hq, Hkv, dk, dv, W, seed: int = 0):
 @dataclass(frozen=True)
 class Workload:
     name: str
-    kind: str  # "swa", "strided", "global", "diff", "decode", "diff_decode"
+    kind: str  # "swa", "strided", "global", "dilated", "diff", "decode", "diff_decode"
     B: int
     Hq: int
     Hkv: int
@@ -100,6 +100,8 @@ WORKLOADS = {
     # window + global tokens with a Longformer-like shape (16 heads of 64,
     # a 512-token window, 64 global tokens at the start); S carries g
     "longformer_global_prefill": Workload("longformer_global_prefill", "global", 1, 16, 16, 16384, 64, 512, S=64),
+    # the same shape with a dilated window (dilation 2, S carries it)
+    "longformer_dilated_prefill": Workload("longformer_dilated_prefill", "dilated", 1, 16, 16, 16384, 64, 512, S=2),
     "gemma_swa_decode": Workload("gemma_swa_decode", "decode", 64, 16, 8, 0, 128, 1024, steps=256,
                                  pos0=131072),
     # the same decode with 4 attention-sink slots ahead of the window

@@ -107,6 +107,19 @@ swa_status_t global_attn_fwd(const void* q, const void* k, const void* v, void* 
                              int B, int Hq, int Hkv, int N, int d, int W, int n_global,
                              float scale, void* stream);
 
+/* Dilated sliding-window attention forward: row i attends the W keys
+ * i, i - dilation, ..., i - (W-1)*dilation (those >= 0).
+ * Source: "Learn: Sparse & Sliding-Window Attention", section 3b
+ * (Longformer: gaps of size d_dil inside the window, so the same budget of
+ * keys reaches d_dil times further). Rows and keys of one residue class mod
+ * `dilation` form a plain window of W keys, so the call runs the window
+ * kernel once per class on strided views of Q, K, V and O (no copies).
+ *   Arguments as swa_attn_fwd, plus dilation >= 1 (1 is swa_attn_fwd);
+ *   lse, if given, is written at the original row positions. */
+swa_status_t dilated_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                              int B, int Hq, int Hkv, int N, int d, int W, int dilation,
+                              float scale, void* stream);
+
 /* Differential attention forward:
  *     o = softmax(Q1 K1^T * scale + log M) V - lambda[h] * softmax(Q2 K2^T * scale + log M) V
  * over one shared V, both maps under the same window mask (W >= N: causal).

@@ -156,3 +156,15 @@ def test_diff_decode_bad_arguments_rejected_before_launch(lib):
     assert call(scale=0.0) == swa.ERR_INVALID_ARG
     assert call(dqk=128) == swa.ERR_UNSUPPORTED
     assert call(Hq=24, Hkv=8) == swa.ERR_UNSUPPORTED  # group of 3
+
+
+def test_global_and_dilated_bad_arguments(lib):
+    P = ctypes.c_void_p
+    g = P(0x10000)
+    st = lib.global_attn_fwd(g, g, g, g, None, 1, 2, 2, 256, 64, 16, -1, ctypes.c_float(0.1), None)
+    assert st == swa.ERR_INVALID_ARG  # negative number of global tokens
+    st = lib.dilated_attn_fwd(g, g, g, g, None, 1, 2, 2, 256, 64, 16, 0, ctypes.c_float(0.1), None)
+    assert st == swa.ERR_INVALID_ARG  # dilation 0
+    st = lib.dilated_attn_fwd(g, g, g, g, None, 1, 2, 2, 256, 96, 16, 2, ctypes.c_float(0.1), None)
+    assert st == swa.ERR_UNSUPPORTED  # head dim
+    assert lib.swa_count_nonmasked(3, 10, 4, -1) == -1

@@ -48,6 +48,8 @@ def run_prefill(kind, q, k, v, W, S, lse=False):
         r = swa.swa_attn_fwd(qd, kd, vd, W, return_lse=lse)
     elif kind == "global":  # S carries the number of global tokens
         r = swa.global_attn_fwd(qd, kd, vd, W, S, return_lse=lse)
+    elif kind == "dilated":  # S carries the dilation
+        r = swa.dilated_attn_fwd(qd, kd, vd, W, S, return_lse=lse)
     else:
         r = swa.strided_attn_fwd(qd, kd, vd, W, S, return_lse=lse)
     assert swa.last_device_error() == swa.OK
@@ -88,6 +90,11 @@ EDGE = [
     ("global", 1, 2, 2, 300, 64, 5000, 9),  # window beyond N: full causal
     ("global", 1, 2, 2, 400, 64, 16, 0),    # no global token: the window
     ("global", 1, 2, 2, 333, 64, 1, 1000),  # every token global: full causal
+    ("dilated", 1, 2, 2, 1000, 64, 100, 2), # dilation 2, several tiles per class
+    ("dilated", 1, 4, 2, 777, 128, 64, 3),  # N not a multiple of the dilation, group 2
+    ("dilated", 1, 3, 1, 300, 64, 20, 7),   # group 3 (tile pairs), short classes
+    ("dilated", 1, 2, 2, 250, 64, 30, 1),   # dilation 1: the window
+    ("dilated", 1, 2, 2, 100, 64, 5, 150),  # dilation beyond N: each row sees only itself
 ]
 
 
@@ -222,7 +229,7 @@ def sampled_rows(B, H, N, n, seed):
 
 
 @pytest.mark.parametrize("name", ["mistral_swa_prefill", "local_strided_prefill", "gemma_swa_prefill",
-                                  "longformer_global_prefill"])
+                                  "longformer_global_prefill", "longformer_dilated_prefill"])
 def test_workload_sampled_rows(orc, name):
     w = WORKLOADS[name]
     q, k, v = attn_inputs(w.B, w.Hq, w.Hkv, w.N, w.d, seed=0)
@@ -263,3 +270,12 @@ def test_decode_workload_first_steps(orc):
     outs = [swa.swa_decode_step(qd[t], knd[t], vnd[t], kc, vc, posd[t]) for t in range(T)]
     assert swa.last_device_error() == swa.OK
     compare(torch.stack(outs), ref, "decode workload")
+
+
+def test_dilated_lse_at_original_rows(orc):
+    """The per-class launches write the log-sum-exp at each row's own index."""
+    q, k, v = attn_inputs(1, 2, 2, 500, 64, seed=77)
+    out, lse = run_prefill("dilated", q, k, v, 40, 3, lse=True)
+    ref, ref_lse = orc.attention("dilated", q, k, v, W=40, S=3, scale=0.125, with_lse=True)
+    compare(out, ref, "dilated with lse")
+    assert np.abs(lse.cpu().numpy() - ref_lse).max() < 2e-3
