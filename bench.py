@@ -36,6 +36,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 PREFILL_SOURCES = ["differential_attention_swa_b200/csrc/prefill.cu", "differential_attention_swa_b200/csrc/ptx.cuh",
                    "differential_attention_swa_b200/csrc/schedule.cuh"]
 DECODE_SOURCES = ["differential_attention_swa_b200/csrc/decode.cu", "differential_attention_swa_b200/csrc/ptx.cuh"]
+DIFF_DECODE_SOURCES = ["differential_attention_swa_b200/csrc/diff_decode.cu", "differential_attention_swa_b200/csrc/ptx.cuh"]
 
 
 # ------------------------------------------------------------ host logic --
@@ -414,7 +415,8 @@ def measure_decode(args, rank, peaks, flush, stream, reps=5, name="gemma_swa_dec
             "decode_steps_per_graph": T, "bytes_per_decode_step": bytes_per_step,
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
                          "frac": round(gbs / peak, 4),
-                         "traffic": None if diff else profiled_traffic("decode_gemma.md", DECODE_SOURCES),
+                         "traffic": (profiled_traffic("decode_diff_gqa.md", DIFF_DECODE_SOURCES) if diff else
+                                     profiled_traffic("decode_gemma.md", DECODE_SOURCES)),
                          "kernel": ("diff_decode_split_kernel<2> + diff_decode_combine_kernel" if diff else
                                     "decode_split_kernel<128,2> + decode_combine_kernel<128>")},
             "launches": reps * T * 2}
