@@ -123,7 +123,6 @@ swa_status_t run_prefill(int kind, bool diff, const void* q, const void* k, cons
   p.nq = (N + 127) / 128;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.o = o; p.lse = lse; p.lambda = lambda;
-  p.lse_n = N_full; p.lse_off = row_off; p.lse_mul = row_mul;
   if (dbg) {
     p.dbg_cells = dbg->cells;
     p.dbg_tiles = dbg->tiles;
@@ -148,7 +147,11 @@ swa_status_t run_prefill(int kind, bool diff, const void* q, const void* k, cons
   if (p.num_ctas <= 0) return SWA_ERR_CUDA;
   p.err_flag = device_error_ptr();
   if (p.err_flag == nullptr) return SWA_ERR_CUDA;
-  cudaError_t e = launch_prefill(maps, p, dqk, dv, diff, (int)nunits, static_cast<cudaStream_t>(stream));
+  RowMap rows;
+  rows.n = N_full;
+  rows.off = row_off;
+  rows.mul = row_mul;
+  cudaError_t e = launch_prefill(maps, p, rows, dqk, dv, diff, (int)nunits, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
 }
 

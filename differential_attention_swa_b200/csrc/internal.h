@@ -28,7 +28,6 @@ struct PrefillParams {
   float scale_log2;  // scale * log2(e)
   void* o;
   float* lse;
-  int lse_n, lse_off, lse_mul;  // lse row of (b, hq, i): (b*Hq + hq)*lse_n + lse_off + i*lse_mul
   const float* lambda;
   int64_t* dbg_cells;
   int32_t* dbg_tiles;
@@ -38,13 +37,19 @@ struct PrefillParams {
   int* err_flag;  // device word that receives SWA_ERR_TIMEOUT
 };
 
+// Row map of a strided view (dilated windows): row i of the problem is row
+// off + i*mul of a head holding n rows, which is where its log-sum-exp goes.
+struct RowMap {
+  int n, off, mul;
+};
+
 struct PrefillMaps {
   CUtensorMap q, q2, k, k2, v, ks, vs;
   CUtensorMap o;  // output, 64 x 32-row boxes (one warp's rows)
 };
 
-cudaError_t launch_prefill(const PrefillMaps& maps, const PrefillParams& p, int dqk, int dv, bool diff,
-                           int nunits, cudaStream_t stream);
+cudaError_t launch_prefill(const PrefillMaps& maps, const PrefillParams& p, const RowMap& rows, int dqk, int dv,
+                           bool diff, int nunits, cudaStream_t stream);
 int prefill_smem_bytes(int dqk, int dv, bool diff);
 
 struct DecodeParams {

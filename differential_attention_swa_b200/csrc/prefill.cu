@@ -142,6 +142,9 @@ struct Items {
   int nst, blo, bhi, n;
 };
 
+// GEN: also the window + global-token kind (extra tiles of K/V itself); the
+// window and strided kinds compile without that branch.
+template <bool GEN>
 __device__ __forceinline__ Items unit_items(const PrefillParams& p, const Unit& un) {
   Items it;
   it.nst = 0;
@@ -150,7 +153,8 @@ __device__ __forceinline__ Items unit_items(const PrefillParams& p, const Unit& 
 #pragma unroll
   for (int t = 0; t < 2; ++t) {
     if (un.valid[t]) {
-      it.k[t] = qtile_keys(p.kind, p.N, p.W, p.S, BM, BN, un.qt[t]);
+      it.k[t] = GEN ? qtile_keys(p.kind, p.N, p.W, p.S, BM, BN, un.qt[t])
+                    : qtile_keys_basic(p.kind, p.N, p.W, p.S, BM, BN, un.qt[t]);
       it.nst = imax(it.nst, it.k[t].n_stride);
       it.blo = imin(it.blo, it.k[t].band_lo);
       it.bhi = imax(it.bhi, it.k[t].band_hi);
@@ -179,13 +183,16 @@ __device__ __forceinline__ void record_timeout(volatile int* abort_flag, int* er
   atomicExch(err_flag, 4 /* SWA_ERR_TIMEOUT */);
 }
 
-template <int DQK, int DV, bool DIFF>
+// GEN instantiations serve the window + global-token kind and strided views
+// (dilated windows: rows r, r + dil, ... of each head, with the log-sum-exp
+// written at the original rows); the others compile without that code.
+template <int DQK, int DV, bool DIFF, bool GEN>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_q2,
                    const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_k2,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_ks,
                    const __grid_constant__ CUtensorMap tm_vs, const __grid_constant__ CUtensorMap tm_o,
-                   const PrefillParams p) {
+                   const PrefillParams p, const RowMap rmap) {
   using C = PrefillCfg<DQK, DV, DIFF>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -254,7 +261,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int ui = unit_of(rnd);
         if (ui >= nunits) continue;
         const Unit un = decode_unit(p, ui);
-        const Items it = unit_items(p, un);
+        const Items it = unit_items<GEN>(p, un);
         // Q of this unit once every S MMA of the previous unit is done
         if (nq_ld > 0 && !mbar_wait(bar(BarLayout::kQEmpty), (nq_ld - 1) & 1, abort_flag)) {
           record_timeout(abort_flag, p.err_flag);
@@ -337,7 +344,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int ui = unit_of(rnd);
         if (ui >= nunits) continue;
         const Unit un = decode_unit(p, ui);
-        const Items it = unit_items(p, un);
+        const Items it = unit_items<GEN>(p, un);
         const int ntot[2] = {un.valid[0] ? qtile_nkeys(it.k[0]) : 0, un.valid[1] ? qtile_nkeys(it.k[1]) : 0};
         int kcount[2] = {0, 0};   // S tiles of this unit per sub
         int pv_done[2] = {0, 0};  // PV products of this unit per sub
@@ -505,12 +512,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int ui = unit_of(rnd);
       if (ui >= nunits) continue;
       const Unit un = decode_unit(p, ui);
-      const Items it = unit_items(p, un);
+      const Items it = unit_items<GEN>(p, un);
       if (!un.valid[t]) continue;
       const int i = un.qt[t] * BM + r;  // query index
       const bool row_ok = i < p.N;
       const int lo = window_lo(i, Wc);
-      const int mst = extra_rows_below(p.kind, lo, p.S);  // extra-view rows (stride or global keys) below lo
+      const int mst = GEN ? extra_rows_below(p.kind, lo, p.S)  // extra-view rows below lo
+                          : ((p.kind == kMaskStrided) ? stride_rows_below(lo, p.S) : 0);
       float m_run = -INFINITY;  // running max, log2 units (scores * scale * log2 e)
       float l_run = 0.f;
       long long cells = 0;
@@ -624,7 +632,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       ++nunit;
       tc_fence_after();
       const int hq = un.hq[t];
-      const int64_t orow = (int64_t)(un.b * p.Hq + hq) * p.lse_n + p.lse_off + (int64_t)i * p.lse_mul;
+      const int64_t orow = GEN ? (int64_t)(un.b * p.Hq + hq) * rmap.n + rmap.off + (int64_t)i * rmap.mul
+                               : ((int64_t)(un.b * p.Hq + hq) * p.N + i);
       if (DIFF) {
         if (t == 1) {
           // hands lambda / l2 to sub 0, which reads both accumulators
@@ -683,10 +692,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int DQK, int DV, bool DIFF>
-static cudaError_t launch_one(const PrefillMaps& maps, const PrefillParams& p, int nunits, cudaStream_t stream) {
+template <int DQK, int DV, bool DIFF, bool GEN = false>
+static cudaError_t launch_one(const PrefillMaps& maps, const PrefillParams& p, const RowMap& rows, int nunits,
+                              cudaStream_t stream) {
   using C = PrefillCfg<DQK, DV, DIFF>;
-  auto kern = prefill_kernel<DQK, DV, DIFF>;
+  auto kern = prefill_kernel<DQK, DV, DIFF, GEN>;
   static bool attr_set = false;  // per process; the attribute is per function
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
@@ -695,19 +705,25 @@ static cudaError_t launch_one(const PrefillMaps& maps, const PrefillParams& p, i
   }
   const int grid = nunits < p.num_ctas ? nunits : p.num_ctas;
   kern<<<grid, kThreads, C::kSmemBytes, stream>>>(maps.q, maps.q2, maps.k, maps.k2, maps.v, maps.ks, maps.vs,
-                                                  maps.o, p);
+                                                  maps.o, p, rows);
   return cudaGetLastError();
 }
 
-cudaError_t launch_prefill(const PrefillMaps& maps, const PrefillParams& p, int dqk, int dv, bool diff,
-                           int nunits, cudaStream_t stream) {
+cudaError_t launch_prefill(const PrefillMaps& maps, const PrefillParams& p, const RowMap& rows, int dqk, int dv,
+                           bool diff, int nunits, cudaStream_t stream) {
   if (diff) {
-    if (dqk == 64 && dv == 128) return launch_one<64, 128, true>(maps, p, nunits, stream);
-    if (dqk == 64 && dv == 64) return launch_one<64, 64, true>(maps, p, nunits, stream);
+    if (dqk == 64 && dv == 128) return launch_one<64, 128, true>(maps, p, rows, nunits, stream);
+    if (dqk == 64 && dv == 64) return launch_one<64, 64, true>(maps, p, rows, nunits, stream);
     return cudaErrorInvalidValue;
   }
-  if (dqk == 128 && dv == 128) return launch_one<128, 128, false>(maps, p, nunits, stream);
-  if (dqk == 64 && dv == 64) return launch_one<64, 64, false>(maps, p, nunits, stream);
+  const bool gen = p.kind == kMaskGlobal || rows.mul != 1 || rows.off != 0 || rows.n != p.N;
+  if (gen) {
+    if (dqk == 128 && dv == 128) return launch_one<128, 128, false, true>(maps, p, rows, nunits, stream);
+    if (dqk == 64 && dv == 64) return launch_one<64, 64, false, true>(maps, p, rows, nunits, stream);
+    return cudaErrorInvalidValue;
+  }
+  if (dqk == 128 && dv == 128) return launch_one<128, 128, false>(maps, p, rows, nunits, stream);
+  if (dqk == 64 && dv == 64) return launch_one<64, 64, false>(maps, p, rows, nunits, stream);
   return cudaErrorInvalidValue;
 }
 

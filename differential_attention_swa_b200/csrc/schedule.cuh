@@ -72,8 +72,28 @@ SWA_HD QTileKeys qtile_keys(int kind, int N, int W, int S, int Bq, int Bk, int q
   const int Wc = (kind == kMaskCausal) ? N : W;
   r.band_lo = window_lo(r0, Wc) / Bk;
   r.band_hi = r1 / Bk;
-  const int m = extra_rows_below(kind, window_lo(r1, Wc), S);
-  r.n_stride = (m + Bk - 1) / Bk;
+  r.n_stride = 0;
+  if ((kind == kMaskStrided || kind == kMaskGlobal) && S > 0) {
+    const int m = extra_rows_below(kind, window_lo(r1, Wc), S);
+    r.n_stride = (m + Bk - 1) / Bk;
+  }
+  return r;
+}
+
+// The same for the window, strided and causal kinds only (no global-token
+// branch), for kernels built without the global kind.
+SWA_HD QTileKeys qtile_keys_basic(int kind, int N, int W, int S, int Bq, int Bk, int qt) {
+  QTileKeys r;
+  const int r0 = qt * Bq;
+  const int r1 = imin(N - 1, r0 + Bq - 1);
+  const int Wc = (kind == kMaskCausal) ? N : W;
+  r.band_lo = window_lo(r0, Wc) / Bk;
+  r.band_hi = r1 / Bk;
+  r.n_stride = 0;
+  if (kind == kMaskStrided && S > 0) {
+    const int m = stride_rows_below(window_lo(r1, Wc), S);
+    r.n_stride = (m + Bk - 1) / Bk;
+  }
   return r;
 }
 
