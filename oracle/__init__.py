@@ -76,6 +76,10 @@ def _L():
         lib.orc_sink_decode.restype = I
         lib.orc_diff_decode.argtypes = [P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, D, P]
         lib.orc_diff_decode.restype = I
+        for fn in ("orc_attention_bwd_dq_row", "orc_attention_bwd_dkv_row"):
+            getattr(lib, fn).argtypes = [I, P, P, P, P, I, I, I, I, I, I, I, I, D, I, I, I] + (
+                [P] if fn.endswith("dq_row") else [P, P])
+            getattr(lib, fn).restype = None
         lib.orc_schedule_qtile.argtypes = [I, I, I, I, I, I, I, P, I64, P]
         lib.orc_schedule_qtile.restype = I64
         _lib = lib
@@ -288,6 +292,45 @@ def diff_decode(q1, q2, k1_new, k2_new, v_new, k1_cache, k2_cache, v_cache, lam,
     if rc != 0:
         raise ValueError("oracle: bad arguments")
     return out, k1c, k2c, vc
+
+
+def attention_bwd(kind: str, q, k, v, dO, W: int = 0, S: int = 0, scale: float | None = None,
+                  dq_rows=None, dkv_rows=None):
+    """Gradients of sum(O * dO) for the masked attention forward, from the
+    chain rule written per output row (see oracle.c). q [B,Hq,N,dk], k
+    [B,Hkv,N,dk], v [B,Hkv,N,dv], dO [B,Hq,N,dv]. With no row lists, returns
+    full (dq, dk, dv); else dq for the flat (b*Hq + hq)*N + i rows in dq_rows
+    and (dk, dv) for the flat (b*Hkv + hk)*N + j rows in dkv_rows."""
+    q, k, v, dO = _f32(q), _f32(k), _f32(v), _f32(dO)
+    B, Hq, N, dk = q.shape
+    Hkv, dv = k.shape[1], v.shape[3]
+    if scale is None:
+        scale = 1.0 / np.sqrt(dk)
+    lib, kd = _L(), _KIND[kind]
+    args = (kd, _p(q), _p(k), _p(v), _p(dO), B, Hq, Hkv, N, dk, dv, int(W), int(S), float(scale))
+    full = dq_rows is None and dkv_rows is None
+    qr = np.arange(B * Hq * N) if full else np.asarray(dq_rows if dq_rows is not None else [], dtype=np.int64)
+    kr = np.arange(B * Hkv * N) if full else np.asarray(dkv_rows if dkv_rows is not None else [], dtype=np.int64)
+    dq = np.zeros((qr.size, dk))
+    dkk = np.zeros((kr.size, dk))
+    dvv = np.zeros((kr.size, dv))
+    for n_, r in enumerate(qr):
+        r = int(r)
+        if not 0 <= r < B * Hq * N:
+            raise ValueError("row out of range")
+        buf = np.zeros(dk)
+        lib.orc_attention_bwd_dq_row(*args, r // (Hq * N), (r // N) % Hq, r % N, _p(buf))
+        dq[n_] = buf
+    for n_, r in enumerate(kr):
+        r = int(r)
+        if not 0 <= r < B * Hkv * N:
+            raise ValueError("row out of range")
+        a, b_ = np.zeros(dk), np.zeros(dv)
+        lib.orc_attention_bwd_dkv_row(*args, r // (Hkv * N), (r // N) % Hkv, r % N, _p(a), _p(b_))
+        dkk[n_], dvv[n_] = a, b_
+    if full:
+        return dq.reshape(B, Hq, N, dk), dkk.reshape(B, Hkv, N, dk), dvv.reshape(B, Hkv, N, dv)
+    return dq, dkk, dvv
 
 
 # ------------------------------------------------------------- schedule ---

@@ -649,3 +649,91 @@ int orc_diff_decode(const float* q1, const float* q2, const float* k1_new, const
   free(key_slot);
   return 0;
 }
+
+/* ---------------------------------------------------------------------- */
+/* Backward of the masked attention forward. The pages give no backward   */
+/* pass; these functions apply the chain rule to the forward definition   */
+/* ([SW] section 3: o_i = sum_j w_ij v_j, w_i = softmax_j(scale q_i.k_j    */
+/* + log M_ij)), with dO the gradient of the loss with respect to O:      */
+/*   dv_j  = sum_i w_ij do_i                                              */
+/*   dw_ij = do_i . v_j,   D_i = sum_j w_ij dw_ij (= do_i . o_i)          */
+/*   ds_ij = w_ij (dw_ij - D_i)                                           */
+/*   dq_i  = scale sum_j ds_ij k_j,   dk_j = scale sum_i ds_ij q_i        */
+/* summed over the query heads that share a KV head. Written per output   */
+/* row, straight from these sums; slow, for tests only.                   */
+/* ---------------------------------------------------------------------- */
+
+/* Forward weights w_i (length N) and D_i of query row (b, hq, i). */
+static double bwd_row_weights(int kind, const float* q, const float* k, const float* v, const float* dO,
+                              int B, int Hq, int Hkv, int N, int dk, int dv, int W, int S, double scale,
+                              int b, int hq, int i, double* w, double* mrow, double* s, double* qd,
+                              double* o) {
+  const int G = Hq / Hkv, hk = hq / G;
+  const float* qrow = q + (((int64_t)b * Hq + hq) * N + i) * dk;
+  for (int c = 0; c < dk; ++c) qd[c] = (double)qrow[c];
+  const float* K = k + ((int64_t)b * Hkv + hk) * (int64_t)N * dk;
+  const float* V = v + ((int64_t)b * Hkv + hk) * (int64_t)N * dv;
+  orc_mask_row(kind, N, W, S, i, mrow);
+  orc_attention_row(qd, K, V, mrow, N, dk, dv, scale, o, w, s, NULL);
+  const float* dorow = dO + (((int64_t)b * Hq + hq) * N + i) * dv;
+  double D = 0.0;
+  for (int c = 0; c < dv; ++c) D += (double)dorow[c] * o[c];
+  return D;
+}
+
+/* dq of query row (b, hq, i): dk doubles. */
+void orc_attention_bwd_dq_row(int kind, const float* q, const float* k, const float* v, const float* dO,
+                              int B, int Hq, int Hkv, int N, int dk, int dv, int W, int S, double scale,
+                              int b, int hq, int i, double* dq) {
+  double* w = (double*)malloc(sizeof(double) * (size_t)N);
+  double* mrow = (double*)malloc(sizeof(double) * (size_t)N);
+  double* s = (double*)malloc(sizeof(double) * (size_t)N);
+  double* qd = (double*)malloc(sizeof(double) * (size_t)dk);
+  double* o = (double*)malloc(sizeof(double) * (size_t)dv);
+  const double D = bwd_row_weights(kind, q, k, v, dO, B, Hq, Hkv, N, dk, dv, W, S, scale, b, hq, i, w, mrow, s,
+                                   qd, o);
+  const int hk = hq / (Hq / Hkv);
+  const float* K = k + ((int64_t)b * Hkv + hk) * (int64_t)N * dk;
+  const float* V = v + ((int64_t)b * Hkv + hk) * (int64_t)N * dv;
+  const float* dorow = dO + (((int64_t)b * Hq + hq) * N + i) * dv;
+  for (int c = 0; c < dk; ++c) dq[c] = 0.0;
+  for (int j = 0; j < N; ++j) {
+    if (w[j] == 0.0) continue;
+    double dw = 0.0;
+    for (int c = 0; c < dv; ++c) dw += (double)dorow[c] * (double)V[(int64_t)j * dv + c];
+    const double ds = w[j] * (dw - D);
+    for (int c = 0; c < dk; ++c) dq[c] += scale * ds * (double)K[(int64_t)j * dk + c];
+  }
+  free(w); free(mrow); free(s); free(qd); free(o);
+}
+
+/* dk and dv of key row (b, hk, j): dk and dv doubles, summed over every
+ * query row of every query head of KV head hk. */
+void orc_attention_bwd_dkv_row(int kind, const float* q, const float* k, const float* v, const float* dO,
+                               int B, int Hq, int Hkv, int N, int dk, int dv, int W, int S, double scale,
+                               int b, int hk, int j, double* dkj, double* dvj) {
+  double* w = (double*)malloc(sizeof(double) * (size_t)N);
+  double* mrow = (double*)malloc(sizeof(double) * (size_t)N);
+  double* s = (double*)malloc(sizeof(double) * (size_t)N);
+  double* qd = (double*)malloc(sizeof(double) * (size_t)dk);
+  double* o = (double*)malloc(sizeof(double) * (size_t)dv);
+  const int G = Hq / Hkv;
+  const float* V = v + ((int64_t)b * Hkv + hk) * (int64_t)N * dv;
+  for (int c = 0; c < dk; ++c) dkj[c] = 0.0;
+  for (int c = 0; c < dv; ++c) dvj[c] = 0.0;
+  for (int hq = hk * G; hq < hk * G + G; ++hq) {
+    for (int i = 0; i < N; ++i) {
+      orc_mask_row(kind, N, W, S, i, mrow);
+      if (mrow[j] != 0.0) continue; /* row i does not attend key j */
+      const double D = bwd_row_weights(kind, q, k, v, dO, B, Hq, Hkv, N, dk, dv, W, S, scale, b, hq, i, w, mrow,
+                                       s, qd, o);
+      const float* dorow = dO + (((int64_t)b * Hq + hq) * N + i) * dv;
+      double dw = 0.0;
+      for (int c = 0; c < dv; ++c) dw += (double)dorow[c] * (double)V[(int64_t)j * dv + c];
+      const double ds = w[j] * (dw - D);
+      for (int c = 0; c < dv; ++c) dvj[c] += w[j] * (double)dorow[c];
+      for (int c = 0; c < dk; ++c) dkj[c] += scale * ds * qd[c];
+    }
+  }
+  free(w); free(mrow); free(s); free(qd); free(o);
+}

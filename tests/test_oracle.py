@@ -603,3 +603,71 @@ def test_dilated_attention_matches_torch_sdpa_fp64(orc, B, Hq, Hkv, N, d, W, dil
     ii, jj = np.meshgrid(np.arange(N), np.arange(N), indexing="ij")
     allowed = (jj <= ii) & ((ii - jj) % dil == 0) & ((ii - jj) // dil < W)
     assert np.abs(out - sdpa_ref(q, k, v, allowed, 0.25)).max() < 1e-12
+
+
+# ------------------------------------------------------------- backward ----
+
+def _allowed(kind, N, W, S):
+    ii, jj = np.meshgrid(np.arange(N), np.arange(N), indexing="ij")
+    if kind == "causal":
+        return jj <= ii
+    band = (ii - W < jj) & (jj <= ii)
+    if kind == "strided":
+        return band | ((jj % S == 0) & (jj <= ii))
+    if kind == "global":
+        return band | (((jj < S) | (ii < S)) & (jj <= ii))
+    return band
+
+
+@pytest.mark.parametrize("kind,B,Hq,Hkv,N,dk,dv,W,S", [
+    ("swa", 1, 2, 2, 40, 8, 8, 7, 0), ("swa", 1, 4, 2, 33, 16, 12, 5, 0), ("causal", 2, 2, 1, 25, 8, 8, 0, 0),
+    ("strided", 1, 2, 2, 45, 8, 8, 4, 6), ("global", 1, 2, 1, 38, 8, 8, 5, 3)])
+def test_backward_matches_torch_autograd_fp64(orc, kind, B, Hq, Hkv, N, dk, dv, W, S):
+    """The oracle's per-row chain rule against torch autograd through fp64
+    scaled_dot_product_attention with the explicit mask (GQA by repeating
+    K/V heads, whose gradients autograd sums)."""
+    q, k, v = attn_inputs(B, Hq, Hkv, N, dk, dv, seed=17)
+    dO = randn_bf16((B, Hq, N, dv), 99)
+    scale = 1 / math.sqrt(dk)
+    dq, dkk, dvv = orc.attention_bwd(kind, q, k, v, dO, W=W, S=S, scale=scale)
+    G = Hq // Hkv
+    q64, k64, v64 = (t.double().requires_grad_(True) for t in (q, k, v))
+    o = F.scaled_dot_product_attention(q64, k64.repeat_interleave(G, dim=1), v64.repeat_interleave(G, dim=1),
+                                       attn_mask=torch.from_numpy(_allowed(kind, N, W, S)), scale=scale)
+    (o * dO.double()).sum().backward()
+    assert np.abs(dq - q64.grad.numpy()).max() < 1e-12
+    assert np.abs(dkk - k64.grad.numpy()).max() < 1e-12
+    assert np.abs(dvv - v64.grad.numpy()).max() < 1e-12
+
+
+def test_backward_matches_finite_differences_of_the_oracle_forward(orc):
+    """Central differences of f = sum(O * dO), O from the oracle's forward,
+    for a few entries of Q, K and V (steps of 2^-10 are exact in float32)."""
+    B, Hq, Hkv, N, d, W = 1, 2, 1, 12, 4, 5
+    q, k, v = (t.float() for t in attn_inputs(B, Hq, Hkv, N, d, seed=23))
+    dO = randn_bf16((B, Hq, N, d), 7).float()
+    dq, dkk, dvv = orc.attention_bwd("swa", q, k, v, dO, W=W, scale=0.5)
+    h = 2.0 ** -10
+
+    def f(qq, kk, vv):
+        return float((orc.attention("swa", qq, kk, vv, W=W, scale=0.5) * dO.double().numpy()).sum())
+
+    for name, t, g, idx in (("q", q, dq, (0, 1, 7, 2)), ("k", k, dkk, (0, 0, 4, 1)), ("v", v, dvv, (0, 0, 9, 3)),
+                            ("k0", k, dkk, (0, 0, 0, 0))):
+        plus, minus = t.clone(), t.clone()
+        plus[idx] += h
+        minus[idx] -= h
+        args_p = {"q": (plus, k, v), "k": (q, plus, v), "v": (q, k, plus), "k0": (q, plus, v)}[name]
+        args_m = {"q": (minus, k, v), "k": (q, minus, v), "v": (q, k, minus), "k0": (q, minus, v)}[name]
+        num = (f(*args_p) - f(*args_m)) / (2 * h)
+        assert abs(num - g[idx]) < 2e-5 * max(1.0, abs(g[idx])), (name, num, g[idx])
+
+
+def test_backward_row_subsets_match_full(orc):
+    q, k, v = attn_inputs(2, 4, 2, 30, 8, seed=31)
+    dO = randn_bf16((2, 4, 30, 8), 32)
+    dq, dkk, dvv = orc.attention_bwd("swa", q, k, v, dO, W=6)
+    qr, kr = np.array([0, 29, 31, 4 * 30 + 17, 8 * 30 - 1]), np.array([0, 5, 30 + 29, 3 * 30 + 2])
+    a, b, c = orc.attention_bwd("swa", q, k, v, dO, W=6, dq_rows=qr, dkv_rows=kr)
+    assert np.array_equal(a, dq.reshape(-1, 8)[qr])
+    assert np.array_equal(b, dkk.reshape(-1, 8)[kr]) and np.array_equal(c, dvv.reshape(-1, 8)[kr])
