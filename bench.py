@@ -206,6 +206,19 @@ def prefill_workload(name, rank):
         fn = lambda: swa.diff_attn_fwd(*ins, lam, window=w.W, scale=w.scale, out=out)
         nnz = swa.count_nonmasked(swa.MASK_WINDOW, w.N, w.W)
         flops = nnz * w.B * w.Hq * 2 * (2 * w.d + 2 * w.dv_)  # two maps, each 2*d_qk + 2*d_v per cell
+    elif w.kind == "swa_bwd":
+        from differential_attention_swa_b200.inputs import randn_bf16
+
+        q, k, v = (t.cuda() for t in attn_inputs(w.B, w.Hq, w.Hkv, w.N, w.d, seed=seed))
+        d_o = randn_bf16((w.B, w.Hq, w.N, w.d), seed + 3).cuda()
+        o, lse = swa.swa_attn_fwd(q, k, v, w.W, return_lse=True)  # the forward, outside the timed region
+        ws = torch.empty(swa.attn_bwd_workspace_bytes(w.B, w.Hq, w.N), dtype=torch.uint8, device="cuda")
+        out = None
+        fn = lambda: swa.swa_attn_bwd(q, k, v, o, d_o, lse, w.W, workspace=ws)
+        nnz = swa.count_nonmasked(swa.MASK_WINDOW, w.N, w.W)
+        # the usual accounting: scores, dP, dV, dQ, dK = 5 products of 2*d per cell
+        flops = 10 * w.d * nnz * w.B * w.Hq
+        ins = [q, k, v, o, lse, d_o, ws]
     else:
         q, k, v = (t.cuda() for t in attn_inputs(w.B, w.Hq, w.Hkv, w.N, w.d, seed=seed))
         out = torch.empty_like(q)
@@ -357,7 +370,7 @@ def measure_ours(args, rank, world, peaks, peak_src, dist):
         "clocks": clk,
         "gpu_launches": args.steps,
     }
-    if not args.no_e2e:
+    if not args.no_e2e and out is not None:  # the backward workload has no single output to copy back
         res["e2e"] = measure_e2e(w, fn, ins, out, flops, stream)
     if not args.no_variants and args.only is None:
         res["variants"] = measure_variants(args, rank, peaks, flush, stream)
@@ -430,7 +443,7 @@ def measure_variants(args, rank, peaks, flush, stream):
     out = {}
     reps = max(5, min(args.steps, 10))
     for name in ("local_strided_prefill", "diff_causal", "gemma_swa_prefill", "longformer_global_prefill",
-                 "longformer_dilated_prefill"):
+                 "longformer_dilated_prefill", "mistral_swa_backward"):
         w, fn, flops, ins, o = prefill_workload(name, rank)
         ms = time_steps(fn, reps, 3, flush, stream)
         mean_ms = sum(ms) / len(ms)

@@ -25,7 +25,7 @@ STRIDE_TAG = 0x40000000
 TILE = 128  # query rows and keys per tile in the prefill kernels
 
 __all__ = [
-    "swa_attn_fwd", "strided_attn_fwd", "global_attn_fwd", "dilated_attn_fwd", "diff_attn_fwd", "swa_decode_step", "decode_workspace_bytes",
+    "swa_attn_fwd", "strided_attn_fwd", "global_attn_fwd", "dilated_attn_fwd", "swa_attn_bwd", "diff_attn_fwd", "swa_decode_step", "decode_workspace_bytes",
     "swa_sink_decode_step", "sink_decode_workspace_bytes", "swa_diff_decode_step", "diff_decode_workspace_bytes",
     "prefill_debug", "schedule", "count_nonmasked", "last_device_error", "SwaError", "library",
 ]
@@ -60,6 +60,10 @@ def library() -> ctypes.CDLL:
     lib.global_attn_fwd.restype = I
     lib.dilated_attn_fwd.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, F, P]
     lib.dilated_attn_fwd.restype = I
+    lib.swa_attn_bwd.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, P, SZ, P]
+    lib.swa_attn_bwd.restype = I
+    lib.swa_attn_bwd_workspace_bytes.argtypes = [I, I, I]
+    lib.swa_attn_bwd_workspace_bytes.restype = SZ
     lib.diff_attn_fwd.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, F, P]
     lib.swa_decode_step.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, F, P, SZ, P]
     lib.swa_decode_workspace_bytes.argtypes = [I, I, I, I, I]
@@ -172,6 +176,34 @@ def dilated_attn_fwd(q, k, v, window: int, dilation: int, scale: float | None = 
                                     int(window), int(dilation), float(scale), _stream(stream))
     _raise(st, "dilated_attn_fwd")
     return (out, lse) if return_lse else out
+
+
+def attn_bwd_workspace_bytes(B: int, Hq: int, N: int) -> int:
+    return int(library().swa_attn_bwd_workspace_bytes(B, Hq, N))
+
+
+def swa_attn_bwd(q, k, v, o, d_o, lse, window: int, scale: float | None = None, workspace=None, stream=None):
+    """Gradients (dq, dk, dv) of the window attention forward, given its
+    inputs, output o, log-sum-exp lse (swa_attn_fwd(..., return_lse=True))
+    and the output's gradient d_o."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (d_o, "d_o")):
+        _check(t, n, dim=4)
+    _check(lse, "lse", dtype=torch.float32, dim=3)
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    if o.shape != q.shape or d_o.shape != q.shape or k.shape != (B, Hkv, N, d) or v.shape != k.shape \
+            or lse.shape != (B, Hq, N):
+        raise ValueError("backward shapes do not agree")
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    need = attn_bwd_workspace_bytes(B, Hq, N)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    st = library().swa_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(d_o), _ptr(lse), _ptr(dq), _ptr(dk),
+                                _ptr(dv), B, Hq, Hkv, N, d, int(window), float(scale), _ptr(workspace),
+                                workspace.numel() * workspace.element_size(), _stream(stream))
+    _raise(st, "swa_attn_bwd")
+    return dq, dk, dv
 
 
 def diff_attn_fwd(q1, k1, q2, k2, v, lam, window: int | None = None, scale: float | None = None, out=None,

@@ -14,7 +14,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
-SOURCES = ["api.cu", "prefill.cu", "decode.cu", "diff_decode.cu"]
+SOURCES = ["api.cu", "prefill.cu", "decode.cu", "diff_decode.cu", "backward.cu"]
 HEADERS = ["ptx.cuh", "schedule.cuh", "internal.h"]
 LIB = os.path.join(HERE, "libswa_attn.so")
 

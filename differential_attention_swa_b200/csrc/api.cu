@@ -316,6 +316,48 @@ swa_status_t swa_diff_decode_step(const void* q1, const void* q2, const void* k1
   return e == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
 }
 
+size_t swa_attn_bwd_workspace_bytes(int B, int Hq, int N) {
+  if (B < 1 || Hq < 1 || N < 1) return 0;
+  const int64_t npad = ((int64_t)N + 127) / 128 * 128;
+  return (size_t)(2 * (int64_t)B * Hq * npad * (int64_t)sizeof(float));
+}
+
+swa_status_t swa_attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* d_o,
+                          const float* lse, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N, int d, int W,
+                          float scale, void* workspace, size_t ws_bytes, void* stream) {
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(d_o) || !aligned16(dq) ||
+      !aligned16(dk) || !aligned16(dv) || lse == nullptr || (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return SWA_ERR_INVALID_ARG;
+  if (B < 1 || Hq < 1 || Hkv < 1 || N < 1 || W < 1 || Hq % Hkv != 0) return SWA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return SWA_ERR_INVALID_ARG;
+  if ((int64_t)B * Hq > (1 << 30) / 8 || N > (1 << 30)) return SWA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return SWA_ERR_UNSUPPORTED;
+  if (!aligned16(workspace) || ws_bytes < swa_attn_bwd_workspace_bytes(B, Hq, N)) return SWA_ERR_INVALID_ARG;
+  if (!get_encoder()) return SWA_ERR_CUDA;
+  const int64_t nB = B;
+  BwdMaps m;
+  std::memset(&m, 0, sizeof(m));
+  const bool ok = encode_rows(&m.q, q, d, N, nB * Hq, d, (int64_t)N * d) &&
+                  encode_rows(&m.k, k, d, N, nB * Hkv, d, (int64_t)N * d) &&
+                  encode_rows(&m.v, v, d, N, nB * Hkv, d, (int64_t)N * d) &&
+                  encode_rows(&m.dO, d_o, d, N, nB * Hq, d, (int64_t)N * d);
+  if (!ok) return SWA_ERR_INVALID_ARG;
+  BwdParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.q = q; p.k = k; p.v = v; p.o = o; p.dO = d_o; p.dq = dq; p.dk = dk; p.dv = dv; p.lse = lse;
+  p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.N = N; p.W = W; p.G = Hq / Hkv;
+  p.nq = (N + 127) / 128;
+  p.npad = p.nq * 128;
+  p.lse2 = static_cast<float*>(workspace);
+  p.dd = p.lse2 + (int64_t)B * Hq * p.npad;
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.err_flag = device_error_ptr();
+  if (p.err_flag == nullptr) return SWA_ERR_CUDA;
+  cudaError_t e = launch_backward(m, p, d, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
+}
+
 int64_t swa_schedule(int kind, int N, int W, int stride, int Bq, int Bk, int32_t* qtile_offsets, int32_t* tiles,
                      int64_t cap) {
   if (N < 1 || Bq < 1 || Bk < 1 || kind < 0 || kind > 3) return -1;

@@ -1,0 +1,587 @@
+// backward.cu -- gradients of the sliding-window attention forward on sm_100a.
+//
+// The pages define the forward only (A = softmax(Q K^T * scale + log M) V,
+// "Learn: Sparse & Sliding-Window Attention", section 3); its training use
+// ("Attention Variants -- Sliding Window, Sparse, Differential", opening)
+// needs the gradients. This is the chain rule of that forward, in the
+// flash-attention arrangement that never stores the N x N matrices: with
+// the forward's log-sum-exp L_i and D_i = dO_i . O_i,
+//     P_ij  = exp(scale q_i.k_j - L_i) on attended cells, else 0
+//     dV_j  = sum_i P_ij dO_i,        dP_ij = dO_i . v_j
+//     dS_ij = P_ij (dP_ij - D_i)
+//     dQ_i  = scale sum_j dS_ij k_j,  dK_j = scale sum_i dS_ij q_i
+// over the same window mask, summed over the query heads of a KV head.
+//
+// Three kernels:
+//   bwd_prep      D_i and L_i * log2(e) per query row into a padded
+//                 workspace (one thread per row).
+//   bwd_dkdv      one CTA per (b, KV head, 128-key tile): K and V of the tile
+//                 stay in shared memory; for every query head of the group
+//                 and every query tile that sees the keys, S^T = K Q^T and
+//                 dP^T = V dO^T go to tensor memory, four warps (one key per
+//                 TMEM lane) turn them into P^T and dS^T (bf16, written back
+//                 over them), and dV += P^T dO, dK += dS^T Q accumulate in
+//                 tensor memory (A operand read from TMEM).
+//   bwd_dq        one CTA per (b, head, 128-query tile): Q and dO stay; for
+//                 every key tile of the row block's window, S = Q K^T and
+//                 dP = dO V^T, then dS (bf16 over S) and dQ += dS K.
+// Operand layouts follow the forward's: 128-byte swizzled TMA tiles,
+// K-major for the score products, MN-major for the products that run over
+// the 128 tile rows. Waits are bounded; a timeout records SWA_ERR_TIMEOUT.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "internal.h"
+#include "ptx.cuh"
+#include "schedule.cuh"
+
+namespace swa {
+
+namespace {
+
+constexpr int kBwdThreads = 192;  // producer, MMA, four elementwise warps
+constexpr int kBT = 128;          // rows of a query or key tile
+
+template <int D>
+struct BwdCfg {
+  static constexpr int kTile = kBT * D * 2;              // one tile of D bf16 columns
+  static constexpr int kStage = 2 * kTile + 2 * kBT * 4; // two tiles + two fp32 row tables
+  static constexpr int kStages = 2;
+  static constexpr int kOffA = 0;                        // the CTA's fixed tiles
+  static constexpr int kOffB = kTile;
+  static constexpr int kOffStages = 2 * kTile;
+  static constexpr int kOffBar = kOffStages + kStages * kStage;
+  static constexpr int kSmemBytes = kOffBar + 1024 + 1024;  // barriers area + alignment slack
+  static constexpr uint32_t kColS = 0;      // S (or S^T), then P / dS as bf16 pairs
+  static constexpr uint32_t kColDP = 128;   // dP (or dP^T), then dS^T as bf16 pairs
+  static constexpr uint32_t kColAcc = 256;  // dQ, or dV then dK
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+  static_assert(256 + 2 * D <= 512, "tensor memory");
+};
+
+struct BwdBar {
+  static constexpr int kFixed = 0;
+  static constexpr int kFull = 1;   // + stage
+  static constexpr int kEmpty = 3;  // + stage
+  static constexpr int kS = 5;      // score products of the step in TMEM
+  static constexpr int kP = 6;      // elementwise done: P / dS written
+  static constexpr int kAcc = 7;    // accumulators final
+  static constexpr int kFinal = 8;  // MMA drain on abort
+  static constexpr int kWordsOff = 256;
+};
+
+__device__ __forceinline__ void bwd_timeout(volatile int* abort_flag, int* err) {
+  *abort_flag = 1;
+  atomicExch(err, 4 /* SWA_ERR_TIMEOUT */);
+}
+
+// Query rows i of a key-tile / query-tile pair attended under the window:
+// key <= i, i - key < W, both below N.
+__device__ __forceinline__ bool bwd_attended(int i, int key, int W, int N) {
+  return key <= i && i - key < W && i < N && key < N;
+}
+
+// D_i = dO_i . O_i and L_i * log2(e), rows past N padded with zeros.
+template <int D>
+__global__ void __launch_bounds__(128) bwd_prep_kernel(const BwdParams p) {
+  const int64_t r = (int64_t)blockIdx.x * 128 + threadIdx.x;  // (b*Hq + hq) * npad + i
+  const int64_t total = (int64_t)p.B * p.Hq * p.npad;
+  if (r >= total) return;
+  const int64_t bh = r / p.npad;
+  const int i = (int)(r % p.npad);
+  float d = 0.f, l2 = 0.f;
+  if (i < p.N) {
+    const int64_t row = bh * p.N + i;
+    const uint4* o = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(p.o) + row * D);
+    const uint4* g = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(p.dO) + row * D);
+#pragma unroll 4
+    for (int c = 0; c < D / 8; ++c) {
+      const uint4 a = o[c], b = g[c];
+      const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        d = fmaf(__uint_as_float(wa[e] << 16), __uint_as_float(wb[e] << 16), d);
+        d = fmaf(__uint_as_float(wa[e] & 0xffff0000u), __uint_as_float(wb[e] & 0xffff0000u), d);
+      }
+    }
+    l2 = p.lse[row] * 1.4426950408889634f;
+  }
+  p.dd[r] = d;
+  p.lse2[r] = l2;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                    const __grid_constant__ BwdParams p) {
+  using C = BwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bars = sbase + C::kOffBar;
+  auto bar = [&](int i) -> uint32_t { return bars + 8u * i; };
+  uint32_t* words = reinterpret_cast<uint32_t*>(smem + C::kOffBar + BwdBar::kWordsOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(words + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  const int kt = blockIdx.x;
+  const int b = blockIdx.y / p.Hkv, hkv = blockIdx.y % p.Hkv;
+  // query tiles that see keys kt*128 .. kt*128+127: from the diagonal up to
+  // the last row whose window still reaches the tile's last key
+  const int qt_lo = kt;
+  const int Wc = imin(p.W, p.N);
+  const int reach = kt * kBT + kBT - 1 + Wc - 1;  // last query row that sees the tile's last key
+  const int qt_hi = imin(p.nq - 1, reach / kBT);
+  const int nqt = qt_hi - qt_lo + 1;
+  const int nsteps = p.G * nqt;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(BwdBar::kFixed), 1);
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(bar(BwdBar::kFull + s), 1);
+      mbar_init(bar(BwdBar::kEmpty + s), 1);
+    }
+    mbar_init(bar(BwdBar::kS), 1);
+    mbar_init(bar(BwdBar::kP), 128);
+    mbar_init(bar(BwdBar::kAcc), 1);
+    mbar_init(bar(BwdBar::kFinal), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(words), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = words[0];
+
+  if (warp == 0) {
+    // ------------------------------------------------------ producer ---
+    if (lane == 0) {
+      const int zkv = b * p.Hkv + hkv;
+      mbar_arrive_expect_tx(bar(BwdBar::kFixed), 2 * C::kTile);
+      for (int bx = 0; bx < D / 64; ++bx) {
+        tma_load_3d(sbase + C::kOffA + bx * 16384, &tm_k, bar(BwdBar::kFixed), bx * 64, kt * kBT, zkv);
+        tma_load_3d(sbase + C::kOffB + bx * 16384, &tm_v, bar(BwdBar::kFixed), bx * 64, kt * kBT, zkv);
+      }
+      int issued[C::kStages] = {0, 0};
+      for (int s = 0; s < nsteps; ++s) {
+        const int st = s & 1, use = s >> 1;
+        if (use > 0 && !mbar_wait(bar(BwdBar::kEmpty + st), (use - 1) & 1, abort_flag)) {
+          bwd_timeout(abort_flag, p.err_flag);
+          break;
+        }
+        const int hq = hkv * p.G + s / nqt, qt = qt_lo + s % nqt;
+        const int zq = b * p.Hq + hq;
+        const uint32_t base = sbase + C::kOffStages + st * C::kStage;
+        mbar_arrive_expect_tx(bar(BwdBar::kFull + st), 2 * C::kTile + 2 * kBT * 4);
+        for (int bx = 0; bx < D / 64; ++bx) {
+          tma_load_3d(base + bx * 16384, &tm_q, bar(BwdBar::kFull + st), bx * 64, qt * kBT, zq);
+          tma_load_3d(base + C::kTile + bx * 16384, &tm_do, bar(BwdBar::kFull + st), bx * 64, qt * kBT, zq);
+        }
+        const int64_t rt = (int64_t)zq * p.npad + qt * kBT;
+        bulk_load(base + 2 * C::kTile, p.lse2 + rt, kBT * 4, bar(BwdBar::kFull + st));
+        bulk_load(base + 2 * C::kTile + kBT * 4, p.dd + rt, kBT * 4, bar(BwdBar::kFull + st));
+        issued[st] = use + 1;
+      }
+      if (*abort_flag) {  // drain: every copy issued lands before the CTA may exit
+        mbar_wait_timed(bar(BwdBar::kFixed), 0);
+        for (int st = 0; st < C::kStages; ++st)
+          if (issued[st] > 0) mbar_wait_timed(bar(BwdBar::kFull + st), (issued[st] - 1) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    // ----------------------------------------------------------- MMA ---
+    if (lane == 0) {
+      const uint32_t idesc_s = idesc_bf16_f32(kBT, kBT, false);
+      const uint32_t idesc_acc = idesc_bf16_f32(kBT, D, true);
+      const uint64_t k_desc = sw128_desc(sbase + C::kOffA, 16, 1024);
+      const uint64_t v_desc = sw128_desc(sbase + C::kOffB, 16, 1024);
+      bool ok = mbar_wait(bar(BwdBar::kFixed), 0, abort_flag);
+      if (!ok) bwd_timeout(abort_flag, p.err_flag);
+      tc_fence_after();
+      for (int s = 0; ok && s <= nsteps; ++s) {
+        if (s > 0) {
+          // dV += P^T dO and dK += dS^T Q of the previous step
+          if (!mbar_wait(bar(BwdBar::kP), (s - 1) & 1, abort_flag)) {
+            bwd_timeout(abort_flag, p.err_flag);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t prev = sbase + C::kOffStages + ((s - 1) & 1) * C::kStage;
+          const uint64_t q_mn = sw128_desc(prev, 16384, 1024);
+          const uint64_t do_mn = sw128_desc(prev + C::kTile, 16384, 1024);
+#pragma unroll
+          for (int kk = 0; kk < kBT / 16; ++kk) {
+            const uint32_t acc = (s == 1 && kk == 0) ? 0u : 1u;
+            umma_bf16_ts(tmem + C::kColAcc, tmem + C::kColS + kk * 8, do_mn + (uint64_t)(kk * 2048 >> 4), idesc_acc,
+                         acc);
+            umma_bf16_ts(tmem + C::kColAcc + D, tmem + C::kColDP + kk * 8, q_mn + (uint64_t)(kk * 2048 >> 4),
+                         idesc_acc, acc);
+          }
+          umma_commit(bar(BwdBar::kEmpty + ((s - 1) & 1)));  // Q, dO and the row tables of step s-1 read
+        }
+        if (s == nsteps) {
+          umma_commit(bar(BwdBar::kAcc));
+          break;
+        }
+        if (!mbar_wait(bar(BwdBar::kFull + (s & 1)), (s >> 1) & 1, abort_flag)) {
+          bwd_timeout(abort_flag, p.err_flag);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t cur = sbase + C::kOffStages + (s & 1) * C::kStage;
+        const uint64_t q_k = sw128_desc(cur, 16, 1024);
+        const uint64_t do_k = sw128_desc(cur + C::kTile, 16, 1024);
+        // S^T = K Q^T and dP^T = V dO^T (rows: keys, columns: queries)
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t off = (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
+          umma_bf16_ss(tmem + C::kColS, k_desc + off, q_k + off, idesc_s, kk > 0 ? 1u : 0u);
+          umma_bf16_ss(tmem + C::kColDP, v_desc + off, do_k + off, idesc_s, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(bar(BwdBar::kS));
+      }
+      if (!ok || *abort_flag) {
+        umma_commit(bar(BwdBar::kFinal));
+        mbar_wait_timed(bar(BwdBar::kFinal), 0);
+      }
+    }
+  } else {
+    // --------------------------------------------------- elementwise ---
+    const int qw = warp & 3;             // TMEM lane quarter
+    const int kr = qw * 32 + lane;       // key row within the tile
+    const int key = kt * kBT + kr;
+    const uint32_t lane_addr = static_cast<uint32_t>(qw * 32) << 16;
+    const float sl2 = p.scale_log2;
+    bool ok = true;
+    for (int s = 0; s < nsteps; ++s) {
+      const int qt = qt_lo + s % nqt;
+      const bool got = mbar_wait(bar(BwdBar::kS), s & 1, abort_flag);
+      if (!__all_sync(0xffffffffu, got)) {
+        if (lane == 0) bwd_timeout(abort_flag, p.err_flag);
+        ok = false;
+        break;
+      }
+      // the row tables were written by the copy engine: acquire them from the
+      // stage's own barrier (complete already; the stage cannot be refilled
+      // before this step's P^T and dS^T are consumed)
+      const bool have = mbar_wait(bar(BwdBar::kFull + (s & 1)), (s >> 1) & 1, abort_flag);
+      if (!__all_sync(0xffffffffu, have)) {
+        if (lane == 0) bwd_timeout(abort_flag, p.err_flag);
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const float* lse2 = reinterpret_cast<const float*>(smem + C::kOffStages + (s & 1) * C::kStage + 2 * C::kTile);
+      const float* dd = lse2 + kBT;
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {  // two halves of 64 queries
+        float sv[64], dp[64];
+        uint32_t pk[32], dk[32];
+        tmem_ld64(tmem + lane_addr + C::kColS + 64 * h, sv);
+        tmem_ld64(tmem + lane_addr + C::kColDP + 64 * h, dp);
+#pragma unroll
+        for (int c = 0; c < 64; c += 2) {
+          const int c0 = 64 * h + c;
+          const int i0 = qt * kBT + c0;
+          const bool a0 = bwd_attended(i0, key, p.W, p.N), a1 = bwd_attended(i0 + 1, key, p.W, p.N);
+          const float p0 = a0 ? ex2_approx(fmaf(sv[c], sl2, -lse2[c0])) : 0.f;
+          const float p1 = a1 ? ex2_approx(fmaf(sv[c + 1], sl2, -lse2[c0 + 1])) : 0.f;
+          pk[c >> 1] = pack_bf16(p0, p1);
+          dk[c >> 1] = pack_bf16(p0 * (dp[c] - dd[c0]), p1 * (dp[c + 1] - dd[c0 + 1]));
+        }
+        // P^T over S^T and dS^T over dP^T as bf16 pairs: queries 64h .. 64h+63
+        // land in columns 32h .. 32h+31, all of them already read
+        tmem_st32_u(tmem + lane_addr + C::kColS + 32 * h, pk);
+        tmem_st32_u(tmem + lane_addr + C::kColDP + 32 * h, dk);
+      }
+      tc_fence_before();
+      mbar_arrive(bar(BwdBar::kP));
+    }
+    if (ok) {
+      const bool got = mbar_wait(bar(BwdBar::kAcc), 0, abort_flag);
+      if (!__all_sync(0xffffffffu, got)) {
+        if (lane == 0) bwd_timeout(abort_flag, p.err_flag);
+        ok = false;
+      }
+    }
+    if (ok) {
+      tc_fence_after();
+      const int64_t row = ((int64_t)(b * p.Hkv + hkv) * p.N + key) * D;
+      __nv_bfloat16* dv = reinterpret_cast<__nv_bfloat16*>(p.dv) + row;
+      __nv_bfloat16* dkp = reinterpret_cast<__nv_bfloat16*>(p.dk) + row;
+#pragma unroll 1
+      for (int c = 0; c < D; c += 32) {
+        float a[32], g[32];
+        tmem_ld32(tmem + lane_addr + C::kColAcc + c, a);
+        tmem_ld32(tmem + lane_addr + C::kColAcc + D + c, g);
+        if (key < p.N) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 8) {
+            st_global_v4(dv + c + e, pack_bf16(a[e], a[e + 1]), pack_bf16(a[e + 2], a[e + 3]),
+                         pack_bf16(a[e + 4], a[e + 5]), pack_bf16(a[e + 6], a[e + 7]));
+            st_global_v4(dkp + c + e, pack_bf16(g[e] * p.scale, g[e + 1] * p.scale),
+                         pack_bf16(g[e + 2] * p.scale, g[e + 3] * p.scale),
+                         pack_bf16(g[e + 4] * p.scale, g[e + 5] * p.scale),
+                         pack_bf16(g[e + 6] * p.scale, g[e + 7] * p.scale));
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                  const __grid_constant__ BwdParams p) {
+  using C = BwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bars = sbase + C::kOffBar;
+  auto bar = [&](int i) -> uint32_t { return bars + 8u * i; };
+  uint32_t* words = reinterpret_cast<uint32_t*>(smem + C::kOffBar + BwdBar::kWordsOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(words + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  const int qt = blockIdx.x;
+  const int b = blockIdx.y / p.Hq, hq = blockIdx.y % p.Hq;
+  const int hkv = hq / p.G;
+  // key tiles of the row block: from the tile holding the first row's
+  // window start to the diagonal tile
+  const int Wc = imin(p.W, p.N);
+  const int kt_lo = imax(0, qt * kBT - Wc + 1) / kBT;
+  const int nsteps = qt - kt_lo + 1;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(BwdBar::kFixed), 1);
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(bar(BwdBar::kFull + s), 1);
+      mbar_init(bar(BwdBar::kEmpty + s), 1);
+    }
+    mbar_init(bar(BwdBar::kS), 1);
+    mbar_init(bar(BwdBar::kP), 128);
+    mbar_init(bar(BwdBar::kAcc), 1);
+    mbar_init(bar(BwdBar::kFinal), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(words), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = words[0];
+
+  if (warp == 0) {
+    // ------------------------------------------------------ producer ---
+    if (lane == 0) {
+      const int zq = b * p.Hq + hq, zkv = b * p.Hkv + hkv;
+      mbar_arrive_expect_tx(bar(BwdBar::kFixed), 2 * C::kTile);
+      for (int bx = 0; bx < D / 64; ++bx) {
+        tma_load_3d(sbase + C::kOffA + bx * 16384, &tm_q, bar(BwdBar::kFixed), bx * 64, qt * kBT, zq);
+        tma_load_3d(sbase + C::kOffB + bx * 16384, &tm_do, bar(BwdBar::kFixed), bx * 64, qt * kBT, zq);
+      }
+      int issued[C::kStages] = {0, 0};
+      for (int s = 0; s < nsteps; ++s) {
+        const int st = s & 1, use = s >> 1;
+        if (use > 0 && !mbar_wait(bar(BwdBar::kEmpty + st), (use - 1) & 1, abort_flag)) {
+          bwd_timeout(abort_flag, p.err_flag);
+          break;
+        }
+        const int kt = kt_lo + s;
+        const uint32_t base = sbase + C::kOffStages + st * C::kStage;
+        mbar_arrive_expect_tx(bar(BwdBar::kFull + st), 2 * C::kTile);
+        for (int bx = 0; bx < D / 64; ++bx) {
+          tma_load_3d(base + bx * 16384, &tm_k, bar(BwdBar::kFull + st), bx * 64, kt * kBT, zkv);
+          tma_load_3d(base + C::kTile + bx * 16384, &tm_v, bar(BwdBar::kFull + st), bx * 64, kt * kBT, zkv);
+        }
+        issued[st] = use + 1;
+      }
+      if (*abort_flag) {
+        mbar_wait_timed(bar(BwdBar::kFixed), 0);
+        for (int st = 0; st < C::kStages; ++st)
+          if (issued[st] > 0) mbar_wait_timed(bar(BwdBar::kFull + st), (issued[st] - 1) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    // ----------------------------------------------------------- MMA ---
+    if (lane == 0) {
+      const uint32_t idesc_s = idesc_bf16_f32(kBT, kBT, false);
+      const uint32_t idesc_acc = idesc_bf16_f32(kBT, D, true);
+      const uint64_t q_desc = sw128_desc(sbase + C::kOffA, 16, 1024);
+      const uint64_t do_desc = sw128_desc(sbase + C::kOffB, 16, 1024);
+      bool ok = mbar_wait(bar(BwdBar::kFixed), 0, abort_flag);
+      if (!ok) bwd_timeout(abort_flag, p.err_flag);
+      tc_fence_after();
+      for (int s = 0; ok && s <= nsteps; ++s) {
+        if (s > 0) {
+          // dQ += dS K of the previous step (dS as bf16 pairs over S)
+          if (!mbar_wait(bar(BwdBar::kP), (s - 1) & 1, abort_flag)) {
+            bwd_timeout(abort_flag, p.err_flag);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t k_mn = sw128_desc(sbase + C::kOffStages + ((s - 1) & 1) * C::kStage, 16384, 1024);
+#pragma unroll
+          for (int kk = 0; kk < kBT / 16; ++kk)
+            umma_bf16_ts(tmem + C::kColAcc, tmem + C::kColS + kk * 8, k_mn + (uint64_t)(kk * 2048 >> 4), idesc_acc,
+                         (s == 1 && kk == 0) ? 0u : 1u);
+          umma_commit(bar(BwdBar::kEmpty + ((s - 1) & 1)));  // K and V of step s-1 read
+        }
+        if (s == nsteps) {
+          umma_commit(bar(BwdBar::kAcc));
+          break;
+        }
+        if (!mbar_wait(bar(BwdBar::kFull + (s & 1)), (s >> 1) & 1, abort_flag)) {
+          bwd_timeout(abort_flag, p.err_flag);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t cur = sbase + C::kOffStages + (s & 1) * C::kStage;
+        const uint64_t k_k = sw128_desc(cur, 16, 1024);
+        const uint64_t v_k = sw128_desc(cur + C::kTile, 16, 1024);
+        // S = Q K^T and dP = dO V^T (rows: queries, columns: keys)
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t off = (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
+          umma_bf16_ss(tmem + C::kColS, q_desc + off, k_k + off, idesc_s, kk > 0 ? 1u : 0u);
+          umma_bf16_ss(tmem + C::kColDP, do_desc + off, v_k + off, idesc_s, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(bar(BwdBar::kS));
+      }
+      if (!ok || *abort_flag) {
+        umma_commit(bar(BwdBar::kFinal));
+        mbar_wait_timed(bar(BwdBar::kFinal), 0);
+      }
+    }
+  } else {
+    // --------------------------------------------------- elementwise ---
+    const int qw = warp & 3;
+    const int r = qw * 32 + lane;  // query row within the tile
+    const int i = qt * kBT + r;
+    const uint32_t lane_addr = static_cast<uint32_t>(qw * 32) << 16;
+    const float sl2 = p.scale_log2;
+    const int64_t rt = (int64_t)(b * p.Hq + hq) * p.npad + i;  // padded: always in bounds
+    const float lse2 = p.lse2[rt], dd = p.dd[rt];
+    bool ok = true;
+    for (int s = 0; s < nsteps; ++s) {
+      const int kt = kt_lo + s;
+      const bool got = mbar_wait(bar(BwdBar::kS), s & 1, abort_flag);
+      if (!__all_sync(0xffffffffu, got)) {
+        if (lane == 0) bwd_timeout(abort_flag, p.err_flag);
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {  // two halves of 64 keys
+        float sv[64], dp[64];
+        uint32_t pk[32];
+        tmem_ld64(tmem + lane_addr + C::kColS + 64 * h, sv);
+        tmem_ld64(tmem + lane_addr + C::kColDP + 64 * h, dp);
+#pragma unroll
+        for (int c = 0; c < 64; c += 2) {
+          const int key = kt * kBT + 64 * h + c;
+          const bool a0 = bwd_attended(i, key, p.W, p.N), a1 = bwd_attended(i, key + 1, p.W, p.N);
+          const float p0 = a0 ? ex2_approx(fmaf(sv[c], sl2, -lse2)) : 0.f;
+          const float p1 = a1 ? ex2_approx(fmaf(sv[c + 1], sl2, -lse2)) : 0.f;
+          pk[c >> 1] = pack_bf16(p0 * (dp[c] - dd), p1 * (dp[c + 1] - dd));
+        }
+        // dS over S as bf16 pairs: keys 64h .. 64h+63 in columns 32h .. 32h+31
+        tmem_st32_u(tmem + lane_addr + C::kColS + 32 * h, pk);
+      }
+      tc_fence_before();
+      mbar_arrive(bar(BwdBar::kP));
+    }
+    if (ok) {
+      const bool got = mbar_wait(bar(BwdBar::kAcc), 0, abort_flag);
+      if (!__all_sync(0xffffffffu, got)) {
+        if (lane == 0) bwd_timeout(abort_flag, p.err_flag);
+        ok = false;
+      }
+    }
+    if (ok) {
+      tc_fence_after();
+      __nv_bfloat16* dq = reinterpret_cast<__nv_bfloat16*>(p.dq) + ((int64_t)(b * p.Hq + hq) * p.N + i) * D;
+#pragma unroll 1
+      for (int c = 0; c < D; c += 32) {
+        float a[32];
+        tmem_ld32(tmem + lane_addr + C::kColAcc + c, a);
+        if (i < p.N) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 8)
+            st_global_v4(dq + c + e, pack_bf16(a[e] * p.scale, a[e + 1] * p.scale),
+                         pack_bf16(a[e + 2] * p.scale, a[e + 3] * p.scale),
+                         pack_bf16(a[e + 4] * p.scale, a[e + 5] * p.scale),
+                         pack_bf16(a[e + 6] * p.scale, a[e + 7] * p.scale));
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+template <int D>
+cudaError_t launch_bwd_d(const BwdMaps& m, const BwdParams& p, cudaStream_t stream) {
+  using C = BwdCfg<D>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         C::kSmemBytes);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  const int64_t rows = (int64_t)p.B * p.Hq * p.npad;
+  bwd_prep_kernel<D><<<(unsigned)((rows + 127) / 128), 128, 0, stream>>>(p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int nk = p.nq;  // key tiles of 128 (same count as query tiles)
+  bwd_dkdv_kernel<D><<<dim3(nk, p.B * p.Hkv), kBwdThreads, C::kSmemBytes, stream>>>(m.q, m.k, m.v, m.dO, p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  bwd_dq_kernel<D><<<dim3(p.nq, p.B * p.Hq), kBwdThreads, C::kSmemBytes, stream>>>(m.q, m.k, m.v, m.dO, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_backward(const BwdMaps& m, const BwdParams& p, int d, cudaStream_t stream) {
+  if (d == 128) return launch_bwd_d<128>(m, p, stream);
+  if (d == 64) return launch_bwd_d<64>(m, p, stream);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace swa

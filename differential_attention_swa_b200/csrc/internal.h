@@ -37,6 +37,23 @@ struct PrefillParams {
   int* err_flag;  // device word that receives SWA_ERR_TIMEOUT
 };
 
+// Backward of the window attention (dQ, dK, dV from dO and the forward's
+// O and log-sum-exp). The workspace holds D_i and L_i log2(e) per query row,
+// padded to whole 128-row tiles (npad rows per head).
+struct BwdParams {
+  const void *q, *k, *v, *o, *dO;
+  void *dq, *dk, *dv;
+  const float* lse;
+  float *lse2, *dd;
+  int B, Hq, Hkv, N, W, G, nq, npad;
+  float scale, scale_log2;
+  int* err_flag;
+};
+struct BwdMaps {
+  CUtensorMap q, k, v, dO;
+};
+cudaError_t launch_backward(const BwdMaps& m, const BwdParams& p, int d, cudaStream_t stream);
+
 // Row map of a strided view (dilated windows): row i of the problem is row
 // off + i*mul of a head holding n rows, which is where its log-sum-exp goes.
 struct RowMap {

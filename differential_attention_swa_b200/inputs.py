@@ -65,7 +65,7 @@ def diff_decode_inputs(T, B, Hq, Hkv, dk, dv, W, seed: int = 0):
 @dataclass(frozen=True)
 class Workload:
     name: str
-    kind: str  # "swa", "strided", "global", "dilated", "diff", "decode", "diff_decode"
+    kind: str  # "swa", "strided", "global", "dilated", "swa_bwd", "diff", "decode", "diff_decode"
     B: int
     Hq: int
     Hkv: int
@@ -97,6 +97,8 @@ WORKLOADS = {
     "local_strided_prefill": Workload("local_strided_prefill", "strided", 1, 16, 16, 16384, 64, 128, S=128),
     "diff_causal": Workload("diff_causal", "diff", 1, 16, 16, 4096, 64, 4096, dv=128, lam=0.8),
     "gemma_swa_prefill": Workload("gemma_swa_prefill", "swa", 1, 16, 8, 131072, 128, 1024),
+    # the backward of the Mistral-style window attention (gradients of Q, K, V)
+    "mistral_swa_backward": Workload("mistral_swa_backward", "swa_bwd", 2, 32, 8, 8192, 128, 4096),
     # window + global tokens with a Longformer-like shape (16 heads of 64,
     # a 512-token window, 64 global tokens at the start); S carries g
     "longformer_global_prefill": Workload("longformer_global_prefill", "global", 1, 16, 16, 16384, 64, 512, S=64),

@@ -236,6 +236,31 @@ swa_status_t swa_decode_step_static(const void* q, const void* k_new, const void
                                     int B, int Hq, int Hkv, int d, int W, float scale,
                                     void* stream);
 
+/* Backward of swa_attn_fwd: the gradients dQ, dK, dV of a loss whose
+ * gradient with respect to the output is dO.
+ * The pages define the forward only ("Learn: Sparse & Sliding-Window
+ * Attention", section 3: A = softmax(Q K^T * scale + log M) V); this is its
+ * chain rule under the same window mask, with P = exp(scale Q K^T - L) from
+ * the forward's log-sum-exp L, D = rowsum(dO * O), dS = P * (dO V^T - D):
+ *     dV = P^T dO,   dQ = scale dS K,   dK = scale dS^T Q,
+ * dK and dV summed over the query heads of each KV head.
+ *   q, o, d_o [B,Hq,N,d]; k, v [B,Hkv,N,d] bf16 (device, read only): the
+ *     forward's inputs and output and the output's gradient;
+ *   lse [B,Hq,N] fp32 (device): the forward's log-sum-exp (swa_attn_fwd
+ *     with a non-NULL lse);
+ *   dq [B,Hq,N,d], dk, dv [B,Hkv,N,d] bf16 (device, written);
+ *   d in {64, 128}; W >= 1 (W >= N is full causal); Hq % Hkv == 0;
+ *   workspace: device, 16-byte aligned, at least
+ *     swa_attn_bwd_workspace_bytes(B, Hq, N) bytes (caller-owned).
+ * Three kernels run on `stream`: row terms, dK/dV, dQ. */
+swa_status_t swa_attn_bwd(const void* q, const void* k, const void* v, const void* o,
+                          const void* d_o, const float* lse, void* dq, void* dk, void* dv, int B,
+                          int Hq, int Hkv, int N, int d, int W, float scale, void* workspace,
+                          size_t ws_bytes, void* stream);
+
+/* Scratch bytes swa_attn_bwd needs (0 on bad sizes). */
+size_t swa_attn_bwd_workspace_bytes(int B, int Hq, int N);
+
 /* Prefill with debug outputs. kind 0 = sliding window (stride ignored),
  * kind 1 = local + strided, kind 3 = window + global tokens (stride carries
  * n_global). Same arithmetic as swa_attn_fwd / strided_attn_fwd /

@@ -1,0 +1,74 @@
+"""The backward of the window attention (swa_attn_bwd) against the oracle's
+fp64 chain rule, on the same seeded inputs. The kernel uses its own forward
+output and log-sum-exp and rounds P and dS to bf16 before the products that
+consume them (as the forward rounds P), so its error grows with the number
+of attended keys; the bar is relative to each gradient's largest entry."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import differential_attention_swa_b200 as swa
+from differential_attention_swa_b200.inputs import attn_inputs, randn_bf16
+
+pytestmark = pytest.mark.gpu
+
+# bf16 products (P, dS) and bf16 outputs: each term carries a relative
+# error of about 2^-9; the sums stay within ~1 % of the largest entry
+REL_MAX = 2e-2
+REL_MEAN = 2e-3
+# where a gradient is exactly zero (window 1: dS = P (dP - D) = 0 because
+# D = dO . O = dO . v_i = dP), only rounding residue remains
+ABS_FLOOR = 1e-4
+
+
+def compare_grad(got, want, what):
+    got = got.float().cpu().numpy().astype(np.float64).reshape(want.shape)
+    assert np.isfinite(got).all(), f"{what}: non-finite"
+    scale = max(np.abs(want).max(), ABS_FLOOR / REL_MAX)
+    diff = np.abs(got - want)
+    assert diff.max() <= REL_MAX * scale and diff.mean() <= REL_MEAN * scale, \
+        f"{what}: max {diff.max():.3e} mean {diff.mean():.3e} (largest entry {scale:.3e})"
+    return diff.max() / scale
+
+
+def run(B, Hq, Hkv, N, d, W, seed):
+    q, k, v = attn_inputs(B, Hq, Hkv, N, d, seed=seed)
+    d_o = randn_bf16((B, Hq, N, d), seed + 10)
+    qd, kd, vd, dod = (t.cuda() for t in (q, k, v, d_o))
+    o, lse = swa.swa_attn_fwd(qd, kd, vd, W, return_lse=True)
+    dq, dk, dv = swa.swa_attn_bwd(qd, kd, vd, o, dod, lse, W)
+    torch.cuda.synchronize()
+    assert swa.last_device_error() == swa.OK
+    return (q, k, v, d_o), (dq, dk, dv)
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,N,d,W", [
+    (1, 2, 2, 256, 64, 64),      # two tiles, window of half a tile
+    (1, 4, 2, 300, 128, 100),    # ragged tail, GQA group 2
+    (2, 2, 1, 200, 64, 5000),    # window beyond N: causal, group 2
+    (1, 2, 2, 129, 128, 1),      # window 1, one row in the last tile
+    (1, 6, 2, 257, 64, 130),     # group 3, window just over a tile
+    (1, 8, 1, 384, 128, 256),    # group 8, three tiles
+])
+def test_backward_vs_oracle(orc, B, Hq, Hkv, N, d, W):
+    (q, k, v, d_o), (dq, dk, dv) = run(B, Hq, Hkv, N, d, W, seed=N + W)
+    rq, rk, rv = orc.attention_bwd("swa", q, k, v, d_o, W=W, scale=1 / math.sqrt(d))
+    compare_grad(dq, rq, "dq")
+    compare_grad(dk, rk, "dk")
+    compare_grad(dv, rv, "dv")
+
+
+def test_backward_sampled_rows_at_size(orc):
+    """A Mistral-like head shape at N = 4096 (W = 1024, GQA group 4): sampled
+    rows of dQ and of dK/dV, each from the oracle's per-row chain rule."""
+    B, Hq, Hkv, N, d, W = 1, 8, 2, 4096, 128, 1024
+    (q, k, v, d_o), (dq, dk, dv) = run(B, Hq, Hkv, N, d, W, seed=3)
+    rng = np.random.default_rng(4)
+    qr = np.unique(np.concatenate([rng.integers(0, B * Hq * N, 40), [0, N - 1, 128, 2 * N + 1023]]))
+    kr = np.unique(np.concatenate([rng.integers(0, B * Hkv * N, 6), [0, N - 1, N + 127]]))
+    rq, rk, rv = orc.attention_bwd("swa", q, k, v, d_o, W=W, scale=1 / math.sqrt(d), dq_rows=qr, dkv_rows=kr)
+    compare_grad(dq.reshape(-1, d)[torch.from_numpy(qr).cuda()], rq, "dq rows")
+    compare_grad(dk.reshape(-1, d)[torch.from_numpy(kr).cuda()], rk, "dk rows")
+    compare_grad(dv.reshape(-1, d)[torch.from_numpy(kr).cuda()], rv, "dv rows")
