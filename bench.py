@@ -37,6 +37,7 @@ PREFILL_SOURCES = ["differential_attention_swa_b200/csrc/prefill.cu", "different
                    "differential_attention_swa_b200/csrc/schedule.cuh"]
 DECODE_SOURCES = ["differential_attention_swa_b200/csrc/decode.cu", "differential_attention_swa_b200/csrc/ptx.cuh"]
 DIFF_DECODE_SOURCES = ["differential_attention_swa_b200/csrc/diff_decode.cu", "differential_attention_swa_b200/csrc/ptx.cuh"]
+BWD_SOURCES = ["differential_attention_swa_b200/csrc/backward.cu", "differential_attention_swa_b200/csrc/ptx.cuh"]
 
 
 # ------------------------------------------------------------ host logic --
@@ -448,10 +449,13 @@ def measure_variants(args, rank, peaks, flush, stream):
         ms = time_steps(fn, reps, 3, flush, stream)
         mean_ms = sum(ms) / len(ms)
         tf = flops / (mean_ms * 1e-3) / 1e12
+        traffic = (profiled_traffic("backward_swa_mistral.md", BWD_SOURCES) if name == "mistral_swa_backward"
+                   else None)
         out[name] = {"value": round(tf, 3), "unit": "TFLOP/s", "ms_per_step": round(mean_ms, 4), "steps": reps,
                      "algorithmic_flops": flops,
                      "roofline": {"bound": "tensor", "achieved": round(tf, 2), "peak": peaks["bf16_tflops"],
-                                  "unit": "TFLOP/s", "frac": round(tf / peaks["bf16_tflops"], 4), "traffic": None},
+                                  "unit": "TFLOP/s", "frac": round(tf / peaks["bf16_tflops"], 4),
+                                  "traffic": traffic},
                      "launches": reps}
         del ins, o, fn
         torch.cuda.empty_cache()
