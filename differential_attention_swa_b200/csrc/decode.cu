@@ -32,7 +32,11 @@
 namespace swa {
 
 constexpr int kDecThreads = 128;  // 4 warps
-constexpr int kDecUnroll = 4;     // rows in flight per lane group
+constexpr int kDecUnroll = 8;     // rows in flight per lane group
+// registers capped so that 4 CTAs share an SM for groups of 1-2 query heads
+// (larger groups hold more state per lane: 2 CTAs at G = 4, no cap at 8)
+template <int G>
+constexpr int dec_min_blocks() { return G <= 2 ? 4 : (G == 4 ? 2 : 1); }
 
 __device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
   uint4 r;
@@ -57,8 +61,13 @@ __device__ __forceinline__ int imin_dec(int a, int b) { return a < b ? a : b; }
 __host__ __device__ constexpr int partial_stride(int d) { return d + 4; }
 
 template <int D, int G>
-__global__ void __launch_bounds__(kDecThreads)
+__global__ void __launch_bounds__(kDecThreads, dec_min_blocks<G>())
     decode_split_kernel(const DecodeParams p) {
+  // a step may start while the previous step's merge runs; its partials and
+  // cache writes wait until that grid is complete (programmatic dependent
+  // launch), and the merge that follows may launch early
+  grid_dependency_wait();
+  launch_dependents();
   constexpr int LPR = D / 8;         // lanes per cache row
   constexpr int RPW = 32 / LPR;      // rows per warp per load
   constexpr int ROWS_PER_ITER = 4 * RPW * kDecUnroll;
@@ -224,6 +233,7 @@ __global__ void __launch_bounds__(kDecThreads)
 template <int D>
 __global__ void __launch_bounds__(D)
     decode_combine_kernel(const DecodeParams p) {
+  grid_dependency_wait();  // the split kernel's partials are complete and visible
   const int bh = blockIdx.x;  // b * Hq + hq
   const int c = threadIdx.x;
   const float* recs = p.partial + (int64_t)bh * p.nsplit * partial_stride(D);
@@ -241,7 +251,9 @@ __global__ void __launch_bounds__(D)
 
 int decode_nsplit(int B, int Hkv, int W) {
   const int groups = B * Hkv;
-  int ns = (8 * 148 + groups - 1) / groups;  // aim for several CTAs per SM
+  // about 24 CTAs per SM in total (measured best on the 64 x 8 x 1024-slot
+  // step among 8, 16, 24 and 32), each a whole number of 64-slot blocks
+  int ns = (24 * 148 + groups - 1) / groups;
   if (ns < 1) ns = 1;
   int chunk = (W + ns - 1) / ns;
   chunk = ((chunk + 63) / 64) * 64;           // whole iterations of the load loop
@@ -261,10 +273,32 @@ size_t decode_partial_bytes(int B, int Hq, int Hkv, int d, int slots) {
 template <int D, int G>
 static cudaError_t launch_g(DecodeParams p, cudaStream_t stream) {
   dim3 grid(p.nsplit, p.B * p.Hkv);
-  decode_split_kernel<D, G><<<grid, kDecThreads, 0, stream>>>(p);
+  cudaLaunchAttribute pdl;
+  pdl.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl.val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t scfg = {};
+  scfg.gridDim = grid;
+  scfg.blockDim = dim3(kDecThreads);
+  scfg.dynamicSmemBytes = 0;
+  scfg.stream = stream;
+  scfg.attrs = &pdl;
+  scfg.numAttrs = 1;
+  cudaLaunchKernelEx(&scfg, decode_split_kernel<D, G>, p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  decode_combine_kernel<D><<<p.B * p.Hq, D, 0, stream>>>(p);
+  // the merge may launch while the split grid drains; it waits on the
+  // device for the split grid's partials (programmatic dependent launch)
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.B * p.Hq);
+  cfg.blockDim = dim3(D);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr.val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  cudaLaunchKernelEx(&cfg, decode_combine_kernel<D>, p);
   return cudaGetLastError();
 }
 

@@ -83,6 +83,11 @@ __device__ __forceinline__ void merge_state(float& m, float& l, float* acc, int 
 
 template <int G>
 __global__ void __launch_bounds__(kDdThreads, dd_min_blocks<G>()) diff_decode_split_kernel(const DiffDecodeParams p) {
+  // a step may start while the previous step's merge runs; its partials and
+  // cache writes wait until that grid is complete (programmatic dependent
+  // launch), and the merge that follows may launch early
+  grid_dependency_wait();
+  launch_dependents();
   const int split = blockIdx.x;
   const int bk = blockIdx.y;  // b * Hkv + hkv
   const int b = bk / p.Hkv;
@@ -253,6 +258,7 @@ __global__ void __launch_bounds__(kDdThreads, dd_min_blocks<G>()) diff_decode_sp
 }
 
 __global__ void __launch_bounds__(kDv) diff_decode_combine_kernel(const DiffDecodeParams p) {
+  grid_dependency_wait();  // the split kernel's partials are complete and visible
   const int bh = blockIdx.x;  // b * Hq + hq
   const int c = threadIdx.x;
   const float* recs = p.partial + (int64_t)bh * p.nsplit * diff_partial_stride();
@@ -278,10 +284,32 @@ __global__ void __launch_bounds__(kDv) diff_decode_combine_kernel(const DiffDeco
 template <int G>
 cudaError_t launch_dd(const DiffDecodeParams& p, cudaStream_t stream) {
   dim3 grid(p.nsplit, p.B * p.Hkv);
-  diff_decode_split_kernel<G><<<grid, kDdThreads, 0, stream>>>(p);
+  cudaLaunchAttribute pdl;
+  pdl.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl.val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t scfg = {};
+  scfg.gridDim = grid;
+  scfg.blockDim = dim3(kDdThreads);
+  scfg.dynamicSmemBytes = 0;
+  scfg.stream = stream;
+  scfg.attrs = &pdl;
+  scfg.numAttrs = 1;
+  cudaLaunchKernelEx(&scfg, diff_decode_split_kernel<G>, p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  diff_decode_combine_kernel<<<p.B * p.Hq, kDv, 0, stream>>>(p);
+  // the merge may launch while the split grid drains; it waits on the
+  // device for the split grid's partials (programmatic dependent launch)
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.B * p.Hq);
+  cfg.blockDim = dim3(kDv);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr.val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  cudaLaunchKernelEx(&cfg, diff_decode_combine_kernel, p);
   return cudaGetLastError();
 }
 

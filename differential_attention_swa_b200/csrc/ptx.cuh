@@ -99,6 +99,13 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* m, 
       : "memory");
 }
 
+// Programmatic dependent launch: a grid launched with programmatic stream
+// serialization may start before the previous grid on the stream finishes;
+// grid_dependency_wait() blocks until that grid has completed and its
+// memory is visible, and launch_dependents() lets the next grid start.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // Untiled bulk copy global -> shared (no multicast); completion counted in
 // bytes on `bar`. dst, src and bytes are multiples of 16.
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
