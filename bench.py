@@ -212,11 +212,18 @@ def prefill_workload(name, rank):
 
         q, k, v = (t.cuda() for t in attn_inputs(w.B, w.Hq, w.Hkv, w.N, w.d, seed=seed))
         d_o = randn_bf16((w.B, w.Hq, w.N, w.d), seed + 3).cuda()
-        o, lse = swa.swa_attn_fwd(q, k, v, w.W, return_lse=True)  # the forward, outside the timed region
-        ws = torch.empty(swa.attn_bwd_workspace_bytes(w.B, w.Hq, w.N), dtype=torch.uint8, device="cuda")
+        # the forward, outside the timed region (S > 0: the local + strided mask)
+        if w.S:
+            o, lse = swa.strided_attn_fwd(q, k, v, w.W, w.S, return_lse=True)
+            ws_bytes = int(swa.library().strided_attn_bwd_workspace_bytes(w.B, w.Hq, w.Hkv, w.N, w.d, w.S))
+            nnz = swa.count_nonmasked(swa.MASK_STRIDED, w.N, w.W, w.S)
+        else:
+            o, lse = swa.swa_attn_fwd(q, k, v, w.W, return_lse=True)
+            ws_bytes = swa.attn_bwd_workspace_bytes(w.B, w.Hq, w.N)
+            nnz = swa.count_nonmasked(swa.MASK_WINDOW, w.N, w.W)
+        ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
         out = None
-        fn = lambda: swa.swa_attn_bwd(q, k, v, o, d_o, lse, w.W, workspace=ws)
-        nnz = swa.count_nonmasked(swa.MASK_WINDOW, w.N, w.W)
+        fn = lambda: swa.swa_attn_bwd(q, k, v, o, d_o, lse, w.W, workspace=ws, stride=w.S)
         # the usual accounting: scores, dP, dV, dQ, dK = 5 products of 2*d per cell
         flops = 10 * w.d * nnz * w.B * w.Hq
         ins = [q, k, v, o, lse, d_o, ws]
@@ -444,7 +451,7 @@ def measure_variants(args, rank, peaks, flush, stream):
     out = {}
     reps = max(5, min(args.steps, 10))
     for name in ("local_strided_prefill", "diff_causal", "gemma_swa_prefill", "longformer_global_prefill",
-                 "longformer_dilated_prefill", "mistral_swa_backward"):
+                 "longformer_dilated_prefill", "mistral_swa_backward", "local_strided_backward"):
         w, fn, flops, ins, o = prefill_workload(name, rank)
         ms = time_steps(fn, reps, 3, flush, stream)
         mean_ms = sum(ms) / len(ms)

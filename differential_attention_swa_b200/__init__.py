@@ -64,6 +64,10 @@ def library() -> ctypes.CDLL:
     lib.swa_attn_bwd.restype = I
     lib.swa_attn_bwd_workspace_bytes.argtypes = [I, I, I]
     lib.swa_attn_bwd_workspace_bytes.restype = SZ
+    lib.strided_attn_bwd.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, F, P, SZ, P]
+    lib.strided_attn_bwd.restype = I
+    lib.strided_attn_bwd_workspace_bytes.argtypes = [I, I, I, I, I, I]
+    lib.strided_attn_bwd_workspace_bytes.restype = SZ
     lib.diff_attn_fwd.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, F, P]
     lib.swa_decode_step.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, F, P, SZ, P]
     lib.swa_decode_workspace_bytes.argtypes = [I, I, I, I, I]
@@ -182,10 +186,12 @@ def attn_bwd_workspace_bytes(B: int, Hq: int, N: int) -> int:
     return int(library().swa_attn_bwd_workspace_bytes(B, Hq, N))
 
 
-def swa_attn_bwd(q, k, v, o, d_o, lse, window: int, scale: float | None = None, workspace=None, stream=None):
+def swa_attn_bwd(q, k, v, o, d_o, lse, window: int, scale: float | None = None, workspace=None, stream=None,
+                 stride: int = 0):
     """Gradients (dq, dk, dv) of the window attention forward, given its
     inputs, output o, log-sum-exp lse (swa_attn_fwd(..., return_lse=True))
-    and the output's gradient d_o."""
+    and the output's gradient d_o. With stride >= 1: the backward of the
+    local + strided forward (strided_attn_fwd)."""
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (d_o, "d_o")):
         _check(t, n, dim=4)
     _check(lse, "lse", dtype=torch.float32, dim=3)
@@ -195,14 +201,22 @@ def swa_attn_bwd(q, k, v, o, d_o, lse, window: int, scale: float | None = None, 
             or lse.shape != (B, Hq, N):
         raise ValueError("backward shapes do not agree")
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    need = attn_bwd_workspace_bytes(B, Hq, N)
+    if stride:
+        need = int(library().strided_attn_bwd_workspace_bytes(B, Hq, Hkv, N, d, int(stride)))
+    else:
+        need = attn_bwd_workspace_bytes(B, Hq, N)
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
     scale = 1.0 / math.sqrt(d) if scale is None else scale
-    st = library().swa_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(d_o), _ptr(lse), _ptr(dq), _ptr(dk),
-                                _ptr(dv), B, Hq, Hkv, N, d, int(window), float(scale), _ptr(workspace),
-                                workspace.numel() * workspace.element_size(), _stream(stream))
-    _raise(st, "swa_attn_bwd")
+    common = (_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(d_o), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv), B, Hq, Hkv,
+              N, d, int(window))
+    tail = (float(scale), _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+    if stride:
+        st = library().strided_attn_bwd(*common, int(stride), *tail)
+        _raise(st, "strided_attn_bwd")
+    else:
+        st = library().swa_attn_bwd(*common, *tail)
+        _raise(st, "swa_attn_bwd")
     return dq, dk, dv
 
 

@@ -206,6 +206,58 @@ swa_status_t run_decode(const void* q, const void* k_new, const void* v_new, voi
   cudaError_t e = launch_decode(p, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
 }
+// Backward of the window (S = 0) or local + strided (S >= 1) attention.
+swa_status_t run_bwd(const void* q, const void* k, const void* v, const void* o, const void* d_o, const float* lse,
+                     void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N, int d, int W, int S, float scale,
+                     void* workspace, size_t ws_bytes, void* stream) {
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(d_o) || !aligned16(dq) ||
+      !aligned16(dk) || !aligned16(dv) || lse == nullptr || (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return SWA_ERR_INVALID_ARG;
+  if (B < 1 || Hq < 1 || Hkv < 1 || N < 1 || W < 1 || S < 0 || Hq % Hkv != 0) return SWA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return SWA_ERR_INVALID_ARG;
+  if ((int64_t)B * Hq > (1 << 30) / 8 || N > (1 << 30)) return SWA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return SWA_ERR_UNSUPPORTED;
+  const int64_t npad = ((int64_t)N + 127) / 128 * 128;
+  const int64_t nspad = S > 0 ? (((int64_t)N + S - 1) / S + 127) / 128 * 128 : 0;
+  const size_t need = (size_t)(2 * (int64_t)B * Hq * npad * 4 + 2 * (int64_t)B * Hkv * nspad * d * 4);
+  if (!aligned16(workspace) || ws_bytes < need) return SWA_ERR_INVALID_ARG;
+  if (!get_encoder()) return SWA_ERR_CUDA;
+  const int64_t nB = B;
+  BwdMaps m;
+  std::memset(&m, 0, sizeof(m));
+  bool ok = encode_rows(&m.q, q, d, N, nB * Hq, d, (int64_t)N * d) &&
+            encode_rows(&m.k, k, d, N, nB * Hkv, d, (int64_t)N * d) &&
+            encode_rows(&m.v, v, d, N, nB * Hkv, d, (int64_t)N * d) &&
+            encode_rows(&m.dO, d_o, d, N, nB * Hq, d, (int64_t)N * d);
+  if (ok && S > 0) {
+    // stride row m is key m*S: a view whose row stride is S rows of K/V
+    const int64_t rows = ((int64_t)N + S - 1) / S;
+    ok = encode_rows(&m.ks, k, d, rows, nB * Hkv, (int64_t)S * d, (int64_t)N * d) &&
+         encode_rows(&m.vs, v, d, rows, nB * Hkv, (int64_t)S * d, (int64_t)N * d);
+  } else {
+    m.ks = m.k;
+    m.vs = m.v;
+  }
+  if (!ok) return SWA_ERR_INVALID_ARG;
+  BwdParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.q = q; p.k = k; p.v = v; p.o = o; p.dO = d_o; p.dq = dq; p.dk = dk; p.dv = dv; p.lse = lse;
+  p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.N = N; p.W = W; p.G = Hq / Hkv;
+  p.nq = (int)(npad / 128);
+  p.npad = (int)npad;
+  p.S = S;
+  p.nspad = (int)nspad;
+  p.lse2 = static_cast<float*>(workspace);
+  p.dd = p.lse2 + (int64_t)B * Hq * npad;
+  p.sdk = S > 0 ? p.dd + (int64_t)B * Hq * npad : nullptr;
+  p.sdv = S > 0 ? p.sdk + (int64_t)B * Hkv * nspad * d : nullptr;
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.err_flag = device_error_ptr();
+  if (p.err_flag == nullptr) return SWA_ERR_CUDA;
+  cudaError_t e = launch_backward(m, p, d, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
+}
 }  // namespace
 }  // namespace swa
 
@@ -322,40 +374,23 @@ size_t swa_attn_bwd_workspace_bytes(int B, int Hq, int N) {
   return (size_t)(2 * (int64_t)B * Hq * npad * (int64_t)sizeof(float));
 }
 
+size_t strided_attn_bwd_workspace_bytes(int B, int Hq, int Hkv, int N, int d, int stride) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || N < 1 || stride < 1 || (d != 64 && d != 128)) return 0;
+  const int64_t nspad = (((int64_t)N + stride - 1) / stride + 127) / 128 * 128;
+  return swa_attn_bwd_workspace_bytes(B, Hq, N) + (size_t)(2 * (int64_t)B * Hkv * nspad * d * (int64_t)sizeof(float));
+}
+
 swa_status_t swa_attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* d_o,
                           const float* lse, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N, int d, int W,
                           float scale, void* workspace, size_t ws_bytes, void* stream) {
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(d_o) || !aligned16(dq) ||
-      !aligned16(dk) || !aligned16(dv) || lse == nullptr || (reinterpret_cast<uintptr_t>(lse) & 3u))
-    return SWA_ERR_INVALID_ARG;
-  if (B < 1 || Hq < 1 || Hkv < 1 || N < 1 || W < 1 || Hq % Hkv != 0) return SWA_ERR_INVALID_ARG;
-  if (!(scale > 0.f) || !std::isfinite(scale)) return SWA_ERR_INVALID_ARG;
-  if ((int64_t)B * Hq > (1 << 30) / 8 || N > (1 << 30)) return SWA_ERR_INVALID_ARG;
-  if (d != 64 && d != 128) return SWA_ERR_UNSUPPORTED;
-  if (!aligned16(workspace) || ws_bytes < swa_attn_bwd_workspace_bytes(B, Hq, N)) return SWA_ERR_INVALID_ARG;
-  if (!get_encoder()) return SWA_ERR_CUDA;
-  const int64_t nB = B;
-  BwdMaps m;
-  std::memset(&m, 0, sizeof(m));
-  const bool ok = encode_rows(&m.q, q, d, N, nB * Hq, d, (int64_t)N * d) &&
-                  encode_rows(&m.k, k, d, N, nB * Hkv, d, (int64_t)N * d) &&
-                  encode_rows(&m.v, v, d, N, nB * Hkv, d, (int64_t)N * d) &&
-                  encode_rows(&m.dO, d_o, d, N, nB * Hq, d, (int64_t)N * d);
-  if (!ok) return SWA_ERR_INVALID_ARG;
-  BwdParams p;
-  std::memset(&p, 0, sizeof(p));
-  p.q = q; p.k = k; p.v = v; p.o = o; p.dO = d_o; p.dq = dq; p.dk = dk; p.dv = dv; p.lse = lse;
-  p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.N = N; p.W = W; p.G = Hq / Hkv;
-  p.nq = (N + 127) / 128;
-  p.npad = p.nq * 128;
-  p.lse2 = static_cast<float*>(workspace);
-  p.dd = p.lse2 + (int64_t)B * Hq * p.npad;
-  p.scale = scale;
-  p.scale_log2 = scale * 1.4426950408889634f;
-  p.err_flag = device_error_ptr();
-  if (p.err_flag == nullptr) return SWA_ERR_CUDA;
-  cudaError_t e = launch_backward(m, p, d, static_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
+  return run_bwd(q, k, v, o, d_o, lse, dq, dk, dv, B, Hq, Hkv, N, d, W, 0, scale, workspace, ws_bytes, stream);
+}
+
+swa_status_t strided_attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* d_o,
+                              const float* lse, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N, int d,
+                              int W, int stride, float scale, void* workspace, size_t ws_bytes, void* stream) {
+  if (stride < 1) return SWA_ERR_INVALID_ARG;
+  return run_bwd(q, k, v, o, d_o, lse, dq, dk, dv, B, Hq, Hkv, N, d, W, stride, scale, workspace, ws_bytes, stream);
 }
 
 int64_t swa_schedule(int kind, int N, int W, int stride, int Bq, int Bk, int32_t* qtile_offsets, int32_t* tiles,

@@ -84,6 +84,13 @@ __device__ __forceinline__ bool bwd_attended(int i, int key, int W, int N) {
   return key <= i && i - key < W && i < N && key < N;
 }
 
+// Row i attends the compacted stride key m (key m*S) as an extra key: the key
+// lies below the row's window (m*S < i - W + 1), both below N.
+__device__ __forceinline__ bool bwd_stride_attended(int i, int m, int W, int S, int N) {
+  const int64_t key = (int64_t)m * S;
+  return key < (int64_t)i - W + 1 && i < N && key < N;
+}
+
 // D_i = dO_i . O_i and L_i * log2(e), rows past N padded with zeros.
 template <int D>
 __global__ void __launch_bounds__(128) bwd_prep_kernel(const BwdParams p) {
@@ -111,12 +118,29 @@ __global__ void __launch_bounds__(128) bwd_prep_kernel(const BwdParams p) {
   }
   p.dd[r] = d;
   p.lse2[r] = l2;
+  // the stride pass adds its partials into zeroed memory
+  if (p.S > 0) {
+    const int64_t nz = (int64_t)p.B * p.Hkv * p.nspad * D;
+    for (int64_t z = r; z < nz; z += total) {
+      p.sdk[z] = 0.f;
+      p.sdv[z] = 0.f;
+    }
+  }
 }
 
-template <int D>
+// MODE 0: 128 window keys of the tile. MODE 1: the same, plus the stride
+// pass's fp32 partials added to the stride keys before rounding (local +
+// strided mask). MODE 2 (stride pass): the CTA owns 128 compacted stride
+// keys (m*S for m in ct*128 .. ct*128+127) and one chunk of the later query
+// tiles whose rows have them below their window; it adds its fp32 partial
+// dK / dV into the workspace (several chunks per stride tile).
+constexpr int kStrideChunk = 8;  // query tiles per stride-pass CTA
+
+template <int D, int MODE>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                    const __grid_constant__ CUtensorMap tm_ks, const __grid_constant__ CUtensorMap tm_vs,
                     const __grid_constant__ BwdParams p) {
   using C = BwdCfg<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -128,16 +152,29 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(words + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  const int kt = blockIdx.x;
   const int b = blockIdx.y / p.Hkv, hkv = blockIdx.y % p.Hkv;
   // query tiles that see keys kt*128 .. kt*128+127: from the diagonal up to
   // the last row whose window still reaches the tile's last key
-  const int qt_lo = kt;
+  constexpr bool STRIDE = MODE == 2;
   const int Wc = imin(p.W, p.N);
-  const int reach = kt * kBT + kBT - 1 + Wc - 1;  // last query row that sees the tile's last key
-  const int qt_hi = imin(p.nq - 1, reach / kBT);
+  int qt_lo, qt_hi;
+  int kt = blockIdx.x;
+  if (STRIDE) {
+    // row i has stride key m below its window iff m * S < i - W + 1
+    const int nchunk = (p.nq + kStrideChunk - 1) / kStrideChunk;
+    kt = blockIdx.x / nchunk;
+    const int chunk = blockIdx.x % nchunk;
+    const int64_t first = (int64_t)kt * kBT * p.S + Wc;  // first row that sees m = kt * 128
+    const int q0 = (int)(first < p.N ? first / kBT : p.nq);
+    qt_lo = q0 + chunk * kStrideChunk;
+    qt_hi = imin(p.nq - 1, qt_lo + kStrideChunk - 1);  // empty when past the last tile
+  } else {
+    qt_lo = kt;
+    const int reach = kt * kBT + kBT - 1 + Wc - 1;  // last query row that sees the tile's last key
+    qt_hi = imin(p.nq - 1, reach / kBT);
+  }
   const int nqt = qt_hi - qt_lo + 1;
-  const int nsteps = p.G * nqt;
+  const int nsteps = nqt > 0 ? p.G * nqt : 0;
 
   if (threadIdx.x == 0) {
     mbar_init(bar(BwdBar::kFixed), 1);
@@ -167,8 +204,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const int zkv = b * p.Hkv + hkv;
       mbar_arrive_expect_tx(bar(BwdBar::kFixed), 2 * C::kTile);
       for (int bx = 0; bx < D / 64; ++bx) {
-        tma_load_3d(sbase + C::kOffA + bx * 16384, &tm_k, bar(BwdBar::kFixed), bx * 64, kt * kBT, zkv);
-        tma_load_3d(sbase + C::kOffB + bx * 16384, &tm_v, bar(BwdBar::kFixed), bx * 64, kt * kBT, zkv);
+        tma_load_3d(sbase + C::kOffA + bx * 16384, STRIDE ? &tm_ks : &tm_k, bar(BwdBar::kFixed), bx * 64, kt * kBT,
+                    zkv);
+        tma_load_3d(sbase + C::kOffB + bx * 16384, STRIDE ? &tm_vs : &tm_v, bar(BwdBar::kFixed), bx * 64, kt * kBT,
+                    zkv);
       }
       int issued[C::kStages] = {0, 0};
       for (int s = 0; s < nsteps; ++s) {
@@ -259,7 +298,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     // --------------------------------------------------- elementwise ---
     const int qw = warp & 3;             // TMEM lane quarter
     const int kr = qw * 32 + lane;       // key row within the tile
-    const int key = kt * kBT + kr;
+    const int key = kt * kBT + kr;       // (STRIDE: the compacted index m; the key is m * S)
     const uint32_t lane_addr = static_cast<uint32_t>(qw * 32) << 16;
     const float sl2 = p.scale_log2;
     bool ok = true;
@@ -293,7 +332,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         for (int c = 0; c < 64; c += 2) {
           const int c0 = 64 * h + c;
           const int i0 = qt * kBT + c0;
-          const bool a0 = bwd_attended(i0, key, p.W, p.N), a1 = bwd_attended(i0 + 1, key, p.W, p.N);
+          const bool a0 = STRIDE ? bwd_stride_attended(i0, key, p.W, p.S, p.N) : bwd_attended(i0, key, p.W, p.N);
+          const bool a1 = STRIDE ? bwd_stride_attended(i0 + 1, key, p.W, p.S, p.N)
+                                 : bwd_attended(i0 + 1, key, p.W, p.N);
           const float p0 = a0 ? ex2_approx(fmaf(sv[c], sl2, -lse2[c0])) : 0.f;
           const float p1 = a1 ? ex2_approx(fmaf(sv[c + 1], sl2, -lse2[c0 + 1])) : 0.f;
           pk[c >> 1] = pack_bf16(p0, p1);
@@ -314,16 +355,43 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         ok = false;
       }
     }
-    if (ok) {
+    if (ok && STRIDE) {
+      // this chunk's fp32 partials of the stride keys, added to the others'
+      if (nsteps > 0) {
+        tc_fence_after();
+        const int64_t row = ((int64_t)(b * p.Hkv + hkv) * p.nspad + key) * D;
+#pragma unroll 1
+        for (int c = 0; c < D; c += 32) {
+          float a[32], g[32];
+          tmem_ld32(tmem + lane_addr + C::kColAcc + c, a);
+          tmem_ld32(tmem + lane_addr + C::kColAcc + D + c, g);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            atomicAdd(p.sdv + row + c + e, a[e]);
+            atomicAdd(p.sdk + row + c + e, g[e]);
+          }
+        }
+      }
+    } else if (ok) {
       tc_fence_after();
       const int64_t row = ((int64_t)(b * p.Hkv + hkv) * p.N + key) * D;
       __nv_bfloat16* dv = reinterpret_cast<__nv_bfloat16*>(p.dv) + row;
       __nv_bfloat16* dkp = reinterpret_cast<__nv_bfloat16*>(p.dk) + row;
+      // a stride key also gets the stride pass's partials before the one rounding
+      const bool add = MODE == 1 && key < p.N && key % p.S == 0;
+      const int64_t srow = ((int64_t)(b * p.Hkv + hkv) * p.nspad + (add ? key / p.S : 0)) * D;
 #pragma unroll 1
       for (int c = 0; c < D; c += 32) {
         float a[32], g[32];
         tmem_ld32(tmem + lane_addr + C::kColAcc + c, a);
         tmem_ld32(tmem + lane_addr + C::kColAcc + D + c, g);
+        if (add) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            a[e] += p.sdv[srow + c + e];
+            g[e] += p.sdk[srow + c + e];
+          }
+        }
         if (key < p.N) {
 #pragma unroll
           for (int e = 0; e < 32; e += 8) {
@@ -348,10 +416,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   }
 }
 
-template <int D>
+// SM: the local + strided mask (stride tiles before the window tiles).
+template <int D, bool SM>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                  const __grid_constant__ CUtensorMap tm_ks, const __grid_constant__ CUtensorMap tm_vs,
                   const __grid_constant__ BwdParams p) {
   using C = BwdCfg<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -366,11 +436,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int qt = blockIdx.x;
   const int b = blockIdx.y / p.Hq, hq = blockIdx.y % p.Hq;
   const int hkv = hq / p.G;
-  // key tiles of the row block: from the tile holding the first row's
-  // window start to the diagonal tile
+  // key tiles of the row block: the compacted stride tiles with a key below
+  // the last row's window (strided mask), then the window tiles from the one
+  // holding the first row's window start to the diagonal tile
   const int Wc = imin(p.W, p.N);
   const int kt_lo = imax(0, qt * kBT - Wc + 1) / kBT;
-  const int nsteps = qt - kt_lo + 1;
+  int nst = 0;
+  if (SM) {
+    const int r1 = imin(p.N - 1, qt * kBT + kBT - 1);
+    nst = (stride_rows_below(imax(0, r1 - Wc + 1), p.S) + kBT - 1) / kBT;
+  }
+  const int nsteps = nst + (qt - kt_lo + 1);
 
   if (threadIdx.x == 0) {
     mbar_init(bar(BwdBar::kFixed), 1);
@@ -410,12 +486,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           bwd_timeout(abort_flag, p.err_flag);
           break;
         }
-        const int kt = kt_lo + s;
+        const bool strided = s < nst;
+        const int row = (strided ? s : kt_lo + (s - nst)) * kBT;
         const uint32_t base = sbase + C::kOffStages + st * C::kStage;
         mbar_arrive_expect_tx(bar(BwdBar::kFull + st), 2 * C::kTile);
         for (int bx = 0; bx < D / 64; ++bx) {
-          tma_load_3d(base + bx * 16384, &tm_k, bar(BwdBar::kFull + st), bx * 64, kt * kBT, zkv);
-          tma_load_3d(base + C::kTile + bx * 16384, &tm_v, bar(BwdBar::kFull + st), bx * 64, kt * kBT, zkv);
+          tma_load_3d(base + bx * 16384, strided ? &tm_ks : &tm_k, bar(BwdBar::kFull + st), bx * 64, row, zkv);
+          tma_load_3d(base + C::kTile + bx * 16384, strided ? &tm_vs : &tm_v, bar(BwdBar::kFull + st), bx * 64, row,
+                      zkv);
         }
         issued[st] = use + 1;
       }
@@ -489,7 +567,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const float lse2 = p.lse2[rt], dd = p.dd[rt];
     bool ok = true;
     for (int s = 0; s < nsteps; ++s) {
-      const int kt = kt_lo + s;
+      const bool strided = SM && s < nst;
+      const int kt = strided ? s : kt_lo + (s - nst);  // strided: compacted stride rows kt*128 ..
       const bool got = mbar_wait(bar(BwdBar::kS), s & 1, abort_flag);
       if (!__all_sync(0xffffffffu, got)) {
         if (lane == 0) bwd_timeout(abort_flag, p.err_flag);
@@ -503,14 +582,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         uint32_t pk[32];
         tmem_ld64(tmem + lane_addr + C::kColS + 64 * h, sv);
         tmem_ld64(tmem + lane_addr + C::kColDP + 64 * h, dp);
+        auto body = [&](auto attended) {
 #pragma unroll
-        for (int c = 0; c < 64; c += 2) {
-          const int key = kt * kBT + 64 * h + c;
-          const bool a0 = bwd_attended(i, key, p.W, p.N), a1 = bwd_attended(i, key + 1, p.W, p.N);
-          const float p0 = a0 ? ex2_approx(fmaf(sv[c], sl2, -lse2)) : 0.f;
-          const float p1 = a1 ? ex2_approx(fmaf(sv[c + 1], sl2, -lse2)) : 0.f;
-          pk[c >> 1] = pack_bf16(p0 * (dp[c] - dd), p1 * (dp[c + 1] - dd));
-        }
+          for (int c = 0; c < 64; c += 2) {
+            const int key = kt * kBT + 64 * h + c;  // strided: the compacted index m
+            const bool a0 = attended(key), a1 = attended(key + 1);
+            const float p0 = a0 ? ex2_approx(fmaf(sv[c], sl2, -lse2)) : 0.f;
+            const float p1 = a1 ? ex2_approx(fmaf(sv[c + 1], sl2, -lse2)) : 0.f;
+            pk[c >> 1] = pack_bf16(p0 * (dp[c] - dd), p1 * (dp[c + 1] - dd));
+          }
+        };
+        if (strided)
+          body([&](int m) { return bwd_stride_attended(i, m, p.W, p.S, p.N); });
+        else
+          body([&](int key) { return bwd_attended(i, key, p.W, p.N); });
         // dS over S as bf16 pairs: keys 64h .. 64h+63 in columns 32h .. 32h+31
         tmem_st32_u(tmem + lane_addr + C::kColS + 32 * h, pk);
       }
@@ -557,10 +642,12 @@ cudaError_t launch_bwd_d(const BwdMaps& m, const BwdParams& p, cudaStream_t stre
   using C = BwdCfg<D>;
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         C::kSmemBytes);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    const cudaFuncAttribute a = cudaFuncAttributeMaxDynamicSharedMemorySize;
+    cudaError_t e = cudaFuncSetAttribute(bwd_dkdv_kernel<D, 0>, a, C::kSmemBytes);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(bwd_dkdv_kernel<D, 1>, a, C::kSmemBytes);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(bwd_dkdv_kernel<D, 2>, a, C::kSmemBytes);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(bwd_dq_kernel<D, false>, a, C::kSmemBytes);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(bwd_dq_kernel<D, true>, a, C::kSmemBytes);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
@@ -569,10 +656,23 @@ cudaError_t launch_bwd_d(const BwdMaps& m, const BwdParams& p, cudaStream_t stre
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int nk = p.nq;  // key tiles of 128 (same count as query tiles)
-  bwd_dkdv_kernel<D><<<dim3(nk, p.B * p.Hkv), kBwdThreads, C::kSmemBytes, stream>>>(m.q, m.k, m.v, m.dO, p);
+  const dim3 gk(nk, p.B * p.Hkv), gq(p.nq, p.B * p.Hq);
+  if (p.S > 0) {  // stride keys first: their partials feed the window pass
+    const int nchunk = (p.nq + kStrideChunk - 1) / kStrideChunk;
+    bwd_dkdv_kernel<D, 2><<<dim3(p.nspad / kBT * nchunk, p.B * p.Hkv), kBwdThreads, C::kSmemBytes, stream>>>(
+        m.q, m.k, m.v, m.dO, m.ks, m.vs, p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    bwd_dkdv_kernel<D, 1><<<gk, kBwdThreads, C::kSmemBytes, stream>>>(m.q, m.k, m.v, m.dO, m.ks, m.vs, p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    bwd_dq_kernel<D, true><<<gq, kBwdThreads, C::kSmemBytes, stream>>>(m.q, m.k, m.v, m.dO, m.ks, m.vs, p);
+    return cudaGetLastError();
+  }
+  bwd_dkdv_kernel<D, 0><<<gk, kBwdThreads, C::kSmemBytes, stream>>>(m.q, m.k, m.v, m.dO, m.ks, m.vs, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  bwd_dq_kernel<D><<<dim3(p.nq, p.B * p.Hq), kBwdThreads, C::kSmemBytes, stream>>>(m.q, m.k, m.v, m.dO, p);
+  bwd_dq_kernel<D, false><<<gq, kBwdThreads, C::kSmemBytes, stream>>>(m.q, m.k, m.v, m.dO, m.ks, m.vs, p);
   return cudaGetLastError();
 }
 

@@ -45,12 +45,14 @@ struct BwdParams {
   void *dq, *dk, *dv;
   const float* lse;
   float *lse2, *dd;
+  float *sdk, *sdv;  // strided mask: fp32 partial dK, dV of the stride keys [B*Hkv, nspad, d]
   int B, Hq, Hkv, N, W, G, nq, npad;
+  int S, nspad;      // stride (0: window mask only), compacted stride rows padded to tiles
   float scale, scale_log2;
   int* err_flag;
 };
 struct BwdMaps {
-  CUtensorMap q, k, v, dO;
+  CUtensorMap q, k, v, dO, ks, vs;  // ks, vs: stride row m is key m*S (or K, V when S = 0)
 };
 cudaError_t launch_backward(const BwdMaps& m, const BwdParams& p, int d, cudaStream_t stream);
 

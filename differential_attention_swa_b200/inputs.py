@@ -99,6 +99,8 @@ WORKLOADS = {
     "gemma_swa_prefill": Workload("gemma_swa_prefill", "swa", 1, 16, 8, 131072, 128, 1024),
     # the backward of the Mistral-style window attention (gradients of Q, K, V)
     "mistral_swa_backward": Workload("mistral_swa_backward", "swa_bwd", 2, 32, 8, 8192, 128, 4096),
+    # the backward of the local + strided mask
+    "local_strided_backward": Workload("local_strided_backward", "swa_bwd", 1, 16, 16, 16384, 64, 128, S=128),
     # window + global tokens with a Longformer-like shape (16 heads of 64,
     # a 512-token window, 64 global tokens at the start); S carries g
     "longformer_global_prefill": Workload("longformer_global_prefill", "global", 1, 16, 16, 16384, 64, 512, S=64),

@@ -261,6 +261,21 @@ swa_status_t swa_attn_bwd(const void* q, const void* k, const void* v, const voi
 /* Scratch bytes swa_attn_bwd needs (0 on bad sizes). */
 size_t swa_attn_bwd_workspace_bytes(int B, int Hq, int N);
 
+/* Backward of strided_attn_fwd (window OR keys j % stride == 0, j <= i):
+ * the same chain rule as swa_attn_bwd over the union mask. Stride keys below
+ * a row's window are gathered through a strided view of K and V (no copies);
+ * their dK/dV contributions from every later query row are accumulated in
+ * fp32 in the workspace and added to the window pass's before rounding.
+ *   Arguments as swa_attn_bwd, plus stride >= 1; lse from strided_attn_fwd;
+ *   workspace of at least strided_attn_bwd_workspace_bytes(...) bytes. */
+swa_status_t strided_attn_bwd(const void* q, const void* k, const void* v, const void* o,
+                              const void* d_o, const float* lse, void* dq, void* dk, void* dv,
+                              int B, int Hq, int Hkv, int N, int d, int W, int stride,
+                              float scale, void* workspace, size_t ws_bytes, void* stream);
+
+/* Scratch bytes strided_attn_bwd needs (0 on bad sizes). */
+size_t strided_attn_bwd_workspace_bytes(int B, int Hq, int Hkv, int N, int d, int stride);
+
 /* Prefill with debug outputs. kind 0 = sliding window (stride ignored),
  * kind 1 = local + strided, kind 3 = window + global tokens (stride carries
  * n_global). Same arithmetic as swa_attn_fwd / strided_attn_fwd /

@@ -33,12 +33,15 @@ def compare_grad(got, want, what):
     return diff.max() / scale
 
 
-def run(B, Hq, Hkv, N, d, W, seed):
+def run(B, Hq, Hkv, N, d, W, seed, S=0):
     q, k, v = attn_inputs(B, Hq, Hkv, N, d, seed=seed)
     d_o = randn_bf16((B, Hq, N, d), seed + 10)
     qd, kd, vd, dod = (t.cuda() for t in (q, k, v, d_o))
-    o, lse = swa.swa_attn_fwd(qd, kd, vd, W, return_lse=True)
-    dq, dk, dv = swa.swa_attn_bwd(qd, kd, vd, o, dod, lse, W)
+    if S:
+        o, lse = swa.strided_attn_fwd(qd, kd, vd, W, S, return_lse=True)
+    else:
+        o, lse = swa.swa_attn_fwd(qd, kd, vd, W, return_lse=True)
+    dq, dk, dv = swa.swa_attn_bwd(qd, kd, vd, o, dod, lse, W, stride=S)
     torch.cuda.synchronize()
     assert swa.last_device_error() == swa.OK
     return (q, k, v, d_o), (dq, dk, dv)
@@ -72,3 +75,29 @@ def test_backward_sampled_rows_at_size(orc):
     compare_grad(dq.reshape(-1, d)[torch.from_numpy(qr).cuda()], rq, "dq rows")
     compare_grad(dk.reshape(-1, d)[torch.from_numpy(kr).cuda()], rk, "dk rows")
     compare_grad(dv.reshape(-1, d)[torch.from_numpy(kr).cuda()], rv, "dv rows")
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,N,d,W,S", [
+    (1, 2, 2, 300, 64, 17, 5),      # N not a multiple of S, several stride tiles per row block
+    (1, 4, 2, 1000, 128, 64, 7),    # group 2, stride keys spread over the sequence
+    (1, 2, 2, 256, 64, 3, 1),       # stride 1: every key (full causal)
+    (1, 2, 2, 333, 64, 20, 400),    # stride beyond N: window + key 0
+    (1, 3, 1, 700, 64, 1, 3),       # window 1 + stride, group 3
+    (1, 2, 2, 16384, 64, 128, 128), # the local+strided workload's mask at one batch and two heads
+])
+def test_strided_backward_vs_oracle(orc, B, Hq, Hkv, N, d, W, S):
+    (q, k, v, d_o), (dq, dk, dv) = run(B, Hq, Hkv, N, d, W, seed=N + S, S=S)
+    if N <= 1024:
+        rq, rk, rv = orc.attention_bwd("strided", q, k, v, d_o, W=W, S=S, scale=1 / math.sqrt(d))
+        compare_grad(dq, rq, "dq")
+        compare_grad(dk, rk, "dk")
+        compare_grad(dv, rv, "dv")
+    else:  # sampled rows, stride keys among them
+        rng = np.random.default_rng(5)
+        qr = np.unique(np.concatenate([rng.integers(0, B * Hq * N, 30), [0, N - 1, 128 * 5 + 3]]))
+        kr = np.unique(np.concatenate([rng.integers(0, B * Hkv * N, 4), [0, S, 5 * S, N - 1]]))
+        rq, rk, rv = orc.attention_bwd("strided", q, k, v, d_o, W=W, S=S, scale=1 / math.sqrt(d), dq_rows=qr,
+                                       dkv_rows=kr)
+        compare_grad(dq.reshape(-1, d)[torch.from_numpy(qr).cuda()], rq, "dq rows")
+        compare_grad(dk.reshape(-1, d)[torch.from_numpy(kr).cuda()], rk, "dk rows")
+        compare_grad(dv.reshape(-1, d)[torch.from_numpy(kr).cuda()], rv, "dv rows")
