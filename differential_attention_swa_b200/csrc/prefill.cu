@@ -18,16 +18,23 @@
 // Warp roles (384 threads):
 //   warp 0      TMA producer: Q once, then K and V tiles through a ring of
 //               shared-memory slots.
-//   warp 1      TMEM owner and MMA issuer (one thread). Per key tile and
-//               sub: O_t += P_t(prev) V(prev) (A operand read from TMEM),
-//               then S_t = Q_t K^T into the same TMEM columns that held P_t;
-//               the tensor core runs MMAs in issue order, so P is read
-//               before S overwrites it, and the commit that signals S_t also
-//               covers the PV before it.
+//   warp 1      TMEM owner and MMA issuer. A sub's 128 score columns are
+//               two 64-key buffers: half h of every key tile goes to buffer
+//               h. Per key tile and half, once both subs' P_t,h are written,
+//               one elected lane issues for each sub O_t += P_t,h(prev)
+//               V_h(prev) (A operand read from TMEM), then S_t,h = Q_t K_h^T
+//               into the buffer that held P_t,h, and the commits. The tensor
+//               core runs MMAs in issue order, so P is read before S
+//               overwrites it; while the softmax works on one half, the
+//               tensor core computes the other. The whole warp keeps the
+//               bookkeeping, so the MMA operands are warp-uniform values,
+//               and one issue block per half-step keeps the tensor core's
+//               queue fed.
 //   warps 4-7   softmax of sub 0, warps 8-11 softmax of sub 1: one thread
 //               per query row (TMEM lane), fp32 online softmax in the log2
-//               domain, P as bf16 back into TMEM over the consumed scores,
-//               lazy rescaling of O, then the epilogue O / l -> bf16.
+//               domain over 64-key halves, P as bf16 back into TMEM over the
+//               consumed scores, lazy rescaling of O, then the epilogue
+//               O / l -> bf16.
 // Every wait is bounded; on a timeout the CTA records SWA_ERR_TIMEOUT,
 // drains what it has in flight, frees TMEM and returns.
 #include <cuda.h>
@@ -35,6 +42,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <type_traits>
 
 #include "internal.h"
 #include "ptx.cuh"
@@ -43,7 +51,8 @@
 namespace swa {
 
 constexpr int BM = 128;  // query rows per sub (TMEM lanes)
-constexpr int BN = 128;  // keys per tile (S columns)
+constexpr int BN = 128;  // keys per tile (S columns of a sub)
+constexpr int BH = 64;   // keys per score buffer (half a tile)
 constexpr int kThreads = 384;
 // Lazy rescale threshold (log2 units): O and l keep a stale row max until a
 // new score exceeds it by more than this, so P stays below 2^8.
@@ -71,23 +80,26 @@ struct PrefillCfg {
   static constexpr int kOCol0 = 256;
   static constexpr int kOCol1 = 256 + DV;
   static_assert(256 + 2 * DV <= kTmemCols, "TMEM budget");
+  static_assert(DQK == 64 || DQK == 128, "score bursts cover K = 64 or 128");
 };
 
 // Barrier block layout (8-byte mbarriers, then a few words).
 struct BarLayout {
   static constexpr int kQ = 0;
-  static constexpr int kQEmpty = 25;    // every S MMA of the unit done: Q may be replaced
-  static constexpr int kOFree = 26;     // + sub: epilogue done reading O_t
   static constexpr int kFull = 1;       // + slot
   static constexpr int kEmpty = 9;      // + slot
-  static constexpr int kS = 17;         // + sub
-  static constexpr int kP = 19;         // + sub
-  static constexpr int kO = 21;         // + sub
-  static constexpr int kX = 23;         // differential hand-off of 1/l2
-  static constexpr int kFinal = 24;     // MMA drain on abort
-  static constexpr int kCount = 28;
-  static constexpr int kWordsOff = 256; // bytes: tmem base, abort flag
+  static constexpr int kS = 17;         // + 2 * sub + half: S_t,h written
+  static constexpr int kP = 21;         // + 2 * sub + half: P_t,h written
+  static constexpr int kO = 25;         // + sub: the unit's last PV done
+  static constexpr int kX = 27;         // differential hand-off of 1/l2
+  static constexpr int kFinal = 28;     // MMA drain on abort
+  static constexpr int kQEmpty = 29;    // every S MMA of the unit done: Q may be replaced
+  static constexpr int kOFree = 30;     // + sub: epilogue done reading O_t
+  static constexpr int kLast = 32;      // + sub: PV of half 0 done where no S of half 0 follows
+  static constexpr int kCount = 34;
+  static constexpr int kWordsOff = 384; // bytes: tmem base, abort flag
   static constexpr int kF2Off = 512;    // bytes: 128 floats
+  static_assert(kCount * 8 <= kWordsOff, "barrier block");
 };
 
 struct Unit {
@@ -219,10 +231,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(BarLayout::kEmpty + s), 1);
     }
     for (int t = 0; t < 2; ++t) {
-      mbar_init(bar(BarLayout::kS + t), 1);
-      mbar_init(bar(BarLayout::kP + t), 128);
+      for (int h = 0; h < 2; ++h) {
+        mbar_init(bar(BarLayout::kS + 2 * t + h), 1);
+        mbar_init(bar(BarLayout::kP + 2 * t + h), 128);
+      }
       mbar_init(bar(BarLayout::kO + t), 1);
       mbar_init(bar(BarLayout::kOFree + t), 128);
+      mbar_init(bar(BarLayout::kLast + t), 1);
     }
     mbar_init(bar(BarLayout::kX), 128);
     mbar_init(bar(BarLayout::kFinal), 1);
@@ -328,137 +343,167 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ----------------------------------------------------------- MMA ---
-    if (lane == 0) {
-      const uint32_t idesc_s = idesc_bf16_f32(BM, BN, false);
+    // The whole warp runs the bookkeeping, so every operand is warp-uniform;
+    // one elected lane issues each MMA burst and commit. Sub and half indices
+    // are compile-time constants (generic lambdas over integral_constant),
+    // so the issuer's state stays in registers.
+    {
+      // all lanes wait; the result is made warp-uniform
+      auto wait = [&](uint32_t b, uint32_t parity) -> bool {
+        return __all_sync(0xffffffffu, mbar_wait(b, parity, abort_flag));
+      };
+      auto commit = [&](uint32_t b) {
+        if (elect_one()) umma_commit(b);
+        __syncwarp();
+      };
+      using I0 = std::integral_constant<int, 0>;
+      using I1 = std::integral_constant<int, 1>;
+      const uint32_t idesc_s = idesc_bf16_f32(BM, BH, false);
       const uint32_t idesc_pv = idesc_bf16_f32(BM, DV, true);
-      // descriptors of slice kk differ from slice 0 only in the start
-      // address field (bits 0-13, in 16-byte units)
-      const uint64_t q_desc0[2] = {sw128_desc(sbase + C::kOffQ, 16, 1024),
-                                   sw128_desc(sbase + C::kOffQ + C::kQBytes, 16, 1024)};
+      const uint64_t q_desc_0 = sw128_desc(sbase + C::kOffQ, 16, 1024);
+      const uint64_t q_desc_1 = sw128_desc(sbase + C::kOffQ + C::kQBytes, 16, 1024);
+      struct SubMma {
+        int npv0, npv1;  // PV products of half 0 / 1, across units (P phases)
+        int nunit;       // units in which the sub took part (O-free phases)
+        int ntot;        // key tiles of the sub in this unit
+        int kcount;      // S tiles issued in this unit
+        int pv_done;     // key tiles of this unit whose PVs (both halves) are issued
+        bool pending;    // the previous item's PVs are still to issue
+        int64_t dbg_row;
+      };
+      SubMma sm0 = {0, 0, 0, 0, 0, 0, false, -1}, sm1 = {0, 0, 0, 0, 0, 0, false, -1};
       int L = 0;
-      int ksteps[2] = {0, 0};  // S tiles issued per sub, across units (barrier phases)
-      int nunit[2] = {0, 0};   // units in which the sub took part (O / O-free phases)
-      int nq = 0;              // units started (Q phases)
+      int nq = 0;  // units started (Q phases)
       bool ok = true;
       for (int rnd = 0; rnd * P < nunits && ok; ++rnd) {
         const int ui = unit_of(rnd);
         if (ui >= nunits) continue;
         const Unit un = decode_unit(p, ui);
         const Items it = unit_items<GEN>(p, un);
-        const int ntot[2] = {un.valid[0] ? qtile_nkeys(it.k[0]) : 0, un.valid[1] ? qtile_nkeys(it.k[1]) : 0};
-        int kcount[2] = {0, 0};   // S tiles of this unit per sub
-        int pv_done[2] = {0, 0};  // PV products of this unit per sub
-        bool pending[2] = {false, false};
-        int64_t dbg_row[2] = {-1, -1};
-        for (int t = 0; t < 2; ++t)
-          if (un.valid[t] && p.dbg_tiles && !(DIFF && t == 1))
-            dbg_row[t] = (int64_t)(un.b * p.Hq + un.hq[t]) * p.nq + un.qt[t];
-        if (!mbar_wait(bar(BarLayout::kQ), nq & 1, abort_flag)) {
-          record_timeout(abort_flag, p.err_flag);
+        sm0.ntot = un.valid[0] ? qtile_nkeys(it.k[0]) : 0;
+        sm1.ntot = un.valid[1] ? qtile_nkeys(it.k[1]) : 0;
+        sm0.kcount = sm1.kcount = 0;
+        sm0.pv_done = sm1.pv_done = 0;
+        sm0.pending = sm1.pending = false;
+        sm0.dbg_row = (un.valid[0] && p.dbg_tiles) ? (int64_t)(un.b * p.Hq + un.hq[0]) * p.nq + un.qt[0] : -1;
+        sm1.dbg_row = (un.valid[1] && p.dbg_tiles && !DIFF) ? (int64_t)(un.b * p.Hq + un.hq[1]) * p.nq + un.qt[1] : -1;
+        if (!wait(bar(BarLayout::kQ), nq & 1)) {
+          if (lane == 0) record_timeout(abort_flag, p.err_flag);
           ok = false;
           break;
         }
         ++nq;
         tc_fence_after();
         int prev_vslot = -1, prev_vuse = 0;
-        // O_t += P_t V(prev): P_t is the bf16 tile softmax t wrote over the
-        // first 64 columns of S_t (two keys per column)
-        auto issue_pv = [&](int t) -> bool {
-          if (pv_done[t] == 0 && nunit[t] > 0) {
-            // the first PV overwrites O_t: the previous unit's epilogue must be done with it
-            if (!mbar_wait(bar(BarLayout::kOFree + t), (nunit[t] - 1) & 1, abort_flag)) return false;
-            tc_fence_after();
-          }
-          const uint64_t b0 = sw128_desc(sbase + C::kOffSlots + prev_vslot * C::kSlot, 16384, 1024);
-          const uint32_t a0 = tmem + t * BN;
-          const uint32_t dcol = tmem + (t == 0 ? C::kOCol0 : C::kOCol1);
-          const bool first = (pv_done[t] == 0);
-#pragma unroll
-          for (int kk = 0; kk < BN / 16; ++kk)
-            umma_bf16_ts(dcol, a0 + kk * 8, b0 + (uint64_t)(kk * 2048 >> 4), idesc_pv, (first && kk == 0) ? 0u : 1u);
-          ++pv_done[t];
-          if (pv_done[t] == ntot[t]) umma_commit(bar(BarLayout::kO + t));
-          pending[t] = false;
-          return true;
-        };
-        auto wait_prev_v = [&]() -> bool {
-          if (!mbar_wait(bar(BarLayout::kFull + prev_vslot), prev_vuse & 1, abort_flag)) return false;
+        // One half-step of both subs: wait for both P_t,h, then one elected
+        // lane issues, per sub, O_t += P_t,h V_h(prev) (P read from score
+        // buffer h) and S_t,h = Q_t K_h^T into the same buffer, with their
+        // commits. The tensor core runs MMAs in issue order, so P is read
+        // before S overwrites it. `drain` issues the last item's PVs only.
+        auto half_step = [&](auto hc, bool in0, bool in1, int kslot, int u, bool drain) -> bool {
+          constexpr int h = decltype(hc)::value;
+          int& npv0 = h ? sm0.npv1 : sm0.npv0;
+          int& npv1 = h ? sm1.npv1 : sm1.npv0;
+          if (sm0.pending && !wait(bar(BarLayout::kP + 0 + h), npv0 & 1)) return false;
+          if (sm1.pending && !wait(bar(BarLayout::kP + 2 + h), npv1 & 1)) return false;
+          // the first PV of a unit overwrites O_t: the previous unit's epilogue must be done with it
+          const bool f0 = (h == 0 && sm0.pv_done == 0), f1 = (h == 0 && sm1.pv_done == 0);
+          if (sm0.pending && f0 && sm0.nunit > 0 && !wait(bar(BarLayout::kOFree + 0), (sm0.nunit - 1) & 1))
+            return false;
+          if (sm1.pending && f1 && sm1.nunit > 0 && !wait(bar(BarLayout::kOFree + 1), (sm1.nunit - 1) & 1))
+            return false;
           tc_fence_after();
+          const uint64_t vdesc =
+              sw128_desc(sbase + C::kOffSlots + prev_vslot * C::kSlot + h * (BH / 16) * 2048, 16384, 1024);
+          const uint32_t kbase = sbase + C::kOffSlots + kslot * C::kSlot + h * BH * 128;
+          const uint64_t kdesc0 = sw128_desc(kbase, 16, 1024);
+          const uint64_t kdesc1 = sw128_desc(kbase + (DIFF ? BN * DQK * 2 : 0), 16, 1024);
+          const bool o_done0 = h == 1 && sm0.pending && sm0.pv_done + 1 == sm0.ntot;
+          const bool o_done1 = h == 1 && sm1.pending && sm1.pv_done + 1 == sm1.ntot;
+          if (elect_one()) {
+            if (sm0.pending) {
+              umma_ts_k4(tmem + C::kOCol0, tmem + h * BH, vdesc, idesc_pv, f0 ? 0u : 1u);
+              if (h == 0 && !in0) umma_commit(bar(BarLayout::kLast + 0));  // no S of half 0 follows
+              if (o_done0) umma_commit(bar(BarLayout::kO + 0));
+            }
+            if (in0) {
+              if (DQK == 128) umma_ss_k8(tmem + h * BH, q_desc_0, kdesc0, idesc_s, 0u);
+              else umma_ss_k4(tmem + h * BH, q_desc_0, kdesc0, idesc_s, 0u);
+              umma_commit(bar(BarLayout::kS + 0 + h));
+            }
+            if (sm1.pending) {
+              umma_ts_k4(tmem + C::kOCol1, tmem + BN + h * BH, vdesc, idesc_pv, f1 ? 0u : 1u);
+              if (h == 0 && !in1) umma_commit(bar(BarLayout::kLast + 1));
+              if (o_done1) umma_commit(bar(BarLayout::kO + 1));
+            }
+            if (in1) {
+              if (DQK == 128) umma_ss_k8(tmem + BN + h * BH, q_desc_1, kdesc1, idesc_s, 0u);
+              else umma_ss_k4(tmem + BN + h * BH, q_desc_1, kdesc1, idesc_s, 0u);
+              umma_commit(bar(BarLayout::kS + 2 + h));
+            }
+            if (h == 1) {
+              if (!drain) umma_commit(bar(BarLayout::kEmpty + kslot));                // K(u) read by its S
+              if (prev_vslot >= 0) umma_commit(bar(BarLayout::kEmpty + prev_vslot));  // V(u-1) by its PVs
+              if (!drain && u == it.n - 1) umma_commit(bar(BarLayout::kQEmpty));      // last S of the unit
+            }
+          }
+          __syncwarp();
+          if (sm0.pending) {
+            ++npv0;
+            if (h == 1) ++sm0.pv_done;
+          }
+          if (sm1.pending) {
+            ++npv1;
+            if (h == 1) ++sm1.pv_done;
+          }
+          if (h == 0 && lane == 0 && !drain) {
+            const int tag = item_is_stride(it, u) ? (kStrideTag | item_tile(it, u)) : item_tile(it, u);
+            if (in0 && sm0.dbg_row >= 0 && sm0.kcount < p.dbg_cap) p.dbg_tiles[sm0.dbg_row * p.dbg_cap + sm0.kcount] = tag;
+            if (in1 && sm1.dbg_row >= 0 && sm1.kcount < p.dbg_cap) p.dbg_tiles[sm1.dbg_row * p.dbg_cap + sm1.kcount] = tag;
+          }
+          if (h == 0) {
+            sm0.kcount += in0;
+            sm1.kcount += in1;
+          }
           return true;
         };
-        for (int u = 0; u < it.n && ok; ++u) {
+        for (int u = 0; u < it.n; ++u) {
           const int kslot = L % C::kSlots, kuse = L / C::kSlots;
           ++L;
           const int vslot = L % C::kSlots, vuse = L / C::kSlots;
           ++L;
-          if (!mbar_wait(bar(BarLayout::kFull + kslot), kuse & 1, abort_flag)) {
-            record_timeout(abort_flag, p.err_flag);
+          if (!wait(bar(BarLayout::kFull + kslot), kuse & 1) ||
+              ((sm0.pending || sm1.pending) && !wait(bar(BarLayout::kFull + prev_vslot), prev_vuse & 1))) {
             ok = false;
             break;
           }
           tc_fence_after();
-          bool v_ready = false;
-          for (int t = 0; t < 2 && ok; ++t) {
-            const bool in = item_in_sub(it, t, u);
-            if (!in && !pending[t]) continue;
-            if (ksteps[t] > 0) {  // softmax t has consumed S_t and written P_t
-              if (!mbar_wait(bar(BarLayout::kP + t), (ksteps[t] - 1) & 1, abort_flag)) {
-                record_timeout(abort_flag, p.err_flag);
-                ok = false;
-                break;
-              }
-              tc_fence_after();
-            }
-            if (pending[t]) {
-              if ((!v_ready && !(v_ready = wait_prev_v())) || !issue_pv(t)) {
-                record_timeout(abort_flag, p.err_flag);
-                ok = false;
-                break;
-              }
-            }
-            if (in) {
-              const uint64_t kd0 = sw128_desc(sbase + C::kOffSlots + kslot * C::kSlot +
-                                                  ((DIFF && t == 1) ? BN * DQK * 2 : 0), 16, 1024);
-              const uint32_t dcol = tmem + t * BN;
-#pragma unroll
-              for (int kk = 0; kk < DQK / 16; ++kk) {
-                const uint64_t off = (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
-                umma_bf16_ss(dcol, q_desc0[t] + off, kd0 + off, idesc_s, kk > 0 ? 1u : 0u);
-              }
-              umma_commit(bar(BarLayout::kS + t));
-              if (dbg_row[t] >= 0 && kcount[t] < p.dbg_cap)
-                p.dbg_tiles[dbg_row[t] * p.dbg_cap + kcount[t]] =
-                    item_is_stride(it, u) ? (kStrideTag | item_tile(it, u)) : item_tile(it, u);
-              ++kcount[t];
-              ++ksteps[t];
-            }
-          }
-          if (!ok) break;
-          umma_commit(bar(BarLayout::kEmpty + kslot));                            // K(u) read by this step's S
-          if (prev_vslot >= 0) umma_commit(bar(BarLayout::kEmpty + prev_vslot));  // V(u-1) by its PVs
-          if (u == it.n - 1) umma_commit(bar(BarLayout::kQEmpty));                // last S of the unit: Q free
-          for (int t = 0; t < 2; ++t) pending[t] = item_in_sub(it, t, u);
-          prev_vslot = vslot;
-          prev_vuse = vuse;
-        }
-        bool v_ready = false;
-        for (int t = 0; t < 2 && ok; ++t) {
-          if (!pending[t]) continue;
-          if (!mbar_wait(bar(BarLayout::kP + t), (ksteps[t] - 1) & 1, abort_flag) ||
-              (!v_ready && !(v_ready = wait_prev_v())) || !issue_pv(t)) {
-            record_timeout(abort_flag, p.err_flag);
+          const bool in0 = item_in_sub(it, 0, u), in1 = item_in_sub(it, 1, u);
+          if (!half_step(I0{}, in0, in1, kslot, u, false) || !half_step(I1{}, in0, in1, kslot, u, false)) {
             ok = false;
             break;
           }
+          sm0.pending = in0;
+          sm1.pending = in1;
+          prev_vslot = vslot;
+          prev_vuse = vuse;
         }
-        if (ok && prev_vslot >= 0) umma_commit(bar(BarLayout::kEmpty + prev_vslot));
-        for (int t = 0; t < 2; ++t) {
-          if (dbg_row[t] >= 0) p.dbg_ntiles[dbg_row[t]] = kcount[t];
-          if (un.valid[t]) ++nunit[t];
+        if (ok && (sm0.pending || sm1.pending)) {
+          ok = wait(bar(BarLayout::kFull + prev_vslot), prev_vuse & 1);
+          if (ok) tc_fence_after();
+          ok = ok && half_step(I0{}, false, false, 0, 0, true) && half_step(I1{}, false, false, 0, 0, true);
         }
+        if (!ok) {
+          if (lane == 0) record_timeout(abort_flag, p.err_flag);
+          break;
+        }
+        if (lane == 0 && sm0.dbg_row >= 0) p.dbg_ntiles[sm0.dbg_row] = sm0.kcount;
+        if (lane == 0 && sm1.dbg_row >= 0) p.dbg_ntiles[sm1.dbg_row] = sm1.kcount;
+        if (un.valid[0]) ++sm0.nunit;
+        if (un.valid[1]) ++sm1.nunit;
       }
-      if (!ok || *abort_flag) {
-        umma_commit(bar(BarLayout::kFinal));
+      if (__any_sync(0xffffffffu, !ok || *abort_flag)) {
+        commit(bar(BarLayout::kFinal));
         mbar_wait_timed(bar(BarLayout::kFinal), 0);
       }
     }
@@ -503,7 +548,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         used = true;
       }
     };
-    int kglob = 0;   // S tiles consumed, across units (barrier phases)
+    int kglob = 0;   // key tiles consumed, across units (S / P phases)
+    int nlast = 0;   // kLast signals this sub's MMAs produce, across units
     int nunit = 0;   // units this sub took part in
     int nx = 0;      // differential hand-offs
     bool ok = true;
@@ -522,10 +568,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       float m_run = -INFINITY;  // running max, log2 units (scores * scale * log2 e)
       float l_run = 0.f;
       long long cells = 0;
-      int k = 0;  // tiles of this unit
 
-      for (int u = 0; u < it.n; ++u) {
+      for (int u = 0; u < it.n && ok; ++u) {
         if (!item_in_sub(it, t, u)) continue;
+        // no S of half 0 follows this tile's PV of half 0 in this unit when
+        // the next item is not this sub's: the MMA issuer signals kLast
+        const bool last_run = !(u + 1 < it.n && item_in_sub(it, t, u + 1));
         // attended columns [c0, c1] of this row in this tile
         int c0, c1;
         const int tile = item_tile(it, u);
@@ -538,88 +586,99 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (!row_ok) { c0 = 1; c1 = 0; }
         if (c1 >= c0) cells += c1 - c0 + 1;
-        const bool full = (c0 == 0 && c1 == BN - 1);
 
-        const bool got = mbar_wait(bar(BarLayout::kS + t), kglob & 1, abort_flag);
-        if (!__all_sync(0xffffffffu, got)) { if (lane == 0) record_timeout(abort_flag, p.err_flag); ok = false; break; }
-        tc_fence_after();
-
-        float s[BN];
-        tmem_ld128(s_tmem, s);
-        if (!__all_sync(0xffffffffu, full)) {
-          // Most partial tiles are cut on one side only (the window's start,
-          // or the diagonal): test only the side some row of the warp needs.
-          const bool cut_lo = __any_sync(0xffffffffu, c0 > 0), cut_hi = __any_sync(0xffffffffu, c1 < BN - 1);
-          if (cut_lo && cut_hi) {
-#pragma unroll
-            for (int c = 0; c < BN; ++c) s[c] = (c >= c0 && c <= c1) ? s[c] : -INFINITY;
-          } else if (cut_lo) {
-#pragma unroll
-            for (int c = 0; c < BN; ++c) s[c] = (c >= c0) ? s[c] : -INFINITY;
-          } else {
-#pragma unroll
-            for (int c = 0; c < BN; ++c) s[c] = (c <= c1) ? s[c] : -INFINITY;
-          }
-        }
-        // row max over 8 independent chains
-        float mx8[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) mx8[j] = s[j];
-#pragma unroll
-        for (int c = 8; c < BN; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], s[c]);
-        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-        const float m_tile = mx * cl2;  // -inf stays -inf
-        float m_use = m_run, alpha = 1.f;
-        bool rescale = false;
-        if (m_tile > m_run) {
-          if (m_run == -INFINITY) {
-            m_use = m_tile;  // nothing accumulated yet: the O row is 0 (or not yet written)
-            alpha = 0.f;
-          } else if (m_tile - m_run > kRescaleTau) {
-            m_use = m_tile;
-            alpha = ex2_approx(m_run - m_tile);
-            rescale = true;
-          }
-        }
-        const float msub = (m_use == -INFINITY) ? 0.f : m_use;
-        // p = 2^(s * scale * log2 e - m): packed fp32 pairs for the scaling
-        // and the row sum, MUFU ex2 for the exponential
-        const float2 cl2x2 = make_float2(cl2, cl2), negm = make_float2(-msub, -msub);
-        float2 rs2[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
-        uint32_t pk[BN / 2];
-#pragma unroll
-        for (int j = 0; j < BN / 2; ++j) {
-          const float2 x = __ffma2_rn(make_float2(s[2 * j], s[2 * j + 1]), cl2x2, negm);
-          const float p0 = ex2_approx(x.x);
-          const float p1 = ex2_approx(x.y);
-          rs2[j & 3] = __fadd2_rn(rs2[j & 3], make_float2(p0, p1));
-          pk[j] = pack_bf16(p0, p1);
-        }
-        const float2 rsum = __fadd2_rn(__fadd2_rn(rs2[0], rs2[1]), __fadd2_rn(rs2[2], rs2[3]));
-        const float rs = rsum.x + rsum.y;
-        l_run = l_run * alpha + rs;
-        m_run = m_use;
-
-        // P over the consumed scores: bf16 pairs in the first 64 columns of S_t
-        tmem_st32_u(s_tmem, pk);
-        tmem_st32_u(s_tmem + 32, pk + 32);
-        // the S_t commit also covered PV_t of the previous tile, so O_t is
-        // complete here and may be rescaled before PV_t of this tile
-        if (k > 0 && __any_sync(0xffffffffu, rescale)) {
-          const float f = rescale ? alpha : 1.f;
 #pragma unroll 1
-          for (int c = 0; c < DV; c += 32) {
-            float o[32];
-            tmem_ld32(o_tmem + c, o);
+        for (int h = 0; h < 2; ++h) {
+          const int c0h = c0 - h * BH, c1h = c1 - h * BH;  // attended columns of this half
+          const bool full = (c0h <= 0 && c1h >= BH - 1);
+          const bool got = mbar_wait(bar(BarLayout::kS + 2 * t + h), kglob & 1, abort_flag);
+          if (!__all_sync(0xffffffffu, got)) { if (lane == 0) record_timeout(abort_flag, p.err_flag); ok = false; break; }
+          tc_fence_after();
+
+          float s[BH];
+          tmem_ld64(s_tmem + h * BH, s);
+          if (!__all_sync(0xffffffffu, full)) {
+            // Most partial halves are cut on one side only (the window's
+            // start, or the diagonal): test only the side some row needs.
+            const bool cut_lo = __any_sync(0xffffffffu, c0h > 0), cut_hi = __any_sync(0xffffffffu, c1h < BH - 1);
+            if (cut_lo && cut_hi) {
 #pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] *= f;
-            tmem_st32(o_tmem + c, o);
+              for (int c = 0; c < BH; ++c) s[c] = (c >= c0h && c <= c1h) ? s[c] : -INFINITY;
+            } else if (cut_lo) {
+#pragma unroll
+              for (int c = 0; c < BH; ++c) s[c] = (c >= c0h) ? s[c] : -INFINITY;
+            } else {
+#pragma unroll
+              for (int c = 0; c < BH; ++c) s[c] = (c <= c1h) ? s[c] : -INFINITY;
+            }
           }
+          // row max over 8 independent chains
+          float mx8[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) mx8[j] = s[j];
+#pragma unroll
+          for (int c = 8; c < BH; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], s[c]);
+          const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                 fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+          const float m_tile = mx * cl2;  // -inf stays -inf
+          float m_use = m_run, alpha = 1.f;
+          bool rescale = false;
+          if (m_tile > m_run) {
+            if (m_run == -INFINITY) {
+              m_use = m_tile;  // nothing accumulated yet: the O row is 0 (or not yet written)
+              alpha = 0.f;
+            } else if (m_tile - m_run > kRescaleTau) {
+              m_use = m_tile;
+              alpha = ex2_approx(m_run - m_tile);
+              rescale = true;
+            }
+          }
+          const float msub = (m_use == -INFINITY) ? 0.f : m_use;
+          // p = 2^(s * scale * log2 e - m): packed fp32 pairs for the scaling
+          // and the row sum, MUFU ex2 for the exponential
+          const float2 cl2x2 = make_float2(cl2, cl2), negm = make_float2(-msub, -msub);
+          float2 rs2[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
+          uint32_t pk[BH / 2];
+#pragma unroll
+          for (int j = 0; j < BH / 2; ++j) {
+            const float2 x = __ffma2_rn(make_float2(s[2 * j], s[2 * j + 1]), cl2x2, negm);
+            const float p0 = ex2_approx(x.x);
+            const float p1 = ex2_approx(x.y);
+            rs2[j & 3] = __fadd2_rn(rs2[j & 3], make_float2(p0, p1));
+            pk[j] = pack_bf16(p0, p1);
+          }
+          const float2 rsum = __fadd2_rn(__fadd2_rn(rs2[0], rs2[1]), __fadd2_rn(rs2[2], rs2[3]));
+          const float rs = rsum.x + rsum.y;
+          l_run = l_run * alpha + rs;
+          m_run = m_use;
+
+          // P over the consumed scores: bf16 pairs in the first 32 columns of buffer h
+          tmem_st32_u(s_tmem + h * BH, pk);
+          if (__any_sync(0xffffffffu, rescale)) {
+            // O_t must hold every earlier PV before it is rescaled. Half 0:
+            // the S commit of this tile's half 1 follows the previous PV of
+            // half 1. Half 1: this tile's PV of half 0 is followed by the next
+            // tile's S of half 0, or else by kLast.
+            bool g;
+            if (h == 0) g = mbar_wait(bar(BarLayout::kS + 2 * t + 1), kglob & 1, abort_flag);
+            else if (!last_run) g = mbar_wait(bar(BarLayout::kS + 2 * t), (kglob + 1) & 1, abort_flag);
+            else g = mbar_wait(bar(BarLayout::kLast + t), nlast & 1, abort_flag);
+            if (!__all_sync(0xffffffffu, g)) { if (lane == 0) record_timeout(abort_flag, p.err_flag); ok = false; break; }
+            tc_fence_after();
+            const float f = rescale ? alpha : 1.f;
+#pragma unroll 1
+            for (int c = 0; c < DV; c += 32) {
+              float o[32];
+              tmem_ld32(o_tmem + c, o);
+#pragma unroll
+              for (int e = 0; e < 32; ++e) o[e] *= f;
+              tmem_st32(o_tmem + c, o);
+            }
+          }
+          tc_fence_before();
+          mbar_arrive(bar(BarLayout::kP + 2 * t + h));
         }
-        tc_fence_before();
-        mbar_arrive(bar(BarLayout::kP + t));
-        ++k;
+        if (last_run) ++nlast;
         ++kglob;
       }
       if (!ok) break;
