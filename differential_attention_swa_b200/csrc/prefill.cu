@@ -57,6 +57,39 @@ constexpr int kThreads = 384;
 // Lazy rescale threshold (log2 units): O and l keep a stale row max until a
 // new score exceeds it by more than this, so P stays below 2^8.
 constexpr float kRescaleTau = 8.0f;
+// Of every 8 pairs of exponentials in a score half, this many are evaluated
+// on the FMA pipe (exp2_fma2) instead of the MUFU unit, which both softmax
+// warpgroups share.
+#ifndef SWA_POLY_PAIRS_PER_8
+#define SWA_POLY_PAIRS_PER_8 0
+#endif
+constexpr int kPolyPairsPer8 = SWA_POLY_PAIRS_PER_8;
+
+// 2^x for a pair of floats on the FMA pipe (packed f32x2 arithmetic).
+// Cody-Waite range reduction with round-to-nearest: x = n + f, n integer,
+// f in [-1/2, 1/2]; adding and subtracting 1.5 * 2^23 rounds x to an integer
+// held in the low mantissa bits of j. 2^f comes from a cubic with p(0) = 1
+// whose other coefficients are a discrete minimax fit (linear programming)
+// of the relative error on [-1/2, 1/2]; 2^n is added to the exponent field:
+// the bit pattern of j times 2^23 is n << 23 modulo 2^32. Inputs at or
+// below -127 (-inf included) are clamped to -127, where f = 0, p(0) = 1 and
+// the result is exactly 0. Relative error of the fp32 evaluation: at most
+// 1.02e-4 on [-125, 8].
+constexpr float kExp2C1 = 0.6932829022407532f;
+constexpr float kExp2C2 = 0.24221095442771912f;
+constexpr float kExp2C3 = 0.05500892922282219f;
+__device__ __forceinline__ float2 exp2_fma2(float2 x) {
+  x.x = fmaxf(x.x, -127.f);
+  x.y = fmaxf(x.y, -127.f);
+  const float2 j = __fadd2_rn(x, make_float2(12582912.f, 12582912.f));
+  const float2 n = __fadd2_rn(j, make_float2(-12582912.f, -12582912.f));
+  const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), x);
+  float2 q = __ffma2_rn(make_float2(kExp2C3, kExp2C3), f, make_float2(kExp2C2, kExp2C2));
+  q = __ffma2_rn(q, f, make_float2(kExp2C1, kExp2C1));
+  q = __ffma2_rn(q, f, make_float2(1.f, 1.f));
+  return make_float2(__uint_as_float(__float_as_uint(j.x) * 8388608u + __float_as_uint(q.x)),
+                     __uint_as_float(__float_as_uint(j.y) * 8388608u + __float_as_uint(q.y)));
+}
 
 
 template <int DQK, int DV, bool DIFF>
@@ -559,8 +592,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ui >= nunits) continue;
       const Unit un = decode_unit(p, ui);
       const Items it = unit_items<GEN>(p, un);
-      if (!un.valid[t]) continue;
-      const int i = un.qt[t] * BM + r;  // query index
+      // this sub's fields as scalars: a run-time index into the unit's
+      // arrays would keep them in local memory
+      const bool valid_t = t ? un.valid[1] : un.valid[0];
+      if (!valid_t) continue;
+      const int qt_t = t ? un.qt[1] : un.qt[0];
+      const int hq = t ? un.hq[1] : un.hq[0];
+      const int ks_lo = t ? it.k[1].band_lo : it.k[0].band_lo;
+      const int ks_hi = t ? it.k[1].band_hi : it.k[0].band_hi;
+      const int ks_nst = t ? it.k[1].n_stride : it.k[0].n_stride;
+      auto in_sub = [&](int u) -> bool {
+        if (u < it.nst) return u < ks_nst;
+        const int kt = it.blo + (u - it.nst);
+        return kt >= ks_lo && kt <= ks_hi;
+      };
+      const int i = qt_t * BM + r;  // query index
       const bool row_ok = i < p.N;
       const int lo = window_lo(i, Wc);
       const int mst = GEN ? extra_rows_below(p.kind, lo, p.S)  // extra-view rows below lo
@@ -570,10 +616,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       long long cells = 0;
 
       for (int u = 0; u < it.n && ok; ++u) {
-        if (!item_in_sub(it, t, u)) continue;
+        if (!in_sub(u)) continue;
         // no S of half 0 follows this tile's PV of half 0 in this unit when
         // the next item is not this sub's: the MMA issuer signals kLast
-        const bool last_run = !(u + 1 < it.n && item_in_sub(it, t, u + 1));
+        const bool last_run = !(u + 1 < it.n && in_sub(u + 1));
         // attended columns [c0, c1] of this row in this tile
         int c0, c1;
         const int tile = item_tile(it, u);
@@ -642,8 +688,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int j = 0; j < BH / 2; ++j) {
             const float2 x = __ffma2_rn(make_float2(s[2 * j], s[2 * j + 1]), cl2x2, negm);
-            const float p0 = ex2_approx(x.x);
-            const float p1 = ex2_approx(x.y);
+            float p0, p1;
+            if ((j & 7) < kPolyPairsPer8) {
+              const float2 e = exp2_fma2(x);
+              p0 = e.x;
+              p1 = e.y;
+            } else {
+              p0 = ex2_approx(x.x);
+              p1 = ex2_approx(x.y);
+            }
             rs2[j & 3] = __fadd2_rn(rs2[j & 3], make_float2(p0, p1));
             pk[j] = pack_bf16(p0, p1);
           }
@@ -690,7 +743,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       ++nunit;
       tc_fence_after();
-      const int hq = un.hq[t];
       const int64_t orow = GEN ? (int64_t)(un.b * p.Hq + hq) * rmap.n + rmap.off + (int64_t)i * rmap.mul
                                : ((int64_t)(un.b * p.Hq + hq) * p.N + i);
       if (DIFF) {
@@ -713,7 +765,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_ld32(o2_tmem + c, b2);
 #pragma unroll
             for (int e = 0; e < 32; ++e) v[e] = v[e] * inv1 - b2[e] * f2;
-          }, un.b * p.Hq + hq, un.qt[t] * BM + qw * 32);
+          }, un.b * p.Hq + hq, qt_t * BM + qw * 32);
           // both accumulators read: the next unit's first PVs may overwrite them
           tc_fence_before();
           mbar_arrive(bar(BarLayout::kOFree + 0));
@@ -725,7 +777,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld32(o_tmem + c, v);
 #pragma unroll
           for (int e = 0; e < 32; ++e) v[e] *= inv;
-        }, un.b * p.Hq + hq, un.qt[t] * BM + qw * 32);
+        }, un.b * p.Hq + hq, qt_t * BM + qw * 32);
         tc_fence_before();
         mbar_arrive(bar(BarLayout::kOFree + t));  // O_t read: the next unit may overwrite it
         if (p.lse && row_ok) p.lse[orow] = (m_run + __log2f(l_run)) * 0.6931471805599453f;
@@ -735,7 +787,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) c += __shfl_xor_sync(0xffffffffu, c, off);
         if (lane == 0)
-          atomicAdd(reinterpret_cast<unsigned long long*>(p.dbg_cells + (int64_t)(un.b * p.Hq + hq) * p.nq + un.qt[t]),
+          atomicAdd(reinterpret_cast<unsigned long long*>(p.dbg_cells + (int64_t)(un.b * p.Hq + hq) * p.nq + qt_t),
                     static_cast<unsigned long long>(c));
       }
     }
