@@ -18,23 +18,23 @@
 // Warp roles (384 threads):
 //   warp 0      TMA producer: Q once, then K and V tiles through a ring of
 //               shared-memory slots.
-//   warp 1      TMEM owner and MMA issuer. A sub's 128 score columns are
-//               two 64-key buffers: half h of every key tile goes to buffer
-//               h. Per key tile and half, once both subs' P_t,h are written,
-//               one elected lane issues for each sub O_t += P_t,h(prev)
-//               V_h(prev) (A operand read from TMEM), then S_t,h = Q_t K_h^T
-//               into the buffer that held P_t,h, and the commits. The tensor
-//               core runs MMAs in issue order, so P is read before S
-//               overwrites it; while the softmax works on one half, the
-//               tensor core computes the other. The whole warp keeps the
-//               bookkeeping, so the MMA operands are warp-uniform values,
-//               and one issue block per half-step keeps the tensor core's
-//               queue fed.
+//   warp 1      TMEM owner and MMA issuer. A sub's 128 score columns hold
+//               one 128-key S (d = 128 and differential kernels) or two
+//               64-key buffers, one per half of the key tile (d = 64 window
+//               kernels). Per key tile (or half), as soon as a sub's P is
+//               written, one elected lane issues for that sub
+//               O_t += P V(prev) (A operand read from TMEM), then
+//               S_t = Q_t K^T into the columns that held P, and the commits.
+//               The tensor core runs MMAs in issue order, so P is read
+//               before S overwrites it. The sub whose softmax finishes first
+//               gets its next S first, so one sub's MMAs overlap the other
+//               sub's exponentials; with two halves, S of one half also
+//               overlaps the softmax of the other. The whole warp keeps the
+//               bookkeeping, so the MMA operands are warp-uniform values.
 //   warps 4-7   softmax of sub 0, warps 8-11 softmax of sub 1: one thread
 //               per query row (TMEM lane), fp32 online softmax in the log2
-//               domain over 64-key halves, P as bf16 back into TMEM over the
-//               consumed scores, lazy rescaling of O, then the epilogue
-//               O / l -> bf16.
+//               domain, P as bf16 back into TMEM over the consumed scores,
+//               lazy rescaling of O, then the epilogue O / l -> bf16.
 // Every wait is bounded; on a timeout the CTA records SWA_ERR_TIMEOUT,
 // drains what it has in flight, frees TMEM and returns.
 #include <cuda.h>
@@ -52,18 +52,44 @@ namespace swa {
 
 constexpr int BM = 128;  // query rows per sub (TMEM lanes)
 constexpr int BN = 128;  // keys per tile (S columns of a sub)
-constexpr int BH = 64;   // keys per score buffer (half a tile)
+
+
+// warp 0 producer, warp 1 MMA issuer, warps 4-11 softmax (warp w reaches
+// TMEM lanes 32 * (w % 4) .. + 31). Warps 2-3 have no role: registers are
+// allocated to whole groups of four warps, so dropping them would not raise
+// the 168 registers a thread gets.
+constexpr int kSmxWarp0 = 4;
 constexpr int kThreads = 384;
 // Lazy rescale threshold (log2 units): O and l keep a stale row max until a
 // new score exceeds it by more than this, so P stays below 2^8.
 constexpr float kRescaleTau = 8.0f;
-// Of every 8 pairs of exponentials in a score half, this many are evaluated
-// on the FMA pipe (exp2_fma2) instead of the MUFU unit, which both softmax
-// warpgroups share.
-#ifndef SWA_POLY_PAIRS_PER_8
-#define SWA_POLY_PAIRS_PER_8 0
+
+
+// Per-instantiation choices, measured on B200 (tcgen05 MMAs with M = 128 and
+// both operands in shared memory cost about as much at N = 64 as at N = 128,
+// because reading the operands takes as long as the math):
+//   NH    score buffers per key tile and sub: 1 = one 128-key S (N = 128
+//         MMAs), 2 = two 64-key halves, so S of one half runs during the
+//         softmax of the other at twice the MMA cost per score;
+//   POLY  of every 8 pairs of exponentials, how many are evaluated on the FMA
+//         pipe (exp2_fma2) instead of the MUFU unit.
+// d = 128 window kernels: one buffer (the MMA cost dominates); differential
+// (d_qk = 64, d_v = 128): one buffer, 2 of 8 pairs on the FMA pipe; d = 64
+// window and strided kernels (short units, MUFU-bound): two halves.
+template <int DQK, int DV, bool DIFF>
+struct PrefillTune {
+#ifdef SWA_NH
+  static constexpr int NH = SWA_NH;
+#else
+  static constexpr int NH = (DQK == 128 || DIFF) ? 1 : 2;
 #endif
-constexpr int kPolyPairsPer8 = SWA_POLY_PAIRS_PER_8;
+#ifdef SWA_POLY_PAIRS_PER_8
+  static constexpr int POLY = SWA_POLY_PAIRS_PER_8;
+#else
+  static constexpr int POLY = DIFF ? 2 : 0;
+#endif
+  static_assert(NH == 1 || NH == 2, "one or two score buffers per tile");
+};
 
 // 2^x for a pair of floats on the FMA pipe (packed f32x2 arithmetic).
 // Cody-Waite range reduction with round-to-nearest: x = n + f, n integer,
@@ -239,6 +265,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                    const __grid_constant__ CUtensorMap tm_vs, const __grid_constant__ CUtensorMap tm_o,
                    const PrefillParams p, const RowMap rmap) {
   using C = PrefillCfg<DQK, DV, DIFF>;
+  constexpr int NH = PrefillTune<DQK, DV, DIFF>::NH;
+  constexpr int BH = BN / NH;  // keys per score buffer
+  constexpr int kPolyPairsPer8 = PrefillTune<DQK, DV, DIFF>::POLY;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -437,44 +466,57 @@ __global__ void __launch_bounds__(kThreads, 1)
           constexpr int h = decltype(hc)::value;
           int& npv0 = h ? sm0.npv1 : sm0.npv0;
           int& npv1 = h ? sm1.npv1 : sm1.npv0;
-          if (sm0.pending && !wait(bar(BarLayout::kP + 0 + h), npv0 & 1)) return false;
-          if (sm1.pending && !wait(bar(BarLayout::kP + 2 + h), npv1 & 1)) return false;
-          // the first PV of a unit overwrites O_t: the previous unit's epilogue must be done with it
           const bool f0 = (h == 0 && sm0.pv_done == 0), f1 = (h == 0 && sm1.pv_done == 0);
-          if (sm0.pending && f0 && sm0.nunit > 0 && !wait(bar(BarLayout::kOFree + 0), (sm0.nunit - 1) & 1))
-            return false;
-          if (sm1.pending && f1 && sm1.nunit > 0 && !wait(bar(BarLayout::kOFree + 1), (sm1.nunit - 1) & 1))
-            return false;
-          tc_fence_after();
           const uint64_t vdesc =
               sw128_desc(sbase + C::kOffSlots + prev_vslot * C::kSlot + h * (BH / 16) * 2048, 16384, 1024);
           const uint32_t kbase = sbase + C::kOffSlots + kslot * C::kSlot + h * BH * 128;
           const uint64_t kdesc0 = sw128_desc(kbase, 16, 1024);
           const uint64_t kdesc1 = sw128_desc(kbase + (DIFF ? BN * DQK * 2 : 0), 16, 1024);
-          const bool o_done0 = h == 1 && sm0.pending && sm0.pv_done + 1 == sm0.ntot;
-          const bool o_done1 = h == 1 && sm1.pending && sm1.pv_done + 1 == sm1.ntot;
+          const bool o_done0 = h == NH - 1 && sm0.pending && sm0.pv_done + 1 == sm0.ntot;
+          const bool o_done1 = h == NH - 1 && sm1.pending && sm1.pv_done + 1 == sm1.ntot;
+          // PV of the previous key tile (A = P in TMEM over its scores), then S
+          // of this one into the same columns; BH keys of P per PV
+          auto pv = [&](uint32_t d, uint32_t a, uint32_t acc) {
+            if (BH == 128) umma_ts_k8(d, a, vdesc, idesc_pv, acc);
+            else umma_ts_k4(d, a, vdesc, idesc_pv, acc);
+          };
+          auto qk = [&](uint32_t d, uint64_t qd, uint64_t kd) {
+            if (DQK == 128) umma_ss_k8(d, qd, kd, idesc_s, 0u);
+            else umma_ss_k4(d, qd, kd, idesc_s, 0u);
+          };
+          // each sub's burst goes out as soon as that sub's P is written, so a
+          // sub that finishes its softmax first gets its next S first
+          if (sm0.pending && !wait(bar(BarLayout::kP + 0 + h), npv0 & 1)) return false;
+          if (sm0.pending && f0 && sm0.nunit > 0 && !wait(bar(BarLayout::kOFree + 0), (sm0.nunit - 1) & 1))
+            return false;
+          tc_fence_after();
           if (elect_one()) {
             if (sm0.pending) {
-              umma_ts_k4(tmem + C::kOCol0, tmem + h * BH, vdesc, idesc_pv, f0 ? 0u : 1u);
-              if (h == 0 && !in0) umma_commit(bar(BarLayout::kLast + 0));  // no S of half 0 follows
+              pv(tmem + C::kOCol0, tmem + h * BH, f0 ? 0u : 1u);
+              if (NH == 2 && h == 0 && !in0) umma_commit(bar(BarLayout::kLast + 0));  // no S of half 0 follows
               if (o_done0) umma_commit(bar(BarLayout::kO + 0));
             }
             if (in0) {
-              if (DQK == 128) umma_ss_k8(tmem + h * BH, q_desc_0, kdesc0, idesc_s, 0u);
-              else umma_ss_k4(tmem + h * BH, q_desc_0, kdesc0, idesc_s, 0u);
+              qk(tmem + h * BH, q_desc_0, kdesc0);
               umma_commit(bar(BarLayout::kS + 0 + h));
             }
+          }
+          __syncwarp();
+          if (sm1.pending && !wait(bar(BarLayout::kP + 2 + h), npv1 & 1)) return false;
+          if (sm1.pending && f1 && sm1.nunit > 0 && !wait(bar(BarLayout::kOFree + 1), (sm1.nunit - 1) & 1))
+            return false;
+          tc_fence_after();
+          if (elect_one()) {
             if (sm1.pending) {
-              umma_ts_k4(tmem + C::kOCol1, tmem + BN + h * BH, vdesc, idesc_pv, f1 ? 0u : 1u);
-              if (h == 0 && !in1) umma_commit(bar(BarLayout::kLast + 1));
+              pv(tmem + C::kOCol1, tmem + BN + h * BH, f1 ? 0u : 1u);
+              if (NH == 2 && h == 0 && !in1) umma_commit(bar(BarLayout::kLast + 1));
               if (o_done1) umma_commit(bar(BarLayout::kO + 1));
             }
             if (in1) {
-              if (DQK == 128) umma_ss_k8(tmem + BN + h * BH, q_desc_1, kdesc1, idesc_s, 0u);
-              else umma_ss_k4(tmem + BN + h * BH, q_desc_1, kdesc1, idesc_s, 0u);
+              qk(tmem + BN + h * BH, q_desc_1, kdesc1);
               umma_commit(bar(BarLayout::kS + 2 + h));
             }
-            if (h == 1) {
+            if (h == NH - 1) {
               if (!drain) umma_commit(bar(BarLayout::kEmpty + kslot));                // K(u) read by its S
               if (prev_vslot >= 0) umma_commit(bar(BarLayout::kEmpty + prev_vslot));  // V(u-1) by its PVs
               if (!drain && u == it.n - 1) umma_commit(bar(BarLayout::kQEmpty));      // last S of the unit
@@ -483,11 +525,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           __syncwarp();
           if (sm0.pending) {
             ++npv0;
-            if (h == 1) ++sm0.pv_done;
+            if (h == NH - 1) ++sm0.pv_done;
           }
           if (sm1.pending) {
             ++npv1;
-            if (h == 1) ++sm1.pv_done;
+            if (h == NH - 1) ++sm1.pv_done;
           }
           if (h == 0 && lane == 0 && !drain) {
             const int tag = item_is_stride(it, u) ? (kStrideTag | item_tile(it, u)) : item_tile(it, u);
@@ -512,7 +554,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_fence_after();
           const bool in0 = item_in_sub(it, 0, u), in1 = item_in_sub(it, 1, u);
-          if (!half_step(I0{}, in0, in1, kslot, u, false) || !half_step(I1{}, in0, in1, kslot, u, false)) {
+          if (!half_step(I0{}, in0, in1, kslot, u, false) ||
+              (NH == 2 && !half_step(I1{}, in0, in1, kslot, u, false))) {
             ok = false;
             break;
           }
@@ -524,7 +567,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok && (sm0.pending || sm1.pending)) {
           ok = wait(bar(BarLayout::kFull + prev_vslot), prev_vuse & 1);
           if (ok) tc_fence_after();
-          ok = ok && half_step(I0{}, false, false, 0, 0, true) && half_step(I1{}, false, false, 0, 0, true);
+          ok = ok && half_step(I0{}, false, false, 0, 0, true) &&
+               (NH == 1 || half_step(I1{}, false, false, 0, 0, true));
         }
         if (!ok) {
           if (lane == 0) record_timeout(abort_flag, p.err_flag);
@@ -540,9 +584,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait_timed(bar(BarLayout::kFinal), 0);
       }
     }
-  } else if (warp >= 4) {
+  } else if (warp >= kSmxWarp0) {
     // ------------------------------------------------------- softmax ---
-    const int t = (warp - 4) >> 2;       // sub
+    const int t = (warp - kSmxWarp0) >> 2;  // sub
     const int qw = warp & 3;             // TMEM lane quarter
     const int r = qw * 32 + lane;        // row within the sub's tile
     const uint32_t lane_addr = static_cast<uint32_t>(qw * 32) << 16;
@@ -553,7 +597,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Epilogue store: this warp's 32 output rows go through a 4 KB
     // shared-memory box (128-byte swizzle), 64 columns at a time, and lane 0
     // writes the box with one TMA store; rows past N are clipped by TMA.
-    const uint32_t stage = sbase + C::kOffStage + (warp - 4) * 4096;
+    const uint32_t stage = sbase + C::kOffStage + (warp - kSmxWarp0) * 4096;
     bool stage_used = false;
     auto store_rows = [&](bool& used, auto&& fetch, int zrow, int row0) {
 #pragma unroll 1
@@ -634,7 +678,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (c1 >= c0) cells += c1 - c0 + 1;
 
 #pragma unroll 1
-        for (int h = 0; h < 2; ++h) {
+        for (int h = 0; h < NH; ++h) {
           const int c0h = c0 - h * BH, c1h = c1 - h * BH;  // attended columns of this half
           const bool full = (c0h <= 0 && c1h >= BH - 1);
           const bool got = mbar_wait(bar(BarLayout::kS + 2 * t + h), kglob & 1, abort_flag);
@@ -642,7 +686,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
 
           float s[BH];
-          tmem_ld64(s_tmem + h * BH, s);
+          if (BH == 128) tmem_ld128(s_tmem, s);
+          else tmem_ld64(s_tmem + h * BH, s);
           if (!__all_sync(0xffffffffu, full)) {
             // Most partial halves are cut on one side only (the window's
             // start, or the diagonal): test only the side some row needs.
@@ -705,15 +750,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           l_run = l_run * alpha + rs;
           m_run = m_use;
 
-          // P over the consumed scores: bf16 pairs in the first 32 columns of buffer h
+          // P over the consumed scores: bf16 pairs, 32 columns per 64 keys
           tmem_st32_u(s_tmem + h * BH, pk);
+          if (BH == 128) tmem_st32_u(s_tmem + 32, pk + 32);
           if (__any_sync(0xffffffffu, rescale)) {
-            // O_t must hold every earlier PV before it is rescaled. Half 0:
-            // the S commit of this tile's half 1 follows the previous PV of
-            // half 1. Half 1: this tile's PV of half 0 is followed by the next
-            // tile's S of half 0, or else by kLast.
-            bool g;
-            if (h == 0) g = mbar_wait(bar(BarLayout::kS + 2 * t + 1), kglob & 1, abort_flag);
+            // O_t must hold every earlier PV before it is rescaled. One
+            // buffer per tile: the commit of S_t (waited for above) follows
+            // the PV of the previous tile, so O_t is complete already. Two
+            // halves: for half 0, the S commit of this tile's half 1 follows
+            // the previous PV of half 1; for half 1, this tile's PV of half 0
+            // is followed by the next tile's S of half 0, or else by kLast.
+            bool g = true;
+            if (NH == 1) g = true;
+            else if (h == 0) g = mbar_wait(bar(BarLayout::kS + 2 * t + 1), kglob & 1, abort_flag);
             else if (!last_run) g = mbar_wait(bar(BarLayout::kS + 2 * t), (kglob + 1) & 1, abort_flag);
             else g = mbar_wait(bar(BarLayout::kLast + t), nlast & 1, abort_flag);
             if (!__all_sync(0xffffffffu, g)) { if (lane == 0) record_timeout(abort_flag, p.err_flag); ok = false; break; }
@@ -793,7 +842,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
-  if (warp >= 4 && lane == 0) bulk_wait_all();  // output stores complete before exit
+  if (warp >= kSmxWarp0 && lane == 0) bulk_wait_all();  // output stores complete before exit
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
