@@ -204,7 +204,7 @@ def prefill_workload(name, rank):
         ins = [t.cuda() for t in diff_inputs(w.B, w.Hq, w.Hkv, w.N, w.d, w.dv, seed=seed)]
         lam = torch.full((w.Hq,), w.lam, dtype=torch.float32, device="cuda")
         out = torch.empty((w.B, w.Hq, w.N, w.dv_), dtype=torch.bfloat16, device="cuda")
-        fn = lambda: swa.diff_attn_fwd(*ins, lam, window=w.W, scale=w.scale, out=out)
+        call = lambda xs, o: swa.diff_attn_fwd(*xs, lam, window=w.W, scale=w.scale, out=o)
         nnz = swa.count_nonmasked(swa.MASK_WINDOW, w.N, w.W)
         flops = nnz * w.B * w.Hq * 2 * (2 * w.d + 2 * w.dv_)  # two maps, each 2*d_qk + 2*d_v per cell
     elif w.kind == "swa_bwd":
@@ -223,28 +223,29 @@ def prefill_workload(name, rank):
             nnz = swa.count_nonmasked(swa.MASK_WINDOW, w.N, w.W)
         ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
         out = None
-        fn = lambda: swa.swa_attn_bwd(q, k, v, o, d_o, lse, w.W, workspace=ws, stride=w.S)
+        call = lambda xs, _o: swa.swa_attn_bwd(*xs[:6], w.W, workspace=xs[6], stride=w.S)
         # the usual accounting: scores, dP, dV, dQ, dK = 5 products of 2*d per cell
         flops = 10 * w.d * nnz * w.B * w.Hq
-        ins = [q, k, v, o, lse, d_o, ws]
+        ins = [q, k, v, o, d_o, lse, ws]
     else:
         q, k, v = (t.cuda() for t in attn_inputs(w.B, w.Hq, w.Hkv, w.N, w.d, seed=seed))
         out = torch.empty_like(q)
         if w.kind == "swa":
-            fn = lambda: swa.swa_attn_fwd(q, k, v, w.W, out=out)
+            call = lambda xs, o: swa.swa_attn_fwd(*xs, w.W, out=o)
             nnz = swa.count_nonmasked(swa.MASK_WINDOW, w.N, w.W)
         elif w.kind == "global":  # S carries the number of global tokens
-            fn = lambda: swa.global_attn_fwd(q, k, v, w.W, w.S, out=out)
+            call = lambda xs, o: swa.global_attn_fwd(*xs, w.W, w.S, out=o)
             nnz = swa.count_nonmasked(swa.MASK_GLOBAL, w.N, w.W, w.S)
         elif w.kind == "dilated":  # S carries the dilation; each row sees min(W, i // S + 1) keys
-            fn = lambda: swa.dilated_attn_fwd(q, k, v, w.W, w.S, out=out)
+            call = lambda xs, o: swa.dilated_attn_fwd(*xs, w.W, w.S, out=o)
             nnz = sum(min(w.W, i // w.S + 1) for i in range(w.N))
         else:
-            fn = lambda: swa.strided_attn_fwd(q, k, v, w.W, w.S, out=out)
+            call = lambda xs, o: swa.strided_attn_fwd(*xs, w.W, w.S, out=o)
             nnz = swa.count_nonmasked(swa.MASK_STRIDED, w.N, w.W, w.S)
         flops = 4 * w.d * nnz * w.B * w.Hq
         ins = [q, k, v]
-    return w, fn, flops, ins, out
+    fn = lambda: call(ins, out)
+    return w, fn, call, flops, ins, out
 
 
 def decode_workload(rank, name="gemma_swa_decode"):
@@ -343,7 +344,7 @@ def measure_ours(args, rank, world, peaks, peak_src, dist):
     main_name = args.only or "mistral_swa_prefill"
     if main_name.endswith("_decode"):
         return measure_decode_only(args, rank, world, peaks, flush, stream, main_name)
-    w, fn, flops, ins, out = prefill_workload(main_name, rank)
+    w, fn, call, flops, ins, out = prefill_workload(main_name, rank)
     clocks = ClockSampler(bus)
     if dist:
         dist.barrier()
@@ -379,40 +380,61 @@ def measure_ours(args, rank, world, peaks, peak_src, dist):
         "gpu_launches": args.steps,
     }
     if not args.no_e2e and out is not None:  # the backward workload has no single output to copy back
-        res["e2e"] = measure_e2e(w, fn, ins, out, flops, stream)
+        res["e2e"] = measure_e2e(call, ins, out, flops, stream)
     if not args.no_variants and args.only is None:
         res["variants"] = measure_variants(args, rank, peaks, flush, stream)
     return res
 
 
-def measure_e2e(w, fn, ins, out, flops, stream, steps=5):
-    """Same metric through the public call with host buffers: pinned host
-    inputs copied in, the kernel, the output copied back, every step."""
+def measure_e2e(call, ins, out, flops, stream, steps=8):
+    """Same metric through the public call with host buffers: every step
+    copies its inputs in from pinned host memory, runs the call and copies
+    its output back. Steps are pipelined over two sets of device buffers on
+    three streams (inputs of step k+1 go in while step k computes and step
+    k-1's output comes back), as a serving loop would; the timed region runs
+    from the first input copy to the last output copy."""
     import torch
 
     hosts = [t.cpu().pin_memory() for t in ins]
-    host_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    host_out = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
+    dev_in = [list(ins), [torch.empty_like(t) for t in ins]]
+    dev_out = [out, torch.empty_like(out)]
     h2d = sum(t.numel() * t.element_size() for t in hosts)
-    d2h = host_out.numel() * host_out.element_size()
+    d2h = out.numel() * out.element_size()
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_comp = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
 
-    def step():
-        for h, d in zip(hosts, ins):
-            d.copy_(h, non_blocking=True)
-        fn()
-        host_out.copy_(out, non_blocking=True)
+    def run(n):
+        for k in range(n):
+            b = k % 2
+            with torch.cuda.stream(s_in):
+                if k >= 2:
+                    s_in.wait_event(ev_comp[b])  # step k-2 has finished reading these inputs
+                for h, d in zip(hosts, dev_in[b]):
+                    d.copy_(h, non_blocking=True)
+                ev_in[b].record(s_in)
+            stream.wait_event(ev_in[b])
+            if k >= 2:
+                stream.wait_event(ev_out[b])  # step k-2's output has been copied out
+            call(dev_in[b], dev_out[b])
+            ev_comp[b].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_comp[b])
+                host_out[b].copy_(dev_out[b], non_blocking=True)
+                ev_out[b].record(s_out)
 
-    for _ in range(2):
-        step()
+    run(2)
     torch.cuda.synchronize()
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record(stream)
-    for _ in range(steps):
-        step()
-    b.record(stream)
+    a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(s_in)
+    run(steps)
+    z.record(s_out)
     torch.cuda.synchronize()
-    ms = a.elapsed_time(b) / steps
+    ms = a.elapsed_time(z) / steps
     return {"value": round(flops / (ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s", "ms_per_step": round(ms, 4),
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "pipelined": "2 buffer sets, 3 streams"}
 
 
 def measure_decode_only(args, rank, world, peaks, flush, stream, name):
@@ -452,7 +474,7 @@ def measure_variants(args, rank, peaks, flush, stream):
     reps = max(5, min(args.steps, 10))
     for name in ("local_strided_prefill", "diff_causal", "gemma_swa_prefill", "longformer_global_prefill",
                  "longformer_dilated_prefill", "mistral_swa_backward", "local_strided_backward"):
-        w, fn, flops, ins, o = prefill_workload(name, rank)
+        w, fn, _call, flops, ins, o = prefill_workload(name, rank)
         ms = time_steps(fn, reps, 3, flush, stream)
         mean_ms = sum(ms) / len(ms)
         tf = flops / (mean_ms * 1e-3) / 1e12
