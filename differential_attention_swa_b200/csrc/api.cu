@@ -137,6 +137,11 @@ swa_status_t run_prefill(int kind, bool diff, const void* q, const void* k, cons
   } else if (G % 2 == 0) {
     p.mode = kModeHeadPairs;
     nunits = nB * Hkv * (G / 2) * p.nq;
+  } else if (Hq % 2 == 0 && dqk == 64) {
+    // odd group size: pair consecutive query heads at the same query tile,
+    // each with its own KV head, so both subs visit the same key tiles
+    p.mode = kModeKvPairs;
+    nunits = nB * (Hq / 2) * p.nq;
   } else {
     p.mode = kModeTilePairs;
     nunits = nB * Hq * ((p.nq + 1) / 2);

@@ -14,7 +14,8 @@ namespace swa {
 enum UnitMode {
   kModeHeadPairs = 0,  // two query heads of one KV group, same rows
   kModeTilePairs = 1,  // two consecutive query tiles of one head
-  kModeDiff = 2        // the two maps of differential attention
+  kModeDiff = 2,       // the two maps of differential attention
+  kModeKvPairs = 3     // two query heads of different KV groups, same rows
 };
 
 struct PrefillParams {
@@ -69,7 +70,6 @@ struct PrefillMaps {
 
 cudaError_t launch_prefill(const PrefillMaps& maps, const PrefillParams& p, const RowMap& rows, int dqk, int dv,
                            bool diff, int nunits, cudaStream_t stream);
-int prefill_smem_bytes(int dqk, int dv, bool diff);
 
 struct DecodeParams {
   const void* q;

@@ -118,11 +118,13 @@ __device__ __forceinline__ float2 exp2_fma2(float2 x) {
 }
 
 
-template <int DQK, int DV, bool DIFF>
+// KV2: the two subs read different KV heads (kModeKvPairs); a ring slot then
+// holds the K (or V) tiles of both.
+template <int DQK, int DV, bool DIFF, bool KV2 = false>
 struct PrefillCfg {
   static constexpr int kQBytes = BM * DQK * 2;
-  static constexpr int kKBytes = BN * DQK * 2 * (DIFF ? 2 : 1);
-  static constexpr int kVBytes = BN * DV * 2;
+  static constexpr int kKBytes = BN * DQK * 2 * ((DIFF || KV2) ? 2 : 1);
+  static constexpr int kVBytes = BN * DV * 2 * (KV2 ? 2 : 1);
   static constexpr int kSlot = kKBytes > kVBytes ? kKBytes : kVBytes;
   static constexpr int kStageBytes = 8 * 32 * 64 * 2;  // per softmax warp: 32 rows x 64 columns of bf16
   static constexpr int kTiles = 2 * kQBytes + kStageBytes;
@@ -163,6 +165,7 @@ struct BarLayout {
 
 struct Unit {
   int b, hkv;
+  int hkv1;  // KV head of sub 1 (differs from hkv in kModeKvPairs only)
   int hq[2];
   int qt[2];
   int valid[2];
@@ -183,6 +186,20 @@ __device__ __forceinline__ Unit decode_unit(const PrefillParams& p, int u) {
     r.hq[1] = r.hq[0] + 1;
     r.qt[0] = r.qt[1] = qt;
     r.valid[0] = r.valid[1] = 1;
+  } else if (p.mode == kModeKvPairs) {
+    // consecutive query heads 2gp, 2gp+1 at the same query tile; each reads
+    // its own KV head (odd group sizes)
+    const int half = p.Hq / 2;
+    const int qt = p.nq - 1 - u / (p.B * half);
+    const int bh = u % (p.B * half);
+    r.b = bh / half;
+    r.hq[0] = 2 * (bh % half);
+    r.hq[1] = r.hq[0] + 1;
+    r.hkv = r.hq[0] / p.G;
+    r.hkv1 = r.hq[1] / p.G;
+    r.qt[0] = r.qt[1] = qt;
+    r.valid[0] = r.valid[1] = 1;
+    return r;
   } else if (p.mode == kModeTilePairs) {
     const int nqp = (p.nq + 1) / 2;
     const int qp = nqp - 1 - u / (p.B * p.Hq);
@@ -203,6 +220,7 @@ __device__ __forceinline__ Unit decode_unit(const PrefillParams& p, int u) {
     r.qt[0] = r.qt[1] = qt;
     r.valid[0] = r.valid[1] = 1;
   }
+  r.hkv1 = r.hkv;
   return r;
 }
 
@@ -257,14 +275,14 @@ __device__ __forceinline__ void record_timeout(volatile int* abort_flag, int* er
 // GEN instantiations serve the window + global-token kind and strided views
 // (dilated windows: rows r, r + dil, ... of each head, with the log-sum-exp
 // written at the original rows); the others compile without that code.
-template <int DQK, int DV, bool DIFF, bool GEN>
+template <int DQK, int DV, bool DIFF, bool GEN, bool KV2>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_q2,
                    const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_k2,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_ks,
                    const __grid_constant__ CUtensorMap tm_vs, const __grid_constant__ CUtensorMap tm_o,
                    const PrefillParams p, const RowMap rmap) {
-  using C = PrefillCfg<DQK, DV, DIFF>;
+  using C = PrefillCfg<DQK, DV, DIFF, KV2>;
   constexpr int NH = PrefillTune<DQK, DV, DIFF>::NH;
   constexpr int BH = BN / NH;  // keys per score buffer
   constexpr int kPolyPairsPer8 = PrefillTune<DQK, DV, DIFF>::POLY;
@@ -355,6 +373,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         ++nq_ld;
         const int zkv = un.b * p.Hkv + un.hkv;
+        const int zkv1 = un.b * p.Hkv + un.hkv1;
         for (int u = 0; u < it.n && ok; ++u) {
           const bool st = item_is_stride(it, u);
           const int row = item_tile(it, u) * BN;
@@ -376,6 +395,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int bx = 0; bx < DQK / 64; ++bx)
                   tma_load_3d(dst + BN * DQK * 2 + bx * 16384, &tm_k2, bar(BarLayout::kFull + slot), bx * 64,
                               row, zkv);
+              if (KV2)  // sub 1's KV head
+                for (int bx = 0; bx < DQK / 64; ++bx)
+                  tma_load_3d(dst + BN * DQK * 2 + bx * 16384, m, bar(BarLayout::kFull + slot), bx * 64, row,
+                              zkv1);
               issued[slot] = use + 1;
             }
           }
@@ -392,6 +415,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const CUtensorMap* m = st ? &tm_vs : &tm_v;
             for (int bx = 0; bx < DV / 64; ++bx)
               tma_load_3d(dst + bx * 16384, m, bar(BarLayout::kFull + slot), bx * 64, row, zkv);
+            if (KV2)
+              for (int bx = 0; bx < DV / 64; ++bx)
+                tma_load_3d(dst + BN * DV * 2 + bx * 16384, m, bar(BarLayout::kFull + slot), bx * 64, row, zkv1);
             issued[slot] = use + 1;
           }
         }
@@ -471,14 +497,17 @@ __global__ void __launch_bounds__(kThreads, 1)
               sw128_desc(sbase + C::kOffSlots + prev_vslot * C::kSlot + h * (BH / 16) * 2048, 16384, 1024);
           const uint32_t kbase = sbase + C::kOffSlots + kslot * C::kSlot + h * BH * 128;
           const uint64_t kdesc0 = sw128_desc(kbase, 16, 1024);
-          const uint64_t kdesc1 = sw128_desc(kbase + (DIFF ? BN * DQK * 2 : 0), 16, 1024);
+          const uint64_t kdesc1 = sw128_desc(kbase + ((DIFF || KV2) ? BN * DQK * 2 : 0), 16, 1024);
+          // sub 1's V tile (KV2: the second tile in the slot); the start
+          // address field counts 16-byte units
+          const uint64_t vdesc1 = vdesc + (KV2 ? (BN * DV * 2) >> 4 : 0);
           const bool o_done0 = h == NH - 1 && sm0.pending && sm0.pv_done + 1 == sm0.ntot;
           const bool o_done1 = h == NH - 1 && sm1.pending && sm1.pv_done + 1 == sm1.ntot;
           // PV of the previous key tile (A = P in TMEM over its scores), then S
           // of this one into the same columns; BH keys of P per PV
-          auto pv = [&](uint32_t d, uint32_t a, uint32_t acc) {
-            if (BH == 128) umma_ts_k8(d, a, vdesc, idesc_pv, acc);
-            else umma_ts_k4(d, a, vdesc, idesc_pv, acc);
+          auto pv = [&](uint32_t d, uint32_t a, uint64_t vd, uint32_t acc) {
+            if (BH == 128) umma_ts_k8(d, a, vd, idesc_pv, acc);
+            else umma_ts_k4(d, a, vd, idesc_pv, acc);
           };
           auto qk = [&](uint32_t d, uint64_t qd, uint64_t kd) {
             if (DQK == 128) umma_ss_k8(d, qd, kd, idesc_s, 0u);
@@ -492,7 +521,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           if (elect_one()) {
             if (sm0.pending) {
-              pv(tmem + C::kOCol0, tmem + h * BH, f0 ? 0u : 1u);
+              pv(tmem + C::kOCol0, tmem + h * BH, vdesc, f0 ? 0u : 1u);
               if (NH == 2 && h == 0 && !in0) umma_commit(bar(BarLayout::kLast + 0));  // no S of half 0 follows
               if (o_done0) umma_commit(bar(BarLayout::kO + 0));
             }
@@ -508,7 +537,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           if (elect_one()) {
             if (sm1.pending) {
-              pv(tmem + C::kOCol1, tmem + BN + h * BH, f1 ? 0u : 1u);
+              pv(tmem + C::kOCol1, tmem + BN + h * BH, vdesc1, f1 ? 0u : 1u);
               if (NH == 2 && h == 0 && !in1) umma_commit(bar(BarLayout::kLast + 1));
               if (o_done1) umma_commit(bar(BarLayout::kO + 1));
             }
@@ -852,11 +881,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int DQK, int DV, bool DIFF, bool GEN = false>
+template <int DQK, int DV, bool DIFF, bool GEN = false, bool KV2 = false>
 static cudaError_t launch_one(const PrefillMaps& maps, const PrefillParams& p, const RowMap& rows, int nunits,
                               cudaStream_t stream) {
-  using C = PrefillCfg<DQK, DV, DIFF>;
-  auto kern = prefill_kernel<DQK, DV, DIFF, GEN>;
+  using C = PrefillCfg<DQK, DV, DIFF, KV2>;
+  auto kern = prefill_kernel<DQK, DV, DIFF, GEN, KV2>;
   static bool attr_set = false;  // per process; the attribute is per function
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
@@ -877,25 +906,20 @@ cudaError_t launch_prefill(const PrefillMaps& maps, const PrefillParams& p, cons
     return cudaErrorInvalidValue;
   }
   const bool gen = p.kind == kMaskGlobal || rows.mul != 1 || rows.off != 0 || rows.n != p.N;
+  const bool kv2 = p.mode == kModeKvPairs;
+  if (kv2 && !(dqk == 64 && dv == 64)) return cudaErrorInvalidValue;  // the host picks it at d = 64 only
   if (gen) {
     if (dqk == 128 && dv == 128) return launch_one<128, 128, false, true>(maps, p, rows, nunits, stream);
-    if (dqk == 64 && dv == 64) return launch_one<64, 64, false, true>(maps, p, rows, nunits, stream);
+    if (dqk == 64 && dv == 64)
+      return kv2 ? launch_one<64, 64, false, true, true>(maps, p, rows, nunits, stream)
+                 : launch_one<64, 64, false, true>(maps, p, rows, nunits, stream);
     return cudaErrorInvalidValue;
   }
   if (dqk == 128 && dv == 128) return launch_one<128, 128, false>(maps, p, rows, nunits, stream);
-  if (dqk == 64 && dv == 64) return launch_one<64, 64, false>(maps, p, rows, nunits, stream);
+  if (dqk == 64 && dv == 64)
+    return kv2 ? launch_one<64, 64, false, false, true>(maps, p, rows, nunits, stream)
+               : launch_one<64, 64, false>(maps, p, rows, nunits, stream);
   return cudaErrorInvalidValue;
-}
-
-int prefill_smem_bytes(int dqk, int dv, bool diff) {
-  if (diff) {
-    if (dqk == 64 && dv == 128) return PrefillCfg<64, 128, true>::kSmemBytes;
-    if (dqk == 64 && dv == 64) return PrefillCfg<64, 64, true>::kSmemBytes;
-    return -1;
-  }
-  if (dqk == 128 && dv == 128) return PrefillCfg<128, 128, false>::kSmemBytes;
-  if (dqk == 64 && dv == 64) return PrefillCfg<64, 64, false>::kSmemBytes;
-  return -1;
 }
 
 }  // namespace swa
