@@ -328,6 +328,17 @@ def diff_decode_workload(rank, w):
     return w, g, kv + qo + new + 4 * w.Hq, T
 
 
+def prefill_kernel_name(w) -> str:
+    """The prefill kernel instantiation a workload runs (for the roofline label)."""
+    if w.kind == "swa_bwd":
+        return f"bwd_dkdv_kernel<{w.d}> + bwd_dq_kernel<{w.d}>"
+    if w.kind == "diff":
+        return f"prefill_kernel<{w.d},{w.dv_},diff>"
+    gen = ",global" if w.kind == "global" else (",row views" if w.kind == "dilated" else "")
+    pairs = ",kv pairs" if (w.Hq // w.Hkv) % 2 == 1 and w.Hq % 2 == 0 and w.d == 64 else ""
+    return f"prefill_kernel<{w.d},{w.d}{gen}{pairs}>"
+
+
 def measure_ours(args, rank, world, peaks, peak_src, dist):
     import torch
 
@@ -375,7 +386,7 @@ def measure_ours(args, rank, world, peaks, peak_src, dist):
                      "frac": round(achieved / peak, 4), "traffic": traffic,
                      "peak_source": f"{peak_src} bf16 burst (MEASURED_PEAKS.json)" if peak_src == "measured"
                      else "fallback 1.59 PFLOP/s",
-                     "kernel": "prefill_kernel<128,128,false>"},
+                     "kernel": prefill_kernel_name(w)},
         "clocks": clk,
         "gpu_launches": args.steps,
     }
