@@ -8,7 +8,8 @@
  *
  * Every function follows the definitions on these pages:
  *   [CS] "Attention Variants Compared" (cheatsheet): the code of swa_mask and
- *        strided_mask, the task table (count_nonmasked, tiled_softmax_dot).
+ *        strided_mask, and its table of helper functions (count_nonmasked,
+ *        tiled_softmax_dot).
  *   [SW] "Learn: Sparse & Sliding-Window Attention": section 3 "The math"
  *        (A = softmax(QK^T/sqrt(d_k) + log M) V, log M in {0, -inf}, dense
  *        causal M_ij = 1[j <= i], band M_ij = 1[i-w < j <= i]); section 3b

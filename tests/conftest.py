@@ -14,7 +14,7 @@ def pytest_configure(config):
 
 def pytest_collection_modifyitems(config, items):
     """GPU tests are skipped, not failed, on a machine without a GPU when the
-    caller asked for everything; `-m gpu` on a GPU machine runs them."""
+    caller asked for everything; `-m gpu` on a machine with a CUDA device runs them."""
     try:
         import torch
 
