@@ -391,10 +391,25 @@ def measure_ours(args, rank, world, peaks, peak_src, dist):
         "gpu_launches": args.steps,
     }
     if not args.no_e2e and out is not None:  # the backward workload has no single output to copy back
-        res["e2e"] = measure_e2e(call, ins, out, flops, stream)
+        res["e2e"] = whole_job_e2e(measure_e2e(call, ins, out, flops, stream), flops, world, dist, "cuda")
     if not args.no_variants and args.only is None:
         res["variants"] = measure_variants(args, rank, peaks, flush, stream)
     return res
+
+
+def whole_job_e2e(e2e, flops, world, dist, device="cpu"):
+    """A rank's end-to-end record turned whole-job: the slowest rank's step
+    time, every rank's work and copied bytes (weak scaling). Every rank calls
+    it, so every rank takes part in the one collective."""
+    t = max_over_ranks(e2e["ms_raw"], dist, device)
+    value, tmax = aggregate([t] * world, flops)
+    out = dict(e2e)
+    out.pop("ms_raw")
+    out["value"] = round(value / 1e12, 3)
+    out["ms_per_step"] = round(tmax, 4)
+    out["h2d_bytes_per_step"] = e2e["h2d_bytes_per_step"] * world
+    out["d2h_bytes_per_step"] = e2e["d2h_bytes_per_step"] * world
+    return out
 
 
 def measure_e2e(call, ins, out, flops, stream, steps=8):
@@ -445,7 +460,8 @@ def measure_e2e(call, ins, out, flops, stream, steps=8):
     torch.cuda.synchronize()
     ms = a.elapsed_time(z) / steps
     return {"value": round(flops / (ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s", "ms_per_step": round(ms, 4),
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "pipelined": "2 buffer sets, 3 streams"}
+            "ms_raw": ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "pipelined": "2 buffer sets, 3 streams"}
 
 
 def measure_decode_only(args, rank, world, peaks, flush, stream, name):

@@ -30,7 +30,11 @@ def _worker(rank, world, port, q):
         ms = 1.0 + rank  # rank 1 is the slow one
         t = bench.max_over_ranks(ms, dist)
         value, tmax = bench.aggregate([t] * world, 100.0)
-        q.put((rank, t, value, tmax, bench.shard_seed(0, rank)))
+        # the end-to-end record: rank 1 is the slow one again
+        rec = {"value": 0.0, "unit": "TFLOP/s", "ms_per_step": 0.0, "ms_raw": 4.0 + rank,
+               "h2d_bytes_per_step": 10, "d2h_bytes_per_step": 3, "pipelined": "x"}
+        e2e = bench.whole_job_e2e(rec, 1e12, world, dist)
+        q.put((rank, t, value, tmax, bench.shard_seed(0, rank), e2e))
     finally:
         dist.destroy_process_group()
 
@@ -47,9 +51,13 @@ def test_gloo_max_over_ranks_and_weak_aggregate(world):
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
-    for rank, t, value, tmax, seed in res:
+    for rank, t, value, tmax, seed, e2e in res:
         assert t == 2.0 and tmax == 2.0
         assert abs(value - world * 100.0 / 2e-3) < 1e-6
+        # whole job: every rank's work over the slowest rank's step (5 ms)
+        assert e2e["ms_per_step"] == 5.0 and abs(e2e["value"] - world * 1.0 / 5e-3) < 1e-9
+        assert e2e["h2d_bytes_per_step"] == 10 * world and e2e["d2h_bytes_per_step"] == 3 * world
+        assert "ms_raw" not in e2e
     assert len({r[4] for r in res}) == world  # each rank its own batch
 
 
@@ -59,3 +67,14 @@ def test_single_rank_needs_no_collective():
     assert bench.max_over_ranks(3.5, None) == 3.5
     v, t = bench.aggregate([2.0], 10.0)
     assert t == 2.0 and abs(v - 5000.0) < 1e-9
+
+
+def test_single_rank_e2e_record():
+    import bench
+
+    rec = {"value": 0.0, "unit": "TFLOP/s", "ms_per_step": 4.3624, "ms_raw": 4.36237,
+           "h2d_bytes_per_step": 201326592, "d2h_bytes_per_step": 134217728, "pipelined": "x"}
+    e2e = bench.whole_job_e2e(rec, 824.7e9, 1, None)
+    assert e2e["ms_per_step"] == 4.3624 and abs(e2e["value"] - round(824.7e9 / 4.36237e-3 / 1e12, 3)) < 1e-9
+    assert e2e["h2d_bytes_per_step"] == 201326592 and e2e["d2h_bytes_per_step"] == 134217728
+    assert "ms_raw" not in e2e and e2e["unit"] == "TFLOP/s"
