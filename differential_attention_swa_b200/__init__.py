@@ -18,8 +18,9 @@ import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libswa_attn.so")
+DEBUG_LIB_PATH = os.path.join(_HERE, "libswa_attn_debug.so")  # bounds-checking build (tests)
 
-OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT = range(5)
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_SCRATCH_TOO_SMALL, ERR_BOUNDS = range(7)
 MASK_WINDOW, MASK_STRIDED, MASK_CAUSAL, MASK_GLOBAL = 0, 1, 2, 3
 STRIDE_TAG = 0x40000000
 TILE = 128  # query rows and keys per tile in the prefill kernels
@@ -50,9 +51,24 @@ def library() -> ctypes.CDLL:
     global _lib
     if _lib is not None:
         return _lib
-    if not os.path.exists(LIB_PATH):
-        raise RuntimeError(f"{LIB_PATH} is missing: build it with differential_attention_swa_b200/build.py")
-    lib = ctypes.CDLL(LIB_PATH)
+    _lib = load(LIB_PATH)
+    return _lib
+
+
+def use_library(lib: ctypes.CDLL | None) -> ctypes.CDLL | None:
+    """Routes every call of this module to `lib` (for instance the
+    bounds-checking build from load(DEBUG_LIB_PATH)); None restores the
+    release library. Returns the previous one."""
+    global _lib
+    prev, _lib = _lib, lib
+    return prev
+
+
+def load(path: str) -> ctypes.CDLL:
+    """Opens a build of the library and declares its entry points."""
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with differential_attention_swa_b200/build.py")
+    lib = ctypes.CDLL(path)
     P, I, F, I64, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_int64, ctypes.c_size_t
     lib.swa_attn_fwd.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, P]
     lib.strided_attn_fwd.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, F, P]
@@ -85,13 +101,14 @@ def library() -> ctypes.CDLL:
     lib.swa_schedule.restype = I64
     lib.swa_count_nonmasked.argtypes = [I, I, I, I]
     lib.swa_count_nonmasked.restype = I64
+    lib.swa_debug_exp2.argtypes = [P, P, I64, P]
+    lib.swa_debug_exp2.restype = I
     lib.swa_last_device_error.argtypes = [P]
     lib.swa_status_string.argtypes = [I]
     lib.swa_status_string.restype = ctypes.c_char_p
     for name in ("swa_attn_fwd", "strided_attn_fwd", "diff_attn_fwd", "swa_decode_step", "swa_prefill_debug",
                  "swa_last_device_error"):
         getattr(lib, name).restype = I
-    _lib = lib
     return lib
 
 
@@ -352,6 +369,17 @@ def prefill_debug(kind: int, q, k, v, window: int, stride: int = 0, scale: float
                                      int(window), int(stride), float(scale), ctypes.byref(dbg), _stream(stream))
     _raise(st, "swa_prefill_debug")
     return out, cells, tiles, ntiles
+
+
+def debug_exp2(x, out=None, stream=None):
+    """2^x through the prefill kernels' FMA-pipe exponential (a debug entry:
+    the differential kernel evaluates part of its exponentials this way)."""
+    _check(x, "x", dtype=torch.float32)
+    out = torch.empty_like(x) if out is None else out
+    _check(out, "out", dtype=torch.float32)
+    st = library().swa_debug_exp2(_ptr(x), _ptr(out), x.numel(), _stream(stream))
+    _raise(st, "swa_debug_exp2")
+    return out
 
 
 def schedule(kind: int, N: int, W: int, stride: int = 0, Bq: int = TILE, Bk: int = TILE):

@@ -5,10 +5,13 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <set>
+#include <utility>
 
 #include "../../include/swa_attn.h"
 #include "internal.h"
@@ -49,17 +52,18 @@ bool encode_rows(CUtensorMap* m, const void* base, int d, int64_t rows, int64_t 
   return r == CUDA_SUCCESS;
 }
 
-// Streaming multiprocessors of the current device (cached per device).
+// Streaming multiprocessors of the current device (cached per device; host
+// threads may race to fill an entry, all with the same value).
 int sm_count() {
-  static int counts[64] = {0};
+  static std::atomic<int> counts[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return -1;
-  if (counts[dev] == 0) {
-    int n = 0;
+  int n = counts[dev].load(std::memory_order_relaxed);
+  if (n == 0) {
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
-    counts[dev] = n;
+    counts[dev].store(n, std::memory_order_relaxed);
   }
-  return counts[dev];
+  return n;
 }
 
 bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -161,6 +165,20 @@ swa_status_t run_prefill(int kind, bool diff, const void* q, const void* k, cons
 }
 
 }  // namespace
+
+cudaError_t ensure_dynamic_smem(const void* kernel, int bytes) {
+  static std::mutex mu;
+  static std::set<std::pair<const void*, int>> done;  // (kernel, device)
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  if (done.count({kernel, dev})) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) return e;
+  done.insert({kernel, dev});
+  return cudaSuccess;
+}
 
 int* device_error_ptr() {
   static int* ptrs[64] = {nullptr};
@@ -320,7 +338,7 @@ swa_status_t swa_prefill_debug(int kind, const void* q, const void* k, const voi
 }
 
 size_t swa_decode_workspace_bytes(int B, int Hq, int Hkv, int d, int W) {
-  if (B < 1 || Hq < 1 || Hkv < 1 || W < 1 || Hq % Hkv != 0 || (d != 64 && d != 128)) return 0;
+  if (B < 1 || Hq < 1 || Hkv < 1 || W < 1 || W > (1 << 30) || Hq % Hkv != 0 || (d != 64 && d != 128)) return 0;
   return decode_partial_bytes(B, Hq, Hkv, d, W);
 }
 
@@ -339,12 +357,14 @@ swa_status_t swa_sink_decode_step(const void* q, const void* k_new, const void* 
 }
 
 size_t swa_sink_decode_workspace_bytes(int B, int Hq, int Hkv, int d, int n_sink, int W) {
-  if (B < 1 || Hq < 1 || Hkv < 1 || W < 1 || n_sink < 0 || Hq % Hkv != 0 || (d != 64 && d != 128)) return 0;
+  if (B < 1 || Hq < 1 || Hkv < 1 || W < 1 || n_sink < 0 || (int64_t)n_sink + W > (1 << 30) || Hq % Hkv != 0 ||
+      (d != 64 && d != 128))
+    return 0;
   return decode_partial_bytes(B, Hq, Hkv, d, n_sink + W);
 }
 
 size_t swa_diff_decode_workspace_bytes(int B, int Hq, int Hkv, int d_qk, int d_v, int W) {
-  if (B < 1 || Hq < 1 || Hkv < 1 || W < 1 || Hq % Hkv != 0 || d_qk != 64 || d_v != 128) return 0;
+  if (B < 1 || Hq < 1 || Hkv < 1 || W < 1 || W > (1 << 30) || Hq % Hkv != 0 || d_qk != 64 || d_v != 128) return 0;
   return diff_decode_partial_bytes(B, Hq, Hkv, W);
 }
 
@@ -426,6 +446,14 @@ int64_t swa_count_nonmasked(int kind, int N, int W, int stride) {
   return count_attended(kind, N, W, stride);
 }
 
+swa_status_t swa_debug_exp2(const float* x, float* y, int64_t n, void* stream) {
+  if (n < 0) return SWA_ERR_INVALID_ARG;
+  if (n == 0) return SWA_OK;
+  if (x == nullptr || y == nullptr || (reinterpret_cast<uintptr_t>(x) & 3u) || (reinterpret_cast<uintptr_t>(y) & 3u))
+    return SWA_ERR_INVALID_ARG;
+  return launch_exp2_fma2(x, y, n, static_cast<cudaStream_t>(stream)) == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
+}
+
 swa_status_t swa_last_device_error(void* stream) {
   int err = 0;
   if (read_and_clear_device_error(static_cast<cudaStream_t>(stream), &err) != 0) return SWA_ERR_CUDA;
@@ -440,6 +468,7 @@ const char* swa_status_string(swa_status_t s) {
     case SWA_ERR_CUDA: return "CUDA error";
     case SWA_ERR_TIMEOUT: return "in-kernel wait timed out";
     case SWA_ERR_SCRATCH_TOO_SMALL: return "sizes need more scratch than the static decode array holds";
+    case SWA_ERR_BOUNDS: return "debug bounds check failed: an index fell outside its tensor";
   }
   return "unknown status";
 }

@@ -114,7 +114,7 @@ __global__ void __launch_bounds__(128) bwd_prep_kernel(const BwdParams p) {
         d = fmaf(__uint_as_float(wa[e] & 0xffff0000u), __uint_as_float(wb[e] & 0xffff0000u), d);
       }
     }
-    l2 = p.lse[row] * 1.4426950408889634f;
+    if (SWA_IN(row, 0, (int64_t)p.B * p.Hq * p.N, p.err_flag)) l2 = p.lse[row] * 1.4426950408889634f;
   }
   p.dd[r] = d;
   p.lse2[r] = l2;
@@ -202,8 +202,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     // ------------------------------------------------------ producer ---
     if (lane == 0) {
       const int zkv = b * p.Hkv + hkv;
+      const int krows = STRIDE ? (p.N + p.S - 1) / p.S : p.N;  // rows of the stride view, or of K/V
+      (void)krows;
       mbar_arrive_expect_tx(bar(BwdBar::kFixed), 2 * C::kTile);
       for (int bx = 0; bx < D / 64; ++bx) {
+        if (!SWA_TMA_IN(bx * 64, D, kt * kBT, krows, zkv, p.B * p.Hkv, p.err_flag)) continue;
         tma_load_3d(sbase + C::kOffA + bx * 16384, STRIDE ? &tm_ks : &tm_k, bar(BwdBar::kFixed), bx * 64, kt * kBT,
                     zkv);
         tma_load_3d(sbase + C::kOffB + bx * 16384, STRIDE ? &tm_vs : &tm_v, bar(BwdBar::kFixed), bx * 64, kt * kBT,
@@ -221,12 +224,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const uint32_t base = sbase + C::kOffStages + st * C::kStage;
         mbar_arrive_expect_tx(bar(BwdBar::kFull + st), 2 * C::kTile + 2 * kBT * 4);
         for (int bx = 0; bx < D / 64; ++bx) {
+          if (!SWA_TMA_IN(bx * 64, D, qt * kBT, p.N, zq, p.B * p.Hq, p.err_flag)) continue;
           tma_load_3d(base + bx * 16384, &tm_q, bar(BwdBar::kFull + st), bx * 64, qt * kBT, zq);
           tma_load_3d(base + C::kTile + bx * 16384, &tm_do, bar(BwdBar::kFull + st), bx * 64, qt * kBT, zq);
         }
         const int64_t rt = (int64_t)zq * p.npad + qt * kBT;
-        bulk_load(base + 2 * C::kTile, p.lse2 + rt, kBT * 4, bar(BwdBar::kFull + st));
-        bulk_load(base + 2 * C::kTile + kBT * 4, p.dd + rt, kBT * 4, bar(BwdBar::kFull + st));
+        if (SWA_IN(rt, 0, (int64_t)p.B * p.Hq * p.npad - kBT + 1, p.err_flag)) {
+          bulk_load(base + 2 * C::kTile, p.lse2 + rt, kBT * 4, bar(BwdBar::kFull + st));
+          bulk_load(base + 2 * C::kTile + kBT * 4, p.dd + rt, kBT * 4, bar(BwdBar::kFull + st));
+        }
         issued[st] = use + 1;
       }
       if (*abort_flag) {  // drain: every copy issued lands before the CTA may exit
@@ -361,7 +367,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tc_fence_after();
         const int64_t row = ((int64_t)(b * p.Hkv + hkv) * p.nspad + key) * D;
 #pragma unroll 1
-        for (int c = 0; c < D; c += 32) {
+        for (int c = 0; c < D && SWA_IN(row, 0, (int64_t)p.B * p.Hkv * p.nspad * D - D + 1, p.err_flag); c += 32) {
           float a[32], g[32];
           tmem_ld32(tmem + lane_addr + C::kColAcc + c, a);
           tmem_ld32(tmem + lane_addr + C::kColAcc + D + c, g);
@@ -380,19 +386,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       // a stride key also gets the stride pass's partials before the one rounding
       const bool add = MODE == 1 && key < p.N && key % p.S == 0;
       const int64_t srow = ((int64_t)(b * p.Hkv + hkv) * p.nspad + (add ? key / p.S : 0)) * D;
+      const bool in_rows = key >= p.N || SWA_IN(row, 0, (int64_t)p.B * p.Hkv * p.N * D - D + 1, p.err_flag);
+      const bool in_srow = !add || SWA_IN(srow, 0, (int64_t)p.B * p.Hkv * p.nspad * D - D + 1, p.err_flag);
 #pragma unroll 1
       for (int c = 0; c < D; c += 32) {
         float a[32], g[32];
         tmem_ld32(tmem + lane_addr + C::kColAcc + c, a);
         tmem_ld32(tmem + lane_addr + C::kColAcc + D + c, g);
-        if (add) {
+        if (add && in_srow) {
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
             a[e] += p.sdv[srow + c + e];
             g[e] += p.sdk[srow + c + e];
           }
         }
-        if (key < p.N) {
+        if (key < p.N && in_rows) {
 #pragma unroll
           for (int e = 0; e < 32; e += 8) {
             st_global_v4(dv + c + e, pack_bf16(a[e], a[e + 1]), pack_bf16(a[e + 2], a[e + 3]),
@@ -476,6 +484,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const int zq = b * p.Hq + hq, zkv = b * p.Hkv + hkv;
       mbar_arrive_expect_tx(bar(BwdBar::kFixed), 2 * C::kTile);
       for (int bx = 0; bx < D / 64; ++bx) {
+        if (!SWA_TMA_IN(bx * 64, D, qt * kBT, p.N, zq, p.B * p.Hq, p.err_flag)) continue;
         tma_load_3d(sbase + C::kOffA + bx * 16384, &tm_q, bar(BwdBar::kFixed), bx * 64, qt * kBT, zq);
         tma_load_3d(sbase + C::kOffB + bx * 16384, &tm_do, bar(BwdBar::kFixed), bx * 64, qt * kBT, zq);
       }
@@ -490,7 +499,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const int row = (strided ? s : kt_lo + (s - nst)) * kBT;
         const uint32_t base = sbase + C::kOffStages + st * C::kStage;
         mbar_arrive_expect_tx(bar(BwdBar::kFull + st), 2 * C::kTile);
+        const int krows = strided ? (p.N + p.S - 1) / p.S : p.N;
+        (void)krows;
         for (int bx = 0; bx < D / 64; ++bx) {
+          if (!SWA_TMA_IN(bx * 64, D, row, krows, zkv, p.B * p.Hkv, p.err_flag)) continue;
           tma_load_3d(base + bx * 16384, strided ? &tm_ks : &tm_k, bar(BwdBar::kFull + st), bx * 64, row, zkv);
           tma_load_3d(base + C::kTile + bx * 16384, strided ? &tm_vs : &tm_v, bar(BwdBar::kFull + st), bx * 64, row,
                       zkv);
@@ -564,7 +576,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t lane_addr = static_cast<uint32_t>(qw * 32) << 16;
     const float sl2 = p.scale_log2;
     const int64_t rt = (int64_t)(b * p.Hq + hq) * p.npad + i;  // padded: always in bounds
-    const float lse2 = p.lse2[rt], dd = p.dd[rt];
+    const bool rt_ok = SWA_IN(rt, 0, (int64_t)p.B * p.Hq * p.npad, p.err_flag);
+    const float lse2 = rt_ok ? p.lse2[rt] : 0.f, dd = rt_ok ? p.dd[rt] : 0.f;
     bool ok = true;
     for (int s = 0; s < nsteps; ++s) {
       const bool strided = SM && s < nst;
@@ -616,7 +629,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       for (int c = 0; c < D; c += 32) {
         float a[32];
         tmem_ld32(tmem + lane_addr + C::kColAcc + c, a);
-        if (i < p.N) {
+        if (i < p.N && SWA_IN((int64_t)(b * p.Hq + hq) * p.N + i, 0, (int64_t)p.B * p.Hq * p.N, p.err_flag)) {
 #pragma unroll
           for (int e = 0; e < 32; e += 8)
             st_global_v4(dq + c + e, pack_bf16(a[e] * p.scale, a[e + 1] * p.scale),
@@ -640,16 +653,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 template <int D>
 cudaError_t launch_bwd_d(const BwdMaps& m, const BwdParams& p, cudaStream_t stream) {
   using C = BwdCfg<D>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    const cudaFuncAttribute a = cudaFuncAttributeMaxDynamicSharedMemorySize;
-    cudaError_t e = cudaFuncSetAttribute(bwd_dkdv_kernel<D, 0>, a, C::kSmemBytes);
-    if (e == cudaSuccess) e = cudaFuncSetAttribute(bwd_dkdv_kernel<D, 1>, a, C::kSmemBytes);
-    if (e == cudaSuccess) e = cudaFuncSetAttribute(bwd_dkdv_kernel<D, 2>, a, C::kSmemBytes);
-    if (e == cudaSuccess) e = cudaFuncSetAttribute(bwd_dq_kernel<D, false>, a, C::kSmemBytes);
-    if (e == cudaSuccess) e = cudaFuncSetAttribute(bwd_dq_kernel<D, true>, a, C::kSmemBytes);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
+  {
+    const void* kernels[5] = {reinterpret_cast<const void*>(bwd_dkdv_kernel<D, 0>),
+                              reinterpret_cast<const void*>(bwd_dkdv_kernel<D, 1>),
+                              reinterpret_cast<const void*>(bwd_dkdv_kernel<D, 2>),
+                              reinterpret_cast<const void*>(bwd_dq_kernel<D, false>),
+                              reinterpret_cast<const void*>(bwd_dq_kernel<D, true>)};
+    for (const void* k : kernels) {
+      const cudaError_t e = ensure_dynamic_smem(k, C::kSmemBytes);
+      if (e != cudaSuccess) return e;
+    }
   }
   const int64_t rows = (int64_t)p.B * p.Hq * p.npad;
   bwd_prep_kernel<D><<<(unsigned)((rows + 127) / 128), 128, 0, stream>>>(p);

@@ -120,7 +120,7 @@ __global__ void __launch_bounds__(kDecThreads, dec_min_blocks<G>())
 #pragma unroll
     for (int u = 0; u < kDecUnroll; ++u) {
       slot[u] = base + (u * 4 + warp) * RPW + rr;
-      if (slot[u] < s1) {
+      if (slot[u] < s1 && SWA_IN(slot[u], 0, p.n_sink + p.W, p.err_flag)) {
         if (slot[u] == new_slot) {
           kr[u] = *reinterpret_cast<const uint4*>(kn + 8 * e);
           vr[u] = *reinterpret_cast<const uint4*>(vn + 8 * e);
@@ -221,7 +221,9 @@ __global__ void __launch_bounds__(kDecThreads, dec_min_blocks<G>())
       L += sm_l[w][g] * a;
       O += sm_acc[w][g][c] * a;
     }
-    float* rec = p.partial + ((int64_t)(b * p.Hq + hkv * G + g) * p.nsplit + split) * partial_stride(D);
+    const int64_t ri = (int64_t)(b * p.Hq + hkv * G + g) * p.nsplit + split;
+    if (!SWA_IN(ri, 0, (int64_t)p.B * p.Hq * p.nsplit, p.err_flag)) continue;
+    float* rec = p.partial + ri * partial_stride(D);
     if (c == 0) {
       rec[0] = M;
       rec[1] = L;
@@ -236,6 +238,7 @@ __global__ void __launch_bounds__(D)
   grid_dependency_wait();  // the split kernel's partials are complete and visible
   const int bh = blockIdx.x;  // b * Hq + hq
   const int c = threadIdx.x;
+  if (!SWA_IN(bh, 0, p.B * p.Hq, p.err_flag)) return;
   const float* recs = p.partial + (int64_t)bh * p.nsplit * partial_stride(D);
   float M = -INFINITY;
   for (int s = 0; s < p.nsplit; ++s) M = fmaxf(M, recs[s * partial_stride(D)]);
@@ -304,6 +307,8 @@ static cudaError_t launch_g(DecodeParams p, cudaStream_t stream) {
 
 cudaError_t launch_decode(const DecodeParams& p0, cudaStream_t stream) {
   DecodeParams p = p0;
+  p.err_flag = device_error_ptr();
+  if (p.err_flag == nullptr) return cudaErrorUnknown;
   p.nsplit = decode_nsplit(p.B, p.Hkv, p.n_sink + p.W);
   p.chunk = decode_chunk(p.B, p.Hkv, p.n_sink + p.W);
   if (p.d == 128) {
@@ -369,7 +374,7 @@ extern "C" swa_status_t swa_decode_step_static(const void* q, const void* k_new,
   if (!a16(q) || !a16(k_new) || !a16(v_new) || !a16(k_cache) || !a16(v_cache) || !a16(o) || pos == nullptr ||
       (reinterpret_cast<uintptr_t>(pos) & 3u))
     return SWA_ERR_INVALID_ARG;
-  if (B < 1 || Hq < 1 || Hkv < 1 || W < 1 || Hq % Hkv != 0) return SWA_ERR_INVALID_ARG;
+  if (B < 1 || Hq < 1 || Hkv < 1 || W < 1 || W > (1 << 30) || Hq % Hkv != 0) return SWA_ERR_INVALID_ARG;
   if (!(scale > 0.f) || !isfinite(scale)) return SWA_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return SWA_ERR_UNSUPPORTED;
   const int G = Hq / Hkv;

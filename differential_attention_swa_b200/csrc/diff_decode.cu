@@ -136,7 +136,7 @@ __global__ void __launch_bounds__(kDdThreads, dd_min_blocks<G>()) diff_decode_sp
 #pragma unroll
     for (int u = 0; u < kDdUnroll; ++u) {
       slot[u] = base + (u * 4 + warp) * kRpw + rr;
-      if (slot[u] < s1) {
+      if (slot[u] < s1 && SWA_IN(slot[u], 0, p.W, p.err_flag)) {
         const int64_t kofs = (row0 + slot[u]) * kDk + kc8;
         const int64_t vofs = (row0 + slot[u]) * kDv + 8 * e;
         if (slot[u] == new_slot) {
@@ -248,7 +248,9 @@ __global__ void __launch_bounds__(kDdThreads, dd_min_blocks<G>()) diff_decode_sp
       L += sm_ml[w][g][2 * mp + 1] * a;
       O += sm_acc[w][g][mp][c] * a;
     }
-    float* rec = p.partial + ((int64_t)(b * p.Hq + hkv * G + g) * p.nsplit + split) * diff_partial_stride();
+    const int64_t ri = (int64_t)(b * p.Hq + hkv * G + g) * p.nsplit + split;
+    if (!SWA_IN(ri, 0, (int64_t)p.B * p.Hq * p.nsplit, p.err_flag)) continue;
+    float* rec = p.partial + ri * diff_partial_stride();
     if (c == 0) {
       rec[2 * mp] = M;
       rec[2 * mp + 1] = L;
@@ -261,6 +263,7 @@ __global__ void __launch_bounds__(kDv) diff_decode_combine_kernel(const DiffDeco
   grid_dependency_wait();  // the split kernel's partials are complete and visible
   const int bh = blockIdx.x;  // b * Hq + hq
   const int c = threadIdx.x;
+  if (!SWA_IN(bh, 0, p.B * p.Hq, p.err_flag)) return;
   const float* recs = p.partial + (int64_t)bh * p.nsplit * diff_partial_stride();
   float M1 = -INFINITY, M2 = -INFINITY;
   for (int s = 0; s < p.nsplit; ++s) {
@@ -332,6 +335,8 @@ size_t diff_decode_partial_bytes(int B, int Hq, int Hkv, int W) {
 
 cudaError_t launch_diff_decode(const DiffDecodeParams& p0, cudaStream_t stream) {
   DiffDecodeParams p = p0;
+  p.err_flag = device_error_ptr();
+  if (p.err_flag == nullptr) return cudaErrorUnknown;
   p.nsplit = diff_decode_nsplit(p.B, p.Hkv, p.W);
   p.chunk = ((p.W + p.nsplit - 1) / p.nsplit + 63) / 64 * 64;
   switch (p.G) {

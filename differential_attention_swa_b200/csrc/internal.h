@@ -84,6 +84,7 @@ struct DecodeParams {
   int n_sink;  // attention-sink slots ahead of the W window slots (0: none)
   int nsplit, chunk;
   float scale_log2;
+  int* err_flag;  // device error word (bounds-checking debug builds report here)
 };
 
 // Differential decode: two maps (q1/K1, q2/K2) over one rolling window and
@@ -97,6 +98,7 @@ struct DiffDecodeParams {
   int B, Hq, Hkv, W, G;
   int nsplit, chunk;
   float scale_log2;
+  int* err_flag;
 };
 size_t diff_decode_partial_bytes(int B, int Hq, int Hkv, int W);
 cudaError_t launch_diff_decode(const DiffDecodeParams& p, cudaStream_t stream);
@@ -104,6 +106,14 @@ cudaError_t launch_diff_decode(const DiffDecodeParams& p, cudaStream_t stream);
 int decode_nsplit(int B, int Hkv, int W);
 size_t decode_partial_bytes(int B, int Hq, int Hkv, int d, int slots);
 cudaError_t launch_decode(const DecodeParams& p, cudaStream_t stream);
+
+// Raises a kernel's dynamic shared-memory limit to `bytes` on the current
+// device, once per (kernel, device): function attributes live in each
+// device's context. Safe to call from several host threads.
+cudaError_t ensure_dynamic_smem(const void* kernel, int bytes);
+
+// y[i] = 2^x[i] through the prefill kernels' FMA-pipe exponential.
+cudaError_t launch_exp2_fma2(const float* x, float* y, int64_t n, cudaStream_t stream);
 
 int* device_error_ptr();
 int read_and_clear_device_error(cudaStream_t stream, int* err);

@@ -74,7 +74,7 @@ constexpr float kRescaleTau = 8.0f;
 //   POLY  of every 8 pairs of exponentials, how many are evaluated on the FMA
 //         pipe (exp2_fma2) instead of the MUFU unit.
 // d = 128 window kernels: one buffer (the MMA cost dominates); differential
-// (d_qk = 64, d_v = 128): one buffer, 2 of 8 pairs on the FMA pipe; d = 64
+// (d_qk = 64, d_v = 128): one buffer, 1 of 8 pairs on the FMA pipe; d = 64
 // window and strided kernels (short units, MUFU-bound): two halves.
 template <int DQK, int DV, bool DIFF>
 struct PrefillTune {
@@ -86,7 +86,7 @@ struct PrefillTune {
 #ifdef SWA_POLY_PAIRS_PER_8
   static constexpr int POLY = SWA_POLY_PAIRS_PER_8;
 #else
-  static constexpr int POLY = DIFF ? 2 : 0;
+  static constexpr int POLY = DIFF ? 1 : 0;
 #endif
   static_assert(NH == 1 || NH == 2, "one or two score buffers per tile");
 };
@@ -368,8 +368,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!un.valid[t]) continue;
           const CUtensorMap* m = (DIFF && t == 1) ? &tm_q2 : &tm_q;
           for (int bx = 0; bx < DQK / 64; ++bx)
-            tma_load_3d(sbase + C::kOffQ + t * C::kQBytes + bx * 16384, m, bar(BarLayout::kQ), bx * 64,
-                        un.qt[t] * BM, un.b * p.Hq + un.hq[t]);
+            if (SWA_TMA_IN(bx * 64, DQK, un.qt[t] * BM, p.N, un.b * p.Hq + un.hq[t], p.B * p.Hq, p.err_flag))
+              tma_load_3d(sbase + C::kOffQ + t * C::kQBytes + bx * 16384, m, bar(BarLayout::kQ), bx * 64,
+                          un.qt[t] * BM, un.b * p.Hq + un.hq[t]);
         }
         ++nq_ld;
         const int zkv = un.b * p.Hkv + un.hkv;
@@ -377,6 +378,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int u = 0; u < it.n && ok; ++u) {
           const bool st = item_is_stride(it, u);
           const int row = item_tile(it, u) * BN;
+          // rows of the view the tile comes from: the stride view holds
+          // ceil(N / S) rows, the global keys' view is K/V itself
+          const int vrows = (st && p.kind == kMaskStrided) ? (p.N + p.S - 1) / p.S : p.N;
+          (void)vrows;
           {  // K (or K1 and K2)
             const int slot = L % C::kSlots, use = L / C::kSlots;
             ++L;
@@ -390,15 +395,18 @@ __global__ void __launch_bounds__(kThreads, 1)
               const uint32_t dst = sbase + C::kOffSlots + slot * C::kSlot;
               const CUtensorMap* m = st ? &tm_ks : &tm_k;
               for (int bx = 0; bx < DQK / 64; ++bx)
-                tma_load_3d(dst + bx * 16384, m, bar(BarLayout::kFull + slot), bx * 64, row, zkv);
+                if (SWA_TMA_IN(bx * 64, DQK, row, vrows, zkv, p.B * p.Hkv, p.err_flag))
+                  tma_load_3d(dst + bx * 16384, m, bar(BarLayout::kFull + slot), bx * 64, row, zkv);
               if (DIFF)
                 for (int bx = 0; bx < DQK / 64; ++bx)
-                  tma_load_3d(dst + BN * DQK * 2 + bx * 16384, &tm_k2, bar(BarLayout::kFull + slot), bx * 64,
-                              row, zkv);
+                  if (SWA_TMA_IN(bx * 64, DQK, row, vrows, zkv, p.B * p.Hkv, p.err_flag))
+                    tma_load_3d(dst + BN * DQK * 2 + bx * 16384, &tm_k2, bar(BarLayout::kFull + slot), bx * 64,
+                                row, zkv);
               if (KV2)  // sub 1's KV head
                 for (int bx = 0; bx < DQK / 64; ++bx)
-                  tma_load_3d(dst + BN * DQK * 2 + bx * 16384, m, bar(BarLayout::kFull + slot), bx * 64, row,
-                              zkv1);
+                  if (SWA_TMA_IN(bx * 64, DQK, row, vrows, zkv1, p.B * p.Hkv, p.err_flag))
+                    tma_load_3d(dst + BN * DQK * 2 + bx * 16384, m, bar(BarLayout::kFull + slot), bx * 64, row,
+                                zkv1);
               issued[slot] = use + 1;
             }
           }
@@ -414,10 +422,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t dst = sbase + C::kOffSlots + slot * C::kSlot;
             const CUtensorMap* m = st ? &tm_vs : &tm_v;
             for (int bx = 0; bx < DV / 64; ++bx)
-              tma_load_3d(dst + bx * 16384, m, bar(BarLayout::kFull + slot), bx * 64, row, zkv);
+              if (SWA_TMA_IN(bx * 64, DV, row, vrows, zkv, p.B * p.Hkv, p.err_flag))
+                tma_load_3d(dst + bx * 16384, m, bar(BarLayout::kFull + slot), bx * 64, row, zkv);
             if (KV2)
               for (int bx = 0; bx < DV / 64; ++bx)
-                tma_load_3d(dst + BN * DV * 2 + bx * 16384, m, bar(BarLayout::kFull + slot), bx * 64, row, zkv1);
+                if (SWA_TMA_IN(bx * 64, DV, row, vrows, zkv1, p.B * p.Hkv, p.err_flag))
+                  tma_load_3d(dst + BN * DV * 2 + bx * 16384, m, bar(BarLayout::kFull + slot), bx * 64, row, zkv1);
             issued[slot] = use + 1;
           }
         }
@@ -562,8 +572,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (h == 0 && lane == 0 && !drain) {
             const int tag = item_is_stride(it, u) ? (kStrideTag | item_tile(it, u)) : item_tile(it, u);
-            if (in0 && sm0.dbg_row >= 0 && sm0.kcount < p.dbg_cap) p.dbg_tiles[sm0.dbg_row * p.dbg_cap + sm0.kcount] = tag;
-            if (in1 && sm1.dbg_row >= 0 && sm1.kcount < p.dbg_cap) p.dbg_tiles[sm1.dbg_row * p.dbg_cap + sm1.kcount] = tag;
+            const int64_t ndbg = (int64_t)p.B * p.Hq * p.nq;
+            (void)ndbg;
+            if (in0 && sm0.dbg_row >= 0 && sm0.kcount < p.dbg_cap && SWA_IN(sm0.dbg_row, 0, ndbg, p.err_flag))
+              p.dbg_tiles[sm0.dbg_row * p.dbg_cap + sm0.kcount] = tag;
+            if (in1 && sm1.dbg_row >= 0 && sm1.kcount < p.dbg_cap && SWA_IN(sm1.dbg_row, 0, ndbg, p.err_flag))
+              p.dbg_tiles[sm1.dbg_row * p.dbg_cap + sm1.kcount] = tag;
           }
           if (h == 0) {
             sm0.kcount += in0;
@@ -603,8 +617,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (lane == 0) record_timeout(abort_flag, p.err_flag);
           break;
         }
-        if (lane == 0 && sm0.dbg_row >= 0) p.dbg_ntiles[sm0.dbg_row] = sm0.kcount;
-        if (lane == 0 && sm1.dbg_row >= 0) p.dbg_ntiles[sm1.dbg_row] = sm1.kcount;
+        if (lane == 0 && sm0.dbg_row >= 0 && SWA_IN(sm0.dbg_row, 0, (int64_t)p.B * p.Hq * p.nq, p.err_flag))
+          p.dbg_ntiles[sm0.dbg_row] = sm0.kcount;
+        if (lane == 0 && sm1.dbg_row >= 0 && SWA_IN(sm1.dbg_row, 0, (int64_t)p.B * p.Hq * p.nq, p.err_flag))
+          p.dbg_ntiles[sm1.dbg_row] = sm1.kcount;
         if (un.valid[0]) ++sm0.nunit;
         if (un.valid[1]) ++sm1.nunit;
       }
@@ -623,6 +639,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t o_tmem = tmem + lane_addr + (t == 0 ? C::kOCol0 : C::kOCol1);
     const int Wc = (p.kind == kMaskCausal) ? p.N : p.W;
     const float cl2 = p.scale_log2;
+    const bool want_lse = !DIFF && p.lse != nullptr;
     // Epilogue store: this warp's 32 output rows go through a 4 KB
     // shared-memory box (128-byte swizzle), 64 columns at a time, and lane 0
     // writes the box with one TMA store; rows past N are clipped by TMA.
@@ -648,7 +665,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          tma_store_3d(&tm_o, stage, 64 * h, row0, zrow);
+          // a box whose rows all lie past N is clipped whole by the TMA unit
+          if (SWA_TMA_IN(64 * h, DV, row0, p.nq * BM, zrow, p.B * p.Hq, p.err_flag))
+            tma_store_3d(&tm_o, stage, 64 * h, row0, zrow);
           bulk_commit();
         }
         used = true;
@@ -685,7 +704,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int mst = GEN ? extra_rows_below(p.kind, lo, p.S)  // extra-view rows below lo
                           : ((p.kind == kMaskStrided) ? stride_rows_below(lo, p.S) : 0);
       float m_run = -INFINITY;  // running max, log2 units (scores * scale * log2 e)
-      float l_run = 0.f;
+      float l_run = 0.f;  // sum of the bf16 weights the PV products consume
+      float l_exact = 0.f;  // sum of the unrounded weights (log-sum-exp only)
       long long cells = 0;
 
       for (int u = 0; u < it.n && ok; ++u) {
@@ -758,6 +778,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // and the row sum, MUFU ex2 for the exponential
           const float2 cl2x2 = make_float2(cl2, cl2), negm = make_float2(-msub, -msub);
           float2 rs2[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
+          float2 ex2s[2] = {{0.f, 0.f}, {0.f, 0.f}};
           uint32_t pk[BH / 2];
 #pragma unroll
           for (int j = 0; j < BH / 2; ++j) {
@@ -771,12 +792,19 @@ __global__ void __launch_bounds__(kThreads, 1)
               p0 = ex2_approx(x.x);
               p1 = ex2_approx(x.y);
             }
-            rs2[j & 3] = __fadd2_rn(rs2[j & 3], make_float2(p0, p1));
             pk[j] = pack_bf16(p0, p1);
+            // the row sum adds the bf16 values the PV product consumes, so
+            // the weights applied to V sum to one
+            rs2[j & 3] = __fadd2_rn(rs2[j & 3], unpack_bf16(pk[j]));
+            if (want_lse) ex2s[j & 1] = __fadd2_rn(ex2s[j & 1], make_float2(p0, p1));
           }
           const float2 rsum = __fadd2_rn(__fadd2_rn(rs2[0], rs2[1]), __fadd2_rn(rs2[2], rs2[3]));
           const float rs = rsum.x + rsum.y;
           l_run = l_run * alpha + rs;
+          if (want_lse) {
+            const float2 es = __fadd2_rn(ex2s[0], ex2s[1]);
+            l_exact = l_exact * alpha + (es.x + es.y);
+          }
           m_run = m_use;
 
           // P over the consumed scores: bf16 pairs, 32 columns per 64 keys
@@ -826,7 +854,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (DIFF) {
         if (t == 1) {
           // hands lambda / l2 to sub 0, which reads both accumulators
-          f2s[r] = (l_run > 0.f) ? p.lambda[hq] / l_run : 0.f;
+          const float lam = SWA_IN(hq, 0, p.Hq, p.err_flag) ? p.lambda[hq] : 0.f;
+          f2s[r] = (l_run > 0.f) ? lam / l_run : 0.f;
           tc_fence_before();
           mbar_arrive(bar(BarLayout::kX));
         } else {
@@ -858,15 +887,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         }, un.b * p.Hq + hq, qt_t * BM + qw * 32);
         tc_fence_before();
         mbar_arrive(bar(BarLayout::kOFree + t));  // O_t read: the next unit may overwrite it
-        if (p.lse && row_ok) p.lse[orow] = (m_run + __log2f(l_run)) * 0.6931471805599453f;
+        if (want_lse && row_ok && SWA_IN(orow, 0, (int64_t)p.B * p.Hq * (GEN ? rmap.n : p.N), p.err_flag))
+          p.lse[orow] = (m_run + __log2f(l_exact)) * 0.6931471805599453f;
       }
       if (p.dbg_cells && !(DIFF && t == 1)) {
         long long c = row_ok ? cells : 0;
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) c += __shfl_xor_sync(0xffffffffu, c, off);
-        if (lane == 0)
-          atomicAdd(reinterpret_cast<unsigned long long*>(p.dbg_cells + (int64_t)(un.b * p.Hq + hq) * p.nq + qt_t),
-                    static_cast<unsigned long long>(c));
+        const int64_t ci = (int64_t)(un.b * p.Hq + hq) * p.nq + qt_t;
+        if (lane == 0 && SWA_IN(ci, 0, (int64_t)p.B * p.Hq * p.nq, p.err_flag))
+          atomicAdd(reinterpret_cast<unsigned long long*>(p.dbg_cells + ci), static_cast<unsigned long long>(c));
       }
     }
   }
@@ -886,15 +916,32 @@ static cudaError_t launch_one(const PrefillMaps& maps, const PrefillParams& p, c
                               cudaStream_t stream) {
   using C = PrefillCfg<DQK, DV, DIFF, KV2>;
   auto kern = prefill_kernel<DQK, DV, DIFF, GEN, KV2>;
-  static bool attr_set = false;  // per process; the attribute is per function
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(kern), C::kSmemBytes);
+  if (e != cudaSuccess) return e;
   const int grid = nunits < p.num_ctas ? nunits : p.num_ctas;
   kern<<<grid, kThreads, C::kSmemBytes, stream>>>(maps.q, maps.q2, maps.k, maps.k2, maps.v, maps.ks, maps.vs,
                                                   maps.o, p, rows);
+  return cudaGetLastError();
+}
+
+// Evaluates exp2_fma2 elementwise (y[i] = 2^x[i]), so that the polynomial
+// the differential kernel uses for part of its exponentials can be checked
+// against an error bound on its own.
+__global__ void exp2_fma2_kernel(const float* __restrict__ x, float* __restrict__ y, int64_t n) {
+  const int64_t npair = (n + 1) / 2;
+  for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < npair; t += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t i = 2 * t;
+    const bool two = i + 1 < n;
+    const float2 r = exp2_fma2(make_float2(x[i], two ? x[i + 1] : x[i]));
+    y[i] = r.x;
+    if (two) y[i + 1] = r.y;
+  }
+}
+
+cudaError_t launch_exp2_fma2(const float* x, float* y, int64_t n, cudaStream_t stream) {
+  const int64_t npair = (n + 1) / 2;
+  const int64_t blocks = (npair + 255) / 256;
+  exp2_fma2_kernel<<<(unsigned)(blocks < 148 * 16 ? blocks : 148 * 16), 256, 0, stream>>>(x, y, n);
   return cudaGetLastError();
 }
 

@@ -12,6 +12,33 @@ namespace swa {
 // SWA_ERR_TIMEOUT and returns. Legitimate waits last microseconds.
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 
+// Bounds-checking debug build (-DSWA_DEBUG_BOUNDS): every TMA coordinate and
+// computed global index is checked before the access it feeds; a failed
+// check records SWA_ERR_BOUNDS (6) in the device error word and the access is
+// skipped. A skipped load leaves its barrier short, so the consumer's bounded
+// wait ends the launch (the first error recorded stays visible only if no
+// later one overwrites it; either way the status is not SWA_OK). Release
+// builds compile every check to `true`.
+#ifdef SWA_DEBUG_BOUNDS
+__device__ __forceinline__ bool bounds_ok(bool ok, int* err) {
+  if (!ok && err != nullptr) atomicExch(err, 6 /* SWA_ERR_BOUNDS */);
+  return ok;
+}
+// lo <= v < hi
+#define SWA_IN(v, lo, hi, err) \
+  ::swa::bounds_ok((long long)(v) >= (long long)(lo) && (long long)(v) < (long long)(hi), (err))
+// a 64-element-wide TMA box at (x, row, z) of a view with `d` columns,
+// `rows` rows and `nz` outer slices: x a multiple of 64 inside the row, the
+// box's first row and slice inside the view
+#define SWA_TMA_IN(x, d, row, rows, z, nz, err)                                                             \
+  ::swa::bounds_ok((x) >= 0 && (x) % 64 == 0 && (x) < (d) && (long long)(row) >= 0 &&                          \
+                       (long long)(row) < (long long)(rows) && (long long)(z) >= 0 && (long long)(z) < (long long)(nz), \
+                   (err))
+#else
+#define SWA_IN(v, lo, hi, err) true
+#define SWA_TMA_IN(x, d, row, rows, z, nz, err) true
+#endif
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -442,6 +469,11 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
+}
+
+// A bf16 pair (as packed by pack_bf16) back to two floats, exactly.
+__device__ __forceinline__ float2 unpack_bf16(uint32_t v) {
+  return make_float2(__uint_as_float(v << 16), __uint_as_float(v & 0xffff0000u));
 }
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,

@@ -43,8 +43,11 @@ typedef enum {
   SWA_ERR_UNSUPPORTED = 2, /* valid but not built: head dim outside {64,128} */
   SWA_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed           */
   SWA_ERR_TIMEOUT = 4,     /* a bounded in-kernel wait ran out            */
-  SWA_ERR_SCRATCH_TOO_SMALL = 5 /* sizes need more scratch than the library's
-                                   static decode array holds               */
+  SWA_ERR_SCRATCH_TOO_SMALL = 5, /* sizes need more scratch than the library's
+                                    static decode array holds              */
+  SWA_ERR_BOUNDS = 6       /* bounds-checking debug build only: a TMA
+                              coordinate or global index fell outside its
+                              tensor (the access was skipped)              */
 } swa_status_t;
 
 /* Optional device-side debug outputs of the prefill kernels (pass NULL to
@@ -273,6 +276,12 @@ swa_status_t strided_attn_bwd(const void* q, const void* k, const void* v, const
                               int B, int Hq, int Hkv, int N, int d, int W, int stride,
                               float scale, void* workspace, size_t ws_bytes, void* stream);
 
+/* Note on determinism: the stride keys' partial dK/dV are summed in fp32 with
+ * atomic adds, in an order that varies from run to run, so strided_attn_bwd's
+ * dK and dV can differ in the last bit between identical calls (within the
+ * stated accuracy). swa_attn_bwd and every forward entry point are
+ * deterministic. */
+
 /* Scratch bytes strided_attn_bwd needs (0 on bad sizes). */
 size_t strided_attn_bwd_workspace_bytes(int B, int Hq, int Hkv, int N, int d, int stride);
 
@@ -303,6 +312,17 @@ int64_t swa_schedule(int kind, int N, int W, int stride, int Bq, int Bk, int32_t
  * (kind as swa_schedule; stride ignored unless kind is 1 or 3). -1 on bad
  * arguments. Source: "Attention Variants Compared", count_nonmasked. */
 int64_t swa_count_nonmasked(int kind, int N, int W, int stride);
+
+/* Debug: y[i] = 2^x[i] through the prefill kernels' own FMA-pipe exponential
+ * (Cody-Waite range reduction plus a cubic minimax polynomial, evaluated in
+ * fp32 on pairs), which the differential kernel uses for a quarter of its
+ * exponentials instead of the MUFU unit. Exposed so that a test can hold it
+ * to its bound: relative error at most 1.02e-4 for x in [-125, 8], exactly 0
+ * for x <= -127 (-inf included), finite everywhere below 8 (in the kernels
+ * the argument never exceeds 8). Not part of the attention path.
+ *   x, y: device fp32 [n], 4-byte aligned (y written); n >= 0 (0: no-op).
+ *   A null or misaligned pointer or n < 0 returns SWA_ERR_INVALID_ARG. */
+swa_status_t swa_debug_exp2(const float* x, float* y, int64_t n, void* stream);
 
 /* Synchronises `stream`, then returns and clears the device error flag of
  * the current device (SWA_OK if no kernel recorded an error). */

@@ -168,3 +168,31 @@ def test_global_and_dilated_bad_arguments(lib):
     st = lib.dilated_attn_fwd(g, g, g, g, None, 1, 2, 2, 256, 96, 16, 2, ctypes.c_float(0.1), None)
     assert st == swa.ERR_UNSUPPORTED  # head dim
     assert lib.swa_count_nonmasked(3, 10, 4, -1) == -1
+
+
+def test_decode_window_beyond_limit_rejected_before_launch(lib):
+    """A window past 2^30 slots would overflow the split arithmetic: every
+    decode entry rejects it (and the workspace query returns 0) up front."""
+    P, I, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    g = P(0x10000)  # aligned, never dereferenced: validation fails first
+    big = (1 << 30) + 1
+    lib.swa_decode_step_static.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, F, P]
+    lib.swa_decode_step_static.restype = I
+    st = lib.swa_decode_step_static(g, g, g, g, g, g, g, 1, 2, 1, 128, big, F(0.1), None)
+    assert st == swa.ERR_INVALID_ARG
+    st = lib.swa_decode_step_static(g, g, g, g, g, g, g, 1, 2, 1, 128, 0x7fffffff, F(0.1), None)
+    assert st == swa.ERR_INVALID_ARG
+    assert lib.swa_decode_workspace_bytes(1, 2, 1, 128, big) == 0
+    assert lib.swa_sink_decode_workspace_bytes(1, 2, 1, 128, 4, 1 << 30) == 0
+    assert lib.swa_diff_decode_workspace_bytes(1, 2, 1, 64, 128, big) == 0
+    st = lib.swa_decode_step(g, g, g, g, g, g, g, 1, 2, 1, 128, big, 0.1, g, 1 << 40, None)
+    assert st == swa.ERR_INVALID_ARG
+
+
+def test_debug_exp2_bad_arguments(lib):
+    P = ctypes.c_void_p
+    g = P(0x10000)
+    assert lib.swa_debug_exp2(None, g, 4, None) == swa.ERR_INVALID_ARG
+    assert lib.swa_debug_exp2(g, P(0x10002), 4, None) == swa.ERR_INVALID_ARG  # misaligned
+    assert lib.swa_debug_exp2(g, g, -1, None) == swa.ERR_INVALID_ARG
+    assert lib.swa_debug_exp2(g, g, 0, None) == swa.OK  # nothing to do, nothing launched

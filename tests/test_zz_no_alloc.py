@@ -64,7 +64,35 @@ def test_static_scratch_matches_workspace_entry_point(lib):
         diff = (out_a.float() - out_b.float()).abs()
         assert torch.isfinite(out_b.float()).all()
         assert diff.max().item() <= MAX_TOL and diff.mean().item() <= MEAN_TOL
+        # the same kernels with the same split plan: identical bits, so no
+        # record of the shared array may be stale or misplaced
+        assert torch.equal(out_a, out_b)
     assert torch.equal(kc_a, kc_b) and torch.equal(vc_a, vc_b)
+
+
+def test_short_history_after_a_larger_call(lib):
+    """A call whose position is still inside the first window (pos < W, so
+    some splits hold no position yet) right after a call that filled every
+    record of the array: the empty splits must overwrite the old records."""
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    for (B, Hq, Hkv, d, W, pos0) in [(8, 16, 8, 128, 1024, 5000), (8, 16, 8, 128, 1024, 3)]:
+        T = 2
+        q, k_new, v_new, k_cache, v_cache = (t.cuda() for t in decode_inputs(T, B, Hq, Hkv, d, W, seed=pos0))
+        kc_a, vc_a = k_cache.clone(), v_cache.clone()
+        kc_b, vc_b = k_cache.clone(), v_cache.clone()
+        pos = torch.tensor([[pos0 + t] * B for t in range(T)], dtype=torch.int32, device="cuda")
+        ws = torch.empty(swa.decode_workspace_bytes(B, Hq, Hkv, d, W), dtype=torch.uint8, device="cuda")
+        scale = ctypes.c_float(1.0 / np.sqrt(d))
+        for t in range(T):
+            out_a = torch.empty_like(q[t])
+            out_b = torch.full_like(q[t], float("nan"))
+            assert lib.swa_decode_step(ptr(q[t]), ptr(k_new[t]), ptr(v_new[t]), ptr(kc_a), ptr(vc_a), ptr(pos[t]),
+                                       ptr(out_a), B, Hq, Hkv, d, W, scale, ptr(ws), ws.numel(), stream) == swa.OK
+            assert lib.swa_decode_step_static(ptr(q[t]), ptr(k_new[t]), ptr(v_new[t]), ptr(kc_b), ptr(vc_b),
+                                              ptr(pos[t]), ptr(out_b), B, Hq, Hkv, d, W, scale, stream) == swa.OK
+            torch.cuda.synchronize()
+            assert swa.last_device_error() == swa.OK
+            assert torch.equal(out_a, out_b), (pos0, t)
 
 
 def test_sizes_beyond_the_array_are_rejected(lib):
