@@ -302,6 +302,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   // direction evens out the per-CTA totals.
   const int nunits = p.nunits, P = gridDim.x, c_id = blockIdx.x;
   auto unit_of = [&](int rnd) -> int { return rnd * P + ((rnd & 1) ? (P - 1 - c_id) : c_id); };
+  // The first round from r on that gives this CTA a unit (-1: none left),
+  // with the unit decoded and its key items listed. The MMA and softmax
+  // warps call it for the next unit before they drain the current one, so
+  // its integer work is off the path between units.
+  auto next_unit = [&](int r, Unit& un, Items& it) -> int {
+    for (; r * P < nunits; ++r) {
+      const int ui = unit_of(r);
+      if (ui < nunits) {
+        un = decode_unit(p, ui);
+        it = unit_items<GEN>(p, un);
+        return r;
+      }
+    }
+    return -1;
+  };
 
   if (threadIdx.x == 0) {
     mbar_init(bar(BarLayout::kQ), 1);
@@ -473,11 +488,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       int L = 0;
       int nq = 0;  // units started (Q phases)
       bool ok = true;
-      for (int rnd = 0; rnd * P < nunits && ok; ++rnd) {
-        const int ui = unit_of(rnd);
-        if (ui >= nunits) continue;
-        const Unit un = decode_unit(p, ui);
-        const Items it = unit_items<GEN>(p, un);
+      Unit un;
+      Items it;
+      for (int rnd = next_unit(0, un, it); rnd >= 0 && ok;) {
         sm0.ntot = un.valid[0] ? qtile_nkeys(it.k[0]) : 0;
         sm1.ntot = un.valid[1] ? qtile_nkeys(it.k[1]) : 0;
         sm0.kcount = sm1.kcount = 0;
@@ -607,6 +620,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           prev_vslot = vslot;
           prev_vuse = vuse;
         }
+        Unit un_next;
+        Items it_next;
+        const int rnd_next = ok ? next_unit(rnd + 1, un_next, it_next) : -1;
         if (ok && (sm0.pending || sm1.pending)) {
           ok = wait(bar(BarLayout::kFull + prev_vslot), prev_vuse & 1);
           if (ok) tc_fence_after();
@@ -623,6 +639,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           p.dbg_ntiles[sm1.dbg_row] = sm1.kcount;
         if (un.valid[0]) ++sm0.nunit;
         if (un.valid[1]) ++sm1.nunit;
+        un = un_next;
+        it = it_next;
+        rnd = rnd_next;
       }
       if (__any_sync(0xffffffffu, !ok || *abort_flag)) {
         commit(bar(BarLayout::kFinal));
@@ -679,15 +698,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     int nx = 0;      // differential hand-offs
     bool ok = true;
 
-    for (int rnd = 0; rnd * P < nunits && ok; ++rnd) {
-      const int ui = unit_of(rnd);
-      if (ui >= nunits) continue;
-      const Unit un = decode_unit(p, ui);
-      const Items it = unit_items<GEN>(p, un);
+    Unit un;
+    Items it;
+    for (int rnd = next_unit(0, un, it); rnd >= 0 && ok;) {
       // this sub's fields as scalars: a run-time index into the unit's
       // arrays would keep them in local memory
       const bool valid_t = t ? un.valid[1] : un.valid[0];
-      if (!valid_t) continue;
+      if (!valid_t) {
+        rnd = next_unit(rnd + 1, un, it);
+        continue;
+      }
       const int qt_t = t ? un.qt[1] : un.qt[0];
       const int hq = t ? un.hq[1] : un.hq[0];
       const int ks_lo = t ? it.k[1].band_lo : it.k[0].band_lo;
@@ -841,6 +861,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++kglob;
       }
       if (!ok) break;
+      Unit un_next;
+      Items it_next;
+      const int rnd_next = next_unit(rnd + 1, un_next, it_next);  // while the last PV runs
 
       // -------------------------------------------------- epilogue ---
       {
@@ -898,6 +921,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0 && SWA_IN(ci, 0, (int64_t)p.B * p.Hq * p.nq, p.err_flag))
           atomicAdd(reinterpret_cast<unsigned long long*>(p.dbg_cells + ci), static_cast<unsigned long long>(c));
       }
+      un = un_next;
+      it = it_next;
+      rnd = rnd_next;
     }
   }
 
