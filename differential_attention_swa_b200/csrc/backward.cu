@@ -62,14 +62,20 @@ struct BwdCfg {
   static_assert(256 + 2 * D <= 512, "tensor memory");
 };
 
+// Each step's score products run as two halves of 64 columns (queries in
+// the dK/dV kernel, keys in the dQ kernel), each with its own barriers, so
+// the tensor core works on one half (its accumulation, then the next step's
+// scores) while the elementwise warps process the other.
+constexpr int kBH = 64;  // columns of a half
+
 struct BwdBar {
   static constexpr int kFixed = 0;
   static constexpr int kFull = 1;   // + stage
   static constexpr int kEmpty = 3;  // + stage
-  static constexpr int kS = 5;      // score products of the step in TMEM
-  static constexpr int kP = 6;      // elementwise done: P / dS written
-  static constexpr int kAcc = 7;    // accumulators final
-  static constexpr int kFinal = 8;  // MMA drain on abort
+  static constexpr int kS = 5;      // + half: score products of the half in TMEM
+  static constexpr int kP = 7;      // + half: elementwise done, P / dS of the half written
+  static constexpr int kAcc = 9;    // accumulators final
+  static constexpr int kFinal = 10; // MMA drain on abort
   static constexpr int kWordsOff = 256;
 };
 
@@ -182,8 +188,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(bar(BwdBar::kFull + s), 1);
       mbar_init(bar(BwdBar::kEmpty + s), 1);
     }
-    mbar_init(bar(BwdBar::kS), 1);
-    mbar_init(bar(BwdBar::kP), 128);
+    for (int h = 0; h < 2; ++h) {
+      mbar_init(bar(BwdBar::kS + h), 1);
+      mbar_init(bar(BwdBar::kP + h), 128);
+    }
     mbar_init(bar(BwdBar::kAcc), 1);
     mbar_init(bar(BwdBar::kFinal), 1);
     *abort_flag = 0;
@@ -244,57 +252,74 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   } else if (warp == 1) {
     // ----------------------------------------------------------- MMA ---
     if (lane == 0) {
-      const uint32_t idesc_s = idesc_bf16_f32(kBT, kBT, false);
+      const uint32_t idesc_s = idesc_bf16_f32(kBT, kBH, false);
       const uint32_t idesc_acc = idesc_bf16_f32(kBT, D, true);
       const uint64_t k_desc = sw128_desc(sbase + C::kOffA, 16, 1024);
       const uint64_t v_desc = sw128_desc(sbase + C::kOffB, 16, 1024);
       bool ok = mbar_wait(bar(BwdBar::kFixed), 0, abort_flag);
       if (!ok) bwd_timeout(abort_flag, p.err_flag);
       tc_fence_after();
-      for (int s = 0; ok && s <= nsteps; ++s) {
-        if (s > 0) {
-          // dV += P^T dO and dK += dS^T Q of the previous step
-          if (!mbar_wait(bar(BwdBar::kP), (s - 1) & 1, abort_flag)) {
-            bwd_timeout(abort_flag, p.err_flag);
+      // S^T = K Q^T and dP^T = V dO^T of queries 64h .. 64h+63 of step s
+      // (rows: keys, columns: queries; the half's Q and dO rows start 64
+      // rows = 8192 bytes into each 64-column box)
+      auto scores = [&](int s, int h) {
+        const uint32_t cur = sbase + C::kOffStages + (s & 1) * C::kStage + h * 8192;
+        const uint64_t q_k = sw128_desc(cur, 16, 1024);
+        const uint64_t do_k = sw128_desc(cur + C::kTile, 16, 1024);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t off = (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
+          umma_bf16_ss(tmem + C::kColS + kBH * h, k_desc + off, q_k + off, idesc_s, kk > 0 ? 1u : 0u);
+          umma_bf16_ss(tmem + C::kColDP + kBH * h, v_desc + off, do_k + off, idesc_s, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(bar(BwdBar::kS + h));
+      };
+      // dV += P^T dO and dK += dS^T Q over the half's 64 queries (P^T, dS^T
+      // as bf16 pairs in the half's first 32 columns)
+      auto accumulate = [&](int s, int h) {
+        const uint32_t cur = sbase + C::kOffStages + (s & 1) * C::kStage;
+        const uint64_t q_mn = sw128_desc(cur, 16384, 1024);
+        const uint64_t do_mn = sw128_desc(cur + C::kTile, 16384, 1024);
+#pragma unroll
+        for (int kk = 0; kk < kBH / 16; ++kk) {
+          const uint32_t acc = (s == 0 && h == 0 && kk == 0) ? 0u : 1u;
+          const uint64_t row = (uint64_t)(((kBH / 16) * h + kk) * 2048 >> 4);
+          umma_bf16_ts(tmem + C::kColAcc, tmem + C::kColS + kBH * h + kk * 8, do_mn + row, idesc_acc, acc);
+          umma_bf16_ts(tmem + C::kColAcc + D, tmem + C::kColDP + kBH * h + kk * 8, q_mn + row, idesc_acc, acc);
+        }
+      };
+      if (ok && nsteps > 0) {
+        ok = mbar_wait(bar(BwdBar::kFull), 0, abort_flag);
+        if (ok) {
+          tc_fence_after();
+          scores(0, 0);
+          scores(0, 1);
+        }
+      }
+      for (int s = 0; ok && s < nsteps; ++s) {
+        for (int h = 0; h < 2 && ok; ++h) {
+          if (!mbar_wait(bar(BwdBar::kP + h), s & 1, abort_flag)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t prev = sbase + C::kOffStages + ((s - 1) & 1) * C::kStage;
-          const uint64_t q_mn = sw128_desc(prev, 16384, 1024);
-          const uint64_t do_mn = sw128_desc(prev + C::kTile, 16384, 1024);
-#pragma unroll
-          for (int kk = 0; kk < kBT / 16; ++kk) {
-            const uint32_t acc = (s == 1 && kk == 0) ? 0u : 1u;
-            umma_bf16_ts(tmem + C::kColAcc, tmem + C::kColS + kk * 8, do_mn + (uint64_t)(kk * 2048 >> 4), idesc_acc,
-                         acc);
-            umma_bf16_ts(tmem + C::kColAcc + D, tmem + C::kColDP + kk * 8, q_mn + (uint64_t)(kk * 2048 >> 4),
-                         idesc_acc, acc);
+          accumulate(s, h);
+          if (h == 1) umma_commit(bar(BwdBar::kEmpty + (s & 1)));  // Q, dO and the row tables of step s read
+          if (s + 1 < nsteps) {
+            if (h == 0) {
+              if (!mbar_wait(bar(BwdBar::kFull + ((s + 1) & 1)), ((s + 1) >> 1) & 1, abort_flag)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+            }
+            // into the columns the accumulation above reads first (MMAs run in issue order)
+            scores(s + 1, h);
           }
-          umma_commit(bar(BwdBar::kEmpty + ((s - 1) & 1)));  // Q, dO and the row tables of step s-1 read
         }
-        if (s == nsteps) {
-          umma_commit(bar(BwdBar::kAcc));
-          break;
-        }
-        if (!mbar_wait(bar(BwdBar::kFull + (s & 1)), (s >> 1) & 1, abort_flag)) {
-          bwd_timeout(abort_flag, p.err_flag);
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t cur = sbase + C::kOffStages + (s & 1) * C::kStage;
-        const uint64_t q_k = sw128_desc(cur, 16, 1024);
-        const uint64_t do_k = sw128_desc(cur + C::kTile, 16, 1024);
-        // S^T = K Q^T and dP^T = V dO^T (rows: keys, columns: queries)
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t off = (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
-          umma_bf16_ss(tmem + C::kColS, k_desc + off, q_k + off, idesc_s, kk > 0 ? 1u : 0u);
-          umma_bf16_ss(tmem + C::kColDP, v_desc + off, do_k + off, idesc_s, kk > 0 ? 1u : 0u);
-        }
-        umma_commit(bar(BwdBar::kS));
       }
+      if (ok) umma_commit(bar(BwdBar::kAcc));
+      else bwd_timeout(abort_flag, p.err_flag);
       if (!ok || *abort_flag) {
         umma_commit(bar(BwdBar::kFinal));
         mbar_wait_timed(bar(BwdBar::kFinal), 0);
@@ -308,32 +333,27 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t lane_addr = static_cast<uint32_t>(qw * 32) << 16;
     const float sl2 = p.scale_log2;
     bool ok = true;
-    for (int s = 0; s < nsteps; ++s) {
+    for (int s = 0; s < nsteps && ok; ++s) {
       const int qt = qt_lo + s % nqt;
-      const bool got = mbar_wait(bar(BwdBar::kS), s & 1, abort_flag);
-      if (!__all_sync(0xffffffffu, got)) {
-        if (lane == 0) bwd_timeout(abort_flag, p.err_flag);
-        ok = false;
-        break;
-      }
-      // the row tables were written by the copy engine: acquire them from the
-      // stage's own barrier (complete already; the stage cannot be refilled
-      // before this step's P^T and dS^T are consumed)
-      const bool have = mbar_wait(bar(BwdBar::kFull + (s & 1)), (s >> 1) & 1, abort_flag);
-      if (!__all_sync(0xffffffffu, have)) {
-        if (lane == 0) bwd_timeout(abort_flag, p.err_flag);
-        ok = false;
-        break;
-      }
-      tc_fence_after();
       const float* lse2 = reinterpret_cast<const float*>(smem + C::kOffStages + (s & 1) * C::kStage + 2 * C::kTile);
       const float* dd = lse2 + kBT;
 #pragma unroll 1
-      for (int h = 0; h < 2; ++h) {  // two halves of 64 queries
+      for (int h = 0; h < 2; ++h) {  // two halves of 64 queries, each on its own barriers
+        const bool got = mbar_wait(bar(BwdBar::kS + h), s & 1, abort_flag);
+        // the row tables were written by the copy engine: acquire them from
+        // the stage's own barrier (complete already; the stage cannot be
+        // refilled before this step's P^T and dS^T are consumed)
+        const bool have = got && (h == 1 || mbar_wait(bar(BwdBar::kFull + (s & 1)), (s >> 1) & 1, abort_flag));
+        if (!__all_sync(0xffffffffu, have)) {
+          if (lane == 0) bwd_timeout(abort_flag, p.err_flag);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
         float sv[64], dp[64];
         uint32_t pk[32], dk[32];
-        tmem_ld64(tmem + lane_addr + C::kColS + 64 * h, sv);
-        tmem_ld64(tmem + lane_addr + C::kColDP + 64 * h, dp);
+        tmem_ld64(tmem + lane_addr + C::kColS + kBH * h, sv);
+        tmem_ld64(tmem + lane_addr + C::kColDP + kBH * h, dp);
 #pragma unroll
         for (int c = 0; c < 64; c += 2) {
           const int c0 = 64 * h + c;
@@ -346,13 +366,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           pk[c >> 1] = pack_bf16(p0, p1);
           dk[c >> 1] = pack_bf16(p0 * (dp[c] - dd[c0]), p1 * (dp[c + 1] - dd[c0 + 1]));
         }
-        // P^T over S^T and dS^T over dP^T as bf16 pairs: queries 64h .. 64h+63
-        // land in columns 32h .. 32h+31, all of them already read
-        tmem_st32_u(tmem + lane_addr + C::kColS + 32 * h, pk);
-        tmem_st32_u(tmem + lane_addr + C::kColDP + 32 * h, dk);
+        // P^T over S^T and dS^T over dP^T as bf16 pairs: the half's 64
+        // queries land in its own first 32 columns, already read
+        tmem_st32_u(tmem + lane_addr + C::kColS + kBH * h, pk);
+        tmem_st32_u(tmem + lane_addr + C::kColDP + kBH * h, dk);
+        tc_fence_before();
+        mbar_arrive(bar(BwdBar::kP + h));
       }
-      tc_fence_before();
-      mbar_arrive(bar(BwdBar::kP));
     }
     if (ok) {
       const bool got = mbar_wait(bar(BwdBar::kAcc), 0, abort_flag);
@@ -462,8 +482,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(bar(BwdBar::kFull + s), 1);
       mbar_init(bar(BwdBar::kEmpty + s), 1);
     }
-    mbar_init(bar(BwdBar::kS), 1);
-    mbar_init(bar(BwdBar::kP), 128);
+    for (int h = 0; h < 2; ++h) {
+      mbar_init(bar(BwdBar::kS + h), 1);
+      mbar_init(bar(BwdBar::kP + h), 128);
+    }
     mbar_init(bar(BwdBar::kAcc), 1);
     mbar_init(bar(BwdBar::kFinal), 1);
     *abort_flag = 0;
@@ -518,51 +540,69 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   } else if (warp == 1) {
     // ----------------------------------------------------------- MMA ---
     if (lane == 0) {
-      const uint32_t idesc_s = idesc_bf16_f32(kBT, kBT, false);
+      const uint32_t idesc_s = idesc_bf16_f32(kBT, kBH, false);
       const uint32_t idesc_acc = idesc_bf16_f32(kBT, D, true);
       const uint64_t q_desc = sw128_desc(sbase + C::kOffA, 16, 1024);
       const uint64_t do_desc = sw128_desc(sbase + C::kOffB, 16, 1024);
       bool ok = mbar_wait(bar(BwdBar::kFixed), 0, abort_flag);
       if (!ok) bwd_timeout(abort_flag, p.err_flag);
       tc_fence_after();
-      for (int s = 0; ok && s <= nsteps; ++s) {
-        if (s > 0) {
-          // dQ += dS K of the previous step (dS as bf16 pairs over S)
-          if (!mbar_wait(bar(BwdBar::kP), (s - 1) & 1, abort_flag)) {
-            bwd_timeout(abort_flag, p.err_flag);
+      // S = Q K^T and dP = dO V^T over keys 64h .. 64h+63 of step s (rows:
+      // queries, columns: keys; the half's K and V rows start 8192 bytes
+      // into each 64-column box)
+      auto scores = [&](int s, int h) {
+        const uint32_t cur = sbase + C::kOffStages + (s & 1) * C::kStage + h * 8192;
+        const uint64_t k_k = sw128_desc(cur, 16, 1024);
+        const uint64_t v_k = sw128_desc(cur + C::kTile, 16, 1024);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t off = (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
+          umma_bf16_ss(tmem + C::kColS + kBH * h, q_desc + off, k_k + off, idesc_s, kk > 0 ? 1u : 0u);
+          umma_bf16_ss(tmem + C::kColDP + kBH * h, do_desc + off, v_k + off, idesc_s, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(bar(BwdBar::kS + h));
+      };
+      // dQ += dS K over the half's 64 keys (dS as bf16 pairs in the half's
+      // first 32 columns)
+      auto accumulate = [&](int s, int h) {
+        const uint64_t k_mn = sw128_desc(sbase + C::kOffStages + (s & 1) * C::kStage, 16384, 1024);
+#pragma unroll
+        for (int kk = 0; kk < kBH / 16; ++kk)
+          umma_bf16_ts(tmem + C::kColAcc, tmem + C::kColS + kBH * h + kk * 8,
+                       k_mn + (uint64_t)(((kBH / 16) * h + kk) * 2048 >> 4), idesc_acc,
+                       (s == 0 && h == 0 && kk == 0) ? 0u : 1u);
+      };
+      if (ok && nsteps > 0) {
+        ok = mbar_wait(bar(BwdBar::kFull), 0, abort_flag);
+        if (ok) {
+          tc_fence_after();
+          scores(0, 0);
+          scores(0, 1);
+        }
+      }
+      for (int s = 0; ok && s < nsteps; ++s) {
+        for (int h = 0; h < 2 && ok; ++h) {
+          if (!mbar_wait(bar(BwdBar::kP + h), s & 1, abort_flag)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint64_t k_mn = sw128_desc(sbase + C::kOffStages + ((s - 1) & 1) * C::kStage, 16384, 1024);
-#pragma unroll
-          for (int kk = 0; kk < kBT / 16; ++kk)
-            umma_bf16_ts(tmem + C::kColAcc, tmem + C::kColS + kk * 8, k_mn + (uint64_t)(kk * 2048 >> 4), idesc_acc,
-                         (s == 1 && kk == 0) ? 0u : 1u);
-          umma_commit(bar(BwdBar::kEmpty + ((s - 1) & 1)));  // K and V of step s-1 read
+          accumulate(s, h);
+          if (h == 1) umma_commit(bar(BwdBar::kEmpty + (s & 1)));  // K and V of step s read
+          if (s + 1 < nsteps) {
+            if (h == 0) {
+              if (!mbar_wait(bar(BwdBar::kFull + ((s + 1) & 1)), ((s + 1) >> 1) & 1, abort_flag)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+            }
+            scores(s + 1, h);  // into the columns the accumulation above reads first
+          }
         }
-        if (s == nsteps) {
-          umma_commit(bar(BwdBar::kAcc));
-          break;
-        }
-        if (!mbar_wait(bar(BwdBar::kFull + (s & 1)), (s >> 1) & 1, abort_flag)) {
-          bwd_timeout(abort_flag, p.err_flag);
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t cur = sbase + C::kOffStages + (s & 1) * C::kStage;
-        const uint64_t k_k = sw128_desc(cur, 16, 1024);
-        const uint64_t v_k = sw128_desc(cur + C::kTile, 16, 1024);
-        // S = Q K^T and dP = dO V^T (rows: queries, columns: keys)
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t off = (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
-          umma_bf16_ss(tmem + C::kColS, q_desc + off, k_k + off, idesc_s, kk > 0 ? 1u : 0u);
-          umma_bf16_ss(tmem + C::kColDP, do_desc + off, v_k + off, idesc_s, kk > 0 ? 1u : 0u);
-        }
-        umma_commit(bar(BwdBar::kS));
       }
+      if (ok) umma_commit(bar(BwdBar::kAcc));
+      else bwd_timeout(abort_flag, p.err_flag);
       if (!ok || *abort_flag) {
         umma_commit(bar(BwdBar::kFinal));
         mbar_wait_timed(bar(BwdBar::kFinal), 0);
@@ -579,22 +619,22 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const bool rt_ok = SWA_IN(rt, 0, (int64_t)p.B * p.Hq * p.npad, p.err_flag);
     const float lse2 = rt_ok ? p.lse2[rt] : 0.f, dd = rt_ok ? p.dd[rt] : 0.f;
     bool ok = true;
-    for (int s = 0; s < nsteps; ++s) {
+    for (int s = 0; s < nsteps && ok; ++s) {
       const bool strided = SM && s < nst;
       const int kt = strided ? s : kt_lo + (s - nst);  // strided: compacted stride rows kt*128 ..
-      const bool got = mbar_wait(bar(BwdBar::kS), s & 1, abort_flag);
-      if (!__all_sync(0xffffffffu, got)) {
-        if (lane == 0) bwd_timeout(abort_flag, p.err_flag);
-        ok = false;
-        break;
-      }
-      tc_fence_after();
 #pragma unroll 1
-      for (int h = 0; h < 2; ++h) {  // two halves of 64 keys
+      for (int h = 0; h < 2; ++h) {  // two halves of 64 keys, each on its own barriers
+        const bool got = mbar_wait(bar(BwdBar::kS + h), s & 1, abort_flag);
+        if (!__all_sync(0xffffffffu, got)) {
+          if (lane == 0) bwd_timeout(abort_flag, p.err_flag);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
         float sv[64], dp[64];
         uint32_t pk[32];
-        tmem_ld64(tmem + lane_addr + C::kColS + 64 * h, sv);
-        tmem_ld64(tmem + lane_addr + C::kColDP + 64 * h, dp);
+        tmem_ld64(tmem + lane_addr + C::kColS + kBH * h, sv);
+        tmem_ld64(tmem + lane_addr + C::kColDP + kBH * h, dp);
         auto body = [&](auto attended) {
 #pragma unroll
           for (int c = 0; c < 64; c += 2) {
@@ -609,11 +649,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           body([&](int m) { return bwd_stride_attended(i, m, p.W, p.S, p.N); });
         else
           body([&](int key) { return bwd_attended(i, key, p.W, p.N); });
-        // dS over S as bf16 pairs: keys 64h .. 64h+63 in columns 32h .. 32h+31
-        tmem_st32_u(tmem + lane_addr + C::kColS + 32 * h, pk);
+        // dS over S as bf16 pairs: the half's 64 keys in its own first 32
+        // columns, already read
+        tmem_st32_u(tmem + lane_addr + C::kColS + kBH * h, pk);
+        tc_fence_before();
+        mbar_arrive(bar(BwdBar::kP + h));
       }
-      tc_fence_before();
-      mbar_arrive(bar(BwdBar::kP));
     }
     if (ok) {
       const bool got = mbar_wait(bar(BwdBar::kAcc), 0, abort_flag);
