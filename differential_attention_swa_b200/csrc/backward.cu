@@ -354,17 +354,28 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         uint32_t pk[32], dk[32];
         tmem_ld64(tmem + lane_addr + C::kColS + kBH * h, sv);
         tmem_ld64(tmem + lane_addr + C::kColDP + kBH * h, dp);
+        auto body = [&](auto attended) {
 #pragma unroll
-        for (int c = 0; c < 64; c += 2) {
-          const int c0 = 64 * h + c;
-          const int i0 = qt * kBT + c0;
-          const bool a0 = STRIDE ? bwd_stride_attended(i0, key, p.W, p.S, p.N) : bwd_attended(i0, key, p.W, p.N);
-          const bool a1 = STRIDE ? bwd_stride_attended(i0 + 1, key, p.W, p.S, p.N)
-                                 : bwd_attended(i0 + 1, key, p.W, p.N);
-          const float p0 = a0 ? ex2_approx(fmaf(sv[c], sl2, -lse2[c0])) : 0.f;
-          const float p1 = a1 ? ex2_approx(fmaf(sv[c + 1], sl2, -lse2[c0 + 1])) : 0.f;
-          pk[c >> 1] = pack_bf16(p0, p1);
-          dk[c >> 1] = pack_bf16(p0 * (dp[c] - dd[c0]), p1 * (dp[c + 1] - dd[c0 + 1]));
+          for (int c = 0; c < 64; c += 2) {
+            const int c0 = 64 * h + c;
+            const int i0 = qt * kBT + c0;
+            const bool a0 = attended(i0), a1 = attended(i0 + 1);
+            const float p0 = a0 ? ex2_approx(fmaf(sv[c], sl2, -lse2[c0])) : 0.f;
+            const float p1 = a1 ? ex2_approx(fmaf(sv[c + 1], sl2, -lse2[c0 + 1])) : 0.f;
+            pk[c >> 1] = pack_bf16(p0, p1);
+            dk[c >> 1] = pack_bf16(p0 * (dp[c] - dd[c0]), p1 * (dp[c + 1] - dd[c0 + 1]));
+          }
+        };
+        if constexpr (STRIDE) {
+          body([&](int i) { return bwd_stride_attended(i, key, p.W, p.S, p.N); });
+        } else {
+          // every (key, query) cell of this 128 x 64 block attended: no per-cell test
+          const int i_lo = qt * kBT + kBH * h, i_hi = i_lo + kBH - 1;
+          const int k_hi = kt * kBT + kBT - 1;
+          if (k_hi <= i_lo && i_hi - kt * kBT < p.W && i_hi < p.N && k_hi < p.N)
+            body([](int) { return true; });
+          else
+            body([&](int i) { return bwd_attended(i, key, p.W, p.N); });
         }
         // P^T over S^T and dS^T over dP^T as bf16 pairs: the half's 64
         // queries land in its own first 32 columns, already read
@@ -645,7 +656,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             pk[c >> 1] = pack_bf16(p0 * (dp[c] - dd), p1 * (dp[c + 1] - dd));
           }
         };
-        if (strided)
+        // every (query, key) cell of this 128 x 64 block attended: no per-cell test
+        const int64_t k_lo = (int64_t)kt * kBT + kBH * h, k_hi = k_lo + kBH - 1;  // strided: compacted indices
+        const int i_lo = qt * kBT, i_hi = i_lo + kBT - 1;
+        const bool full = strided ? (k_hi * p.S < (int64_t)i_lo - p.W + 1 && i_hi < p.N && k_hi * p.S < p.N)
+                                  : (k_hi <= i_lo && i_hi - k_lo < p.W && i_hi < p.N && k_hi < p.N);
+        if (full)
+          body([](int) { return true; });
+        else if (strided)
           body([&](int m) { return bwd_stride_attended(i, m, p.W, p.S, p.N); });
         else
           body([&](int key) { return bwd_attended(i, key, p.W, p.N); });
