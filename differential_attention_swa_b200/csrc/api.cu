@@ -85,7 +85,9 @@ swa_status_t run_prefill(int kind, bool diff, const void* q, const void* k, cons
   if (B < 1 || Hq < 1 || Hkv < 1 || N < 1 || W < 1 || Hq % Hkv != 0) return SWA_ERR_INVALID_ARG;
   if (kind == kMaskStrided && S < 1) return SWA_ERR_INVALID_ARG;
   if (kind == kMaskGlobal && S < 0) return SWA_ERR_INVALID_ARG;
-  if (!(scale > 0.f) || !std::isfinite(scale)) return SWA_ERR_INVALID_ARG;
+  // masked scores are carried as -FLT_MAX; scale * log2(e) >= 1e-30 keeps
+  // their weights at exactly 0
+  if (!(scale >= 1e-30f) || !std::isfinite(scale)) return SWA_ERR_INVALID_ARG;
   if ((int64_t)B * Hq > (1 << 30) / 8) return SWA_ERR_INVALID_ARG;
   if (!head_dim_ok(dqk) || !head_dim_ok(dv)) return SWA_ERR_UNSUPPORTED;
   if (!diff && dqk != dv) return SWA_ERR_UNSUPPORTED;
@@ -152,6 +154,24 @@ swa_status_t run_prefill(int kind, bool diff, const void* q, const void* k, cons
   }
   if (nunits > 0x7fffffff) return SWA_ERR_INVALID_ARG;
   p.nunits = (int)nunits;
+  // the divisors decode_unit uses (units per query tile, per batch, per KV
+  // head), the group size, and the stride clamped to N (a stride at or
+  // beyond N leaves key 0 as the only stride key either way)
+  if (p.mode == kModeHeadPairs) {
+    p.fd_u1 = make_fastdiv(B * Hkv * (G / 2));
+    p.fd_u2 = make_fastdiv(Hkv * (G / 2));
+    p.fd_u3 = make_fastdiv(G / 2);
+  } else if (p.mode == kModeKvPairs) {
+    p.fd_u1 = make_fastdiv(B * (Hq / 2));
+    p.fd_u2 = make_fastdiv(Hq / 2);
+    p.fd_u3 = make_fastdiv(1);
+  } else {
+    p.fd_u1 = make_fastdiv(B * Hq);
+    p.fd_u2 = make_fastdiv(Hq);
+    p.fd_u3 = make_fastdiv(1);
+  }
+  p.fd_g = make_fastdiv(G);
+  p.fd_s = make_fastdiv(kind == kMaskStrided ? (S < N ? S : N) : 1);
   p.num_ctas = sm_count();
   if (p.num_ctas <= 0) return SWA_ERR_CUDA;
   p.err_flag = device_error_ptr();

@@ -8,6 +8,8 @@
 #include <cstddef>
 #include <cstdint>
 
+#include "schedule.cuh"
+
 namespace swa {
 
 // Work-unit layouts of the prefill kernel (two 128-row "subs" per CTA).
@@ -36,6 +38,9 @@ struct PrefillParams {
   int dbg_cap;
   int inject_timeout;
   int* err_flag;  // device word that receives SWA_ERR_TIMEOUT
+  // divisions of the work-unit index (see decode_unit), by the group size
+  // and by the stride (clamped to N, which leaves the stride keys unchanged)
+  FastDiv fd_u1, fd_u2, fd_u3, fd_g, fd_s;
 };
 
 // Backward of the window attention (dQ, dK, dV from dO and the forward's

@@ -41,6 +41,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <cfloat>
 #include <cstdint>
 #include <type_traits>
 
@@ -63,6 +64,9 @@ constexpr int kThreads = 384;
 // Lazy rescale threshold (log2 units): O and l keep a stale row max until a
 // new score exceeds it by more than this, so P stays below 2^8.
 constexpr float kRescaleTau = 8.0f;
+// Scale of the mask's saturated FMA: |c - c0 +- 1/2| >= 1/2, so the product
+// is far outside [0, 1] for every column either side of the edge.
+constexpr float kMaskScale = 1e30f;
 
 
 // Per-instantiation choices, measured on B200 (tcgen05 MMAs with M = 128 and
@@ -171,53 +175,44 @@ struct Unit {
   int valid[2];
 };
 
+// Unit u of the launch (heaviest query tiles first). The divisions by the
+// group sizes go through the FastDivs the host builds (fd_u1: units per query
+// tile, fd_u2: units per batch, fd_u3: head pairs per KV head, fd_g: Hq/Hkv).
 __device__ __forceinline__ Unit decode_unit(const PrefillParams& p, int u) {
   Unit r;
+  const int q1 = p.fd_u1(u);  // query tile (or tile pair) counted from the last
+  const int bh = u - q1 * (int)p.fd_u1.d;
+  r.b = p.fd_u2(bh);
+  const int rem = bh - r.b * (int)p.fd_u2.d;
   if (p.mode == kModeHeadPairs) {
-    const int half = p.G / 2;
-    const int per_b = p.Hkv * half;
-    const int qt = p.nq - 1 - u / (p.B * per_b);
-    const int bh = u % (p.B * per_b);
-    r.b = bh / per_b;
-    const int rem = bh % per_b;
-    r.hkv = rem / half;
-    const int gp = rem % half;
+    r.hkv = p.fd_u3(rem);
+    const int gp = rem - r.hkv * (int)p.fd_u3.d;
     r.hq[0] = r.hkv * p.G + 2 * gp;
     r.hq[1] = r.hq[0] + 1;
-    r.qt[0] = r.qt[1] = qt;
+    r.qt[0] = r.qt[1] = p.nq - 1 - q1;
     r.valid[0] = r.valid[1] = 1;
   } else if (p.mode == kModeKvPairs) {
-    // consecutive query heads 2gp, 2gp+1 at the same query tile; each reads
+    // consecutive query heads 2j, 2j+1 at the same query tile; each reads
     // its own KV head (odd group sizes)
-    const int half = p.Hq / 2;
-    const int qt = p.nq - 1 - u / (p.B * half);
-    const int bh = u % (p.B * half);
-    r.b = bh / half;
-    r.hq[0] = 2 * (bh % half);
+    r.hq[0] = 2 * rem;
     r.hq[1] = r.hq[0] + 1;
-    r.hkv = r.hq[0] / p.G;
-    r.hkv1 = r.hq[1] / p.G;
-    r.qt[0] = r.qt[1] = qt;
+    r.hkv = p.fd_g(r.hq[0]);
+    r.hkv1 = p.fd_g(r.hq[1]);
+    r.qt[0] = r.qt[1] = p.nq - 1 - q1;
     r.valid[0] = r.valid[1] = 1;
     return r;
   } else if (p.mode == kModeTilePairs) {
-    const int nqp = (p.nq + 1) / 2;
-    const int qp = nqp - 1 - u / (p.B * p.Hq);
-    const int bh = u % (p.B * p.Hq);
-    r.b = bh / p.Hq;
-    r.hq[0] = r.hq[1] = bh % p.Hq;
-    r.hkv = r.hq[0] / p.G;
+    const int qp = (p.nq + 1) / 2 - 1 - q1;
+    r.hq[0] = r.hq[1] = rem;
+    r.hkv = p.fd_g(rem);
     r.qt[0] = 2 * qp;
     r.qt[1] = 2 * qp + 1;
     r.valid[0] = 1;
     r.valid[1] = r.qt[1] < p.nq;
   } else {  // differential: both maps of the same rows
-    const int qt = p.nq - 1 - u / (p.B * p.Hq);
-    const int bh = u % (p.B * p.Hq);
-    r.b = bh / p.Hq;
-    r.hq[0] = r.hq[1] = bh % p.Hq;
-    r.hkv = r.hq[0] / p.G;
-    r.qt[0] = r.qt[1] = qt;
+    r.hq[0] = r.hq[1] = rem;
+    r.hkv = p.fd_g(rem);
+    r.qt[0] = r.qt[1] = p.nq - 1 - q1;
     r.valid[0] = r.valid[1] = 1;
   }
   r.hkv1 = r.hkv;
@@ -242,8 +237,8 @@ __device__ __forceinline__ Items unit_items(const PrefillParams& p, const Unit& 
 #pragma unroll
   for (int t = 0; t < 2; ++t) {
     if (un.valid[t]) {
-      it.k[t] = GEN ? qtile_keys(p.kind, p.N, p.W, p.S, BM, BN, un.qt[t])
-                    : qtile_keys_basic(p.kind, p.N, p.W, p.S, BM, BN, un.qt[t]);
+      it.k[t] = GEN ? qtile_keys(p.kind, p.N, p.W, p.S, BM, BN, un.qt[t], p.fd_s)
+                    : qtile_keys_basic(p.kind, p.N, p.W, p.S, BM, BN, un.qt[t], p.fd_s);
       it.nst = imax(it.nst, it.k[t].n_stride);
       it.blo = imin(it.blo, it.k[t].band_lo);
       it.bhi = imax(it.bhi, it.k[t].band_hi);
@@ -721,8 +716,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int i = qt_t * BM + r;  // query index
       const bool row_ok = i < p.N;
       const int lo = window_lo(i, Wc);
-      const int mst = GEN ? extra_rows_below(p.kind, lo, p.S)  // extra-view rows below lo
-                          : ((p.kind == kMaskStrided) ? stride_rows_below(lo, p.S) : 0);
+      const int mst = GEN ? extra_rows_below(p.kind, lo, p.S, p.fd_s)  // extra-view rows below lo
+                          : ((p.kind == kMaskStrided) ? stride_rows_below(lo, p.S, p.fd_s) : 0);
       float m_run = -INFINITY;  // running max, log2 units (scores * scale * log2 e)
       float l_run = 0.f;  // sum of the bf16 weights the PV products consume
       float l_exact = 0.f;  // sum of the unrounded weights (log-sum-exp only)
@@ -757,30 +752,69 @@ __global__ void __launch_bounds__(kThreads, 1)
           float s[BH];
           if (BH == 128) tmem_ld128(s_tmem, s);
           else tmem_ld64(s_tmem + h * BH, s);
-          if (!__all_sync(0xffffffffu, full)) {
-            // Most partial halves are cut on one side only (the window's
-            // start, or the diagonal): test only the side some row needs.
-            const bool cut_lo = __any_sync(0xffffffffu, c0h > 0), cut_hi = __any_sync(0xffffffffu, c1h < BH - 1);
-            if (cut_lo && cut_hi) {
+          float m_tile;
+          if constexpr (BH == 64) {
+            if (!__all_sync(0xffffffffu, full)) {
+              // Masked columns become -FLT_MAX through FMA-pipe arithmetic
+              // (the ALU pipe, at half the rate, carries the row max): a
+              // saturated FMA gives the weight w = 1 for an attended column
+              // and 0 for a masked one, then s' = s w + (w - 1) FLT_MAX, exact
+              // in both cases. Most partial halves are cut on one side only
+              // (the window's start, or the diagonal): test only the side
+              // some row needs.
+              const bool cut_lo = __any_sync(0xffffffffu, c0h > 0), cut_hi = __any_sync(0xffffffffu, c1h < BH - 1);
+              const float blo = (0.5f - static_cast<float>(c0h)) * kMaskScale;  // c >= c0h: c k + blo > 0
+              const float bhi = (static_cast<float>(c1h) + 0.5f) * kMaskScale;  // c <= c1h: bhi - c k > 0
+              auto apply = [&](auto lo_side, auto hi_side) {
 #pragma unroll
-              for (int c = 0; c < BH; ++c) s[c] = (c >= c0h && c <= c1h) ? s[c] : -INFINITY;
-            } else if (cut_lo) {
-#pragma unroll
-              for (int c = 0; c < BH; ++c) s[c] = (c >= c0h) ? s[c] : -INFINITY;
-            } else {
-#pragma unroll
-              for (int c = 0; c < BH; ++c) s[c] = (c <= c1h) ? s[c] : -INFINITY;
+                for (int c = 0; c < BH; ++c) {
+                  float w = 1.f;
+                  if (decltype(lo_side)::value) w = fma_sat(static_cast<float>(c), kMaskScale, blo);
+                  if (decltype(hi_side)::value) w *= fma_sat(static_cast<float>(c), -kMaskScale, bhi);
+                  s[c] = fmaf(s[c], w, fmaf(w, FLT_MAX, -FLT_MAX));
+                }
+              };
+              using T = std::true_type;
+              using F = std::false_type;
+              if (cut_lo && cut_hi) apply(T{}, T{});
+              else if (cut_lo) apply(T{}, F{});
+              else apply(F{}, T{});
             }
+            // row max over 8 independent chains of three-input maxima
+            float mx8[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) mx8[j] = s[j];
+#pragma unroll
+            for (int c = 8; c < BH; c += 2) mx8[(c >> 1) & 7] = fmax3(mx8[(c >> 1) & 7], s[c], s[c + 1]);
+            const float mx =
+                fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
+            // a row with no attended column here has the maximum -FLT_MAX
+            m_tile = (mx == -FLT_MAX) ? -INFINITY : mx * cl2;
+          } else {
+            // 128-column tiles are partial only at a band's edges: select
+            // -inf for masked columns, two-input maxima
+            if (!__all_sync(0xffffffffu, full)) {
+              const bool cut_lo = __any_sync(0xffffffffu, c0h > 0), cut_hi = __any_sync(0xffffffffu, c1h < BH - 1);
+              if (cut_lo && cut_hi) {
+#pragma unroll
+                for (int c = 0; c < BH; ++c) s[c] = (c >= c0h && c <= c1h) ? s[c] : -INFINITY;
+              } else if (cut_lo) {
+#pragma unroll
+                for (int c = 0; c < BH; ++c) s[c] = (c >= c0h) ? s[c] : -INFINITY;
+              } else {
+#pragma unroll
+                for (int c = 0; c < BH; ++c) s[c] = (c <= c1h) ? s[c] : -INFINITY;
+              }
+            }
+            float mx8[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) mx8[j] = s[j];
+#pragma unroll
+            for (int c = 8; c < BH; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], s[c]);
+            const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                   fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+            m_tile = mx * cl2;  // -inf stays -inf
           }
-          // row max over 8 independent chains
-          float mx8[8];
-#pragma unroll
-          for (int j = 0; j < 8; ++j) mx8[j] = s[j];
-#pragma unroll
-          for (int c = 8; c < BH; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], s[c]);
-          const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                                 fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-          const float m_tile = mx * cl2;  // -inf stays -inf
           float m_use = m_run, alpha = 1.f;
           bool rescale = false;
           if (m_tile > m_run) {

@@ -29,7 +29,41 @@
 #define SWA_HD inline
 #endif
 
+#include <cstdint>
+
 namespace swa {
+
+// n / d for 0 <= n < 2^31 by a fixed divisor d >= 1, as a multiply-high and
+// a shift (the round-up method: s = ceil(log2 d), m = floor(2^32 (2^s - d) / d)
+// + 1, n / d = (umulhi(n, m) + n) >> s). Built once on the host; the kernels
+// use it for their per-unit index arithmetic, where a runtime division costs
+// tens of instructions.
+struct FastDiv {
+  uint32_t d, m, s;
+  SWA_HD int operator()(int n) const {
+#ifdef __CUDA_ARCH__
+    const uint32_t hi = __umulhi(static_cast<uint32_t>(n), m);
+#else
+    const uint32_t hi = static_cast<uint32_t>((static_cast<uint64_t>(static_cast<uint32_t>(n)) * m) >> 32);
+#endif
+    return static_cast<int>((hi + static_cast<uint32_t>(n)) >> s);
+  }
+};
+
+inline FastDiv make_fastdiv(int d) {
+  FastDiv f;
+  f.d = static_cast<uint32_t>(d < 1 ? 1 : d);
+  f.s = 0;
+  while ((1ull << f.s) < f.d) ++f.s;
+  f.m = static_cast<uint32_t>((((1ull << 32) * ((1ull << f.s) - f.d)) / f.d) + 1);
+  return f;
+}
+
+// Plain division, for the host-side schedule export.
+struct PlainDiv {
+  int d;
+  SWA_HD int operator()(int n) const { return n / d; }
+};
 
 constexpr int kStrideTag = 0x40000000;
 
@@ -42,16 +76,20 @@ SWA_HD int imax(int a, int b) { return a > b ? a : b; }
 SWA_HD int window_lo(int i, int W) { return imax(0, i - W + 1); }
 
 // Number of stride rows m with m*S < lo (keys below the window of a row
-// whose window starts at lo).
-SWA_HD int stride_rows_below(int lo, int S) { return (lo + S - 1) / S; }
+// whose window starts at lo). `div` divides by S.
+template <class Div>
+SWA_HD int stride_rows_below(int lo, int S, Div div) { return lo > 0 ? div(lo - 1) + 1 : 0; }
+SWA_HD int stride_rows_below(int lo, int S) { return stride_rows_below(lo, S, PlainDiv{S}); }
 
 // Extra-view rows attended by a row whose window starts at lo: stride rows
 // below lo (strided), the global keys below lo (global; S carries g).
-SWA_HD int extra_rows_below(int kind, int lo, int S) {
-  if (kind == kMaskStrided && S > 0) return stride_rows_below(lo, S);
+template <class Div>
+SWA_HD int extra_rows_below(int kind, int lo, int S, Div div) {
+  if (kind == kMaskStrided && S > 0) return stride_rows_below(lo, S, div);
   if (kind == kMaskGlobal && S > 0) return imin(S, lo);
   return 0;
 }
+SWA_HD int extra_rows_below(int kind, int lo, int S) { return extra_rows_below(kind, lo, S, PlainDiv{S > 0 ? S : 1}); }
 
 struct QTileKeys {
   int band_lo;   // first window key tile
@@ -65,7 +103,8 @@ struct QTileKeys {
 // last row; every tile in it has an attended cell because consecutive rows'
 // windows overlap or abut. Extra tiles are those with an extra-view row
 // below the last row's lo (the largest lo in the tile).
-SWA_HD QTileKeys qtile_keys(int kind, int N, int W, int S, int Bq, int Bk, int qt) {
+template <class Div>
+SWA_HD QTileKeys qtile_keys(int kind, int N, int W, int S, int Bq, int Bk, int qt, Div div) {
   QTileKeys r;
   const int r0 = qt * Bq;
   const int r1 = imin(N - 1, r0 + Bq - 1);
@@ -74,7 +113,7 @@ SWA_HD QTileKeys qtile_keys(int kind, int N, int W, int S, int Bq, int Bk, int q
   r.band_hi = r1 / Bk;
   r.n_stride = 0;
   if ((kind == kMaskStrided || kind == kMaskGlobal) && S > 0) {
-    const int m = extra_rows_below(kind, window_lo(r1, Wc), S);
+    const int m = extra_rows_below(kind, window_lo(r1, Wc), S, div);
     r.n_stride = (m + Bk - 1) / Bk;
   }
   return r;
@@ -82,7 +121,8 @@ SWA_HD QTileKeys qtile_keys(int kind, int N, int W, int S, int Bq, int Bk, int q
 
 // The same for the window, strided and causal kinds only (no global-token
 // branch), for kernels built without the global kind.
-SWA_HD QTileKeys qtile_keys_basic(int kind, int N, int W, int S, int Bq, int Bk, int qt) {
+template <class Div>
+SWA_HD QTileKeys qtile_keys_basic(int kind, int N, int W, int S, int Bq, int Bk, int qt, Div div) {
   QTileKeys r;
   const int r0 = qt * Bq;
   const int r1 = imin(N - 1, r0 + Bq - 1);
@@ -91,10 +131,14 @@ SWA_HD QTileKeys qtile_keys_basic(int kind, int N, int W, int S, int Bq, int Bk,
   r.band_hi = r1 / Bk;
   r.n_stride = 0;
   if (kind == kMaskStrided && S > 0) {
-    const int m = stride_rows_below(window_lo(r1, Wc), S);
+    const int m = stride_rows_below(window_lo(r1, Wc), S, div);
     r.n_stride = (m + Bk - 1) / Bk;
   }
   return r;
+}
+
+SWA_HD QTileKeys qtile_keys(int kind, int N, int W, int S, int Bq, int Bk, int qt) {
+  return qtile_keys(kind, N, W, S, Bq, Bk, qt, PlainDiv{S > 0 ? S : 1});
 }
 
 SWA_HD int qtile_nkeys(const QTileKeys& k) { return k.n_stride + (k.band_hi - k.band_lo + 1); }

@@ -81,7 +81,9 @@ typedef struct {
  *   o [B,Hq,N,d] bf16 (device, written);
  *   lse [B,Hq,N] fp32 natural-log sum of exp of the scaled scores, or NULL;
  *   d in {64, 128}; W >= 1 (W >= N is full causal); Hq % Hkv == 0;
- *   scale > 0 multiplies Q K^T (1/sqrt(d) for the usual attention). */
+ *   scale multiplies Q K^T (1/sqrt(d) for the usual attention); it must be
+ *   finite and at least 1e-30 (masked scores are carried as -FLT_MAX, and
+ *   this keeps their weights exactly 0). */
 swa_status_t swa_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
                           int B, int Hq, int Hkv, int N, int d, int W, float scale, void* stream);
 
