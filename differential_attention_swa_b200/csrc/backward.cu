@@ -43,6 +43,10 @@ namespace swa {
 namespace {
 
 constexpr int kBwdThreads = 192;  // producer, MMA, four elementwise warps
+// dQ kernel: producer, MMA, then four elementwise warps per 64-key half
+// (warps 2-5 take half 0, warps 6-9 half 1, one lane quarter each), so the
+// halves' elementwise work runs side by side
+constexpr int kDqThreads = 320;
 constexpr int kBT = 128;          // rows of a query or key tile
 
 template <int D>
@@ -58,8 +62,12 @@ struct BwdCfg {
   static constexpr uint32_t kColS = 0;      // S (or S^T), then P / dS as bf16 pairs
   static constexpr uint32_t kColDP = 128;   // dP (or dP^T), then dS^T as bf16 pairs
   static constexpr uint32_t kColAcc = 256;  // dQ, or dV then dK
+  // dQ kernel: Q and dO rows as the score products' A operands (bf16 pairs)
+  static constexpr uint32_t kColQ = 256 + D;
+  static constexpr uint32_t kColDO = kColQ + D / 2;
   static_assert(kSmemBytes <= 227 * 1024, "shared memory");
   static_assert(256 + 2 * D <= 512, "tensor memory");
+  static_assert(kColDO + D / 2 <= 512, "tensor memory (dQ kernel)");
 };
 
 // Each step's score products run as two halves of 64 columns (queries in
@@ -76,6 +84,7 @@ struct BwdBar {
   static constexpr int kP = 7;      // + half: elementwise done, P / dS of the half written
   static constexpr int kAcc = 9;    // accumulators final
   static constexpr int kFinal = 10; // MMA drain on abort
+  static constexpr int kA = 11;     // dQ kernel: Q and dO rows copied into TMEM
   static constexpr int kWordsOff = 256;
 };
 
@@ -457,7 +466,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
 // SM: the local + strided mask (stride tiles before the window tiles).
 template <int D, bool SM>
-__global__ void __launch_bounds__(kBwdThreads, 1)
+__global__ void __launch_bounds__(kDqThreads, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                   const __grid_constant__ CUtensorMap tm_ks, const __grid_constant__ CUtensorMap tm_vs,
@@ -499,6 +508,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     mbar_init(bar(BwdBar::kAcc), 1);
     mbar_init(bar(BwdBar::kFinal), 1);
+    mbar_init(bar(BwdBar::kA), 256);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -553,9 +563,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     if (lane == 0) {
       const uint32_t idesc_s = idesc_bf16_f32(kBT, kBH, false);
       const uint32_t idesc_acc = idesc_bf16_f32(kBT, D, true);
-      const uint64_t q_desc = sw128_desc(sbase + C::kOffA, 16, 1024);
-      const uint64_t do_desc = sw128_desc(sbase + C::kOffB, 16, 1024);
-      bool ok = mbar_wait(bar(BwdBar::kFixed), 0, abort_flag);
+      // the score products take Q and dO from TMEM (copied there once by the
+      // elementwise warps): only the half's K or V tile is read from shared
+      // memory, which an N = 64 product with both operands in shared memory
+      // would be bound by
+      bool ok = mbar_wait(bar(BwdBar::kA), 0, abort_flag);
       if (!ok) bwd_timeout(abort_flag, p.err_flag);
       tc_fence_after();
       // S = Q K^T and dP = dO V^T over keys 64h .. 64h+63 of step s (rows:
@@ -568,8 +580,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint64_t off = (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
-          umma_bf16_ss(tmem + C::kColS + kBH * h, q_desc + off, k_k + off, idesc_s, kk > 0 ? 1u : 0u);
-          umma_bf16_ss(tmem + C::kColDP + kBH * h, do_desc + off, v_k + off, idesc_s, kk > 0 ? 1u : 0u);
+          umma_bf16_ts(tmem + C::kColS + kBH * h, tmem + C::kColQ + kk * 8, k_k + off, idesc_s, kk > 0 ? 1u : 0u);
+          umma_bf16_ts(tmem + C::kColDP + kBH * h, tmem + C::kColDO + kk * 8, v_k + off, idesc_s, kk > 0 ? 1u : 0u);
         }
         umma_commit(bar(BwdBar::kS + h));
       };
@@ -622,6 +634,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   } else {
     // --------------------------------------------------- elementwise ---
     const int qw = warp & 3;
+    const int hh = (warp - 2) >> 2;  // the 64-key half this warp takes
     const int r = qw * 32 + lane;  // query row within the tile
     const int i = qt * kBT + r;
     const uint32_t lane_addr = static_cast<uint32_t>(qw * 32) << 16;
@@ -630,49 +643,77 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const bool rt_ok = SWA_IN(rt, 0, (int64_t)p.B * p.Hq * p.npad, p.err_flag);
     const float lse2 = rt_ok ? p.lse2[rt] : 0.f, dd = rt_ok ? p.dd[rt] : 0.f;
     bool ok = true;
+    {
+      // this row of Q (half-0 warps) or of dO (half-1 warps) into TMEM, the
+      // score products' A operands: column j holds elements 2j and 2j + 1
+      // (low half first), which is the row's own word order; the tiles
+      // arrived with the 128-byte swizzle (16-byte chunk c of row r at chunk
+      // c ^ (r % 8))
+      const bool got = mbar_wait(bar(BwdBar::kFixed), 0, abort_flag);
+      if (!__all_sync(0xffffffffu, got)) {
+        if (lane == 0) bwd_timeout(abort_flag, p.err_flag);
+        ok = false;
+      } else {
+        const uint8_t* tile = smem + (hh ? C::kOffB : C::kOffA);
+        uint32_t w[D / 2];
+#pragma unroll
+        for (int bx = 0; bx < D / 64; ++bx)
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const uint4 v = *reinterpret_cast<const uint4*>(tile + bx * 16384 + r * 128 + ((c ^ (r & 7)) << 4));
+            w[bx * 32 + 4 * c] = v.x;
+            w[bx * 32 + 4 * c + 1] = v.y;
+            w[bx * 32 + 4 * c + 2] = v.z;
+            w[bx * 32 + 4 * c + 3] = v.w;
+          }
+        const uint32_t col = tmem + lane_addr + (hh ? C::kColDO : C::kColQ);
+#pragma unroll
+        for (int j = 0; j < D / 2; j += 32) tmem_st32_u(col + j, w + j);
+        tc_fence_before();
+        mbar_arrive(bar(BwdBar::kA));
+      }
+    }
     for (int s = 0; s < nsteps && ok; ++s) {
       const bool strided = SM && s < nst;
       const int kt = strided ? s : kt_lo + (s - nst);  // strided: compacted stride rows kt*128 ..
-#pragma unroll 1
-      for (int h = 0; h < 2; ++h) {  // two halves of 64 keys, each on its own barriers
-        const bool got = mbar_wait(bar(BwdBar::kS + h), s & 1, abort_flag);
-        if (!__all_sync(0xffffffffu, got)) {
-          if (lane == 0) bwd_timeout(abort_flag, p.err_flag);
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        float sv[64], dp[64];
-        uint32_t pk[32];
-        tmem_ld64(tmem + lane_addr + C::kColS + kBH * h, sv);
-        tmem_ld64(tmem + lane_addr + C::kColDP + kBH * h, dp);
-        auto body = [&](auto attended) {
-#pragma unroll
-          for (int c = 0; c < 64; c += 2) {
-            const int key = kt * kBT + 64 * h + c;  // strided: the compacted index m
-            const bool a0 = attended(key), a1 = attended(key + 1);
-            const float p0 = a0 ? ex2_approx(fmaf(sv[c], sl2, -lse2)) : 0.f;
-            const float p1 = a1 ? ex2_approx(fmaf(sv[c + 1], sl2, -lse2)) : 0.f;
-            pk[c >> 1] = pack_bf16(p0 * (dp[c] - dd), p1 * (dp[c + 1] - dd));
-          }
-        };
-        // every (query, key) cell of this 128 x 64 block attended: no per-cell test
-        const int64_t k_lo = (int64_t)kt * kBT + kBH * h, k_hi = k_lo + kBH - 1;  // strided: compacted indices
-        const int i_lo = qt * kBT, i_hi = i_lo + kBT - 1;
-        const bool full = strided ? (k_hi * p.S < (int64_t)i_lo - p.W + 1 && i_hi < p.N && k_hi * p.S < p.N)
-                                  : (k_hi <= i_lo && i_hi - k_lo < p.W && i_hi < p.N && k_hi < p.N);
-        if (full)
-          body([](int) { return true; });
-        else if (strided)
-          body([&](int m) { return bwd_stride_attended(i, m, p.W, p.S, p.N); });
-        else
-          body([&](int key) { return bwd_attended(i, key, p.W, p.N); });
-        // dS over S as bf16 pairs: the half's 64 keys in its own first 32
-        // columns, already read
-        tmem_st32_u(tmem + lane_addr + C::kColS + kBH * h, pk);
-        tc_fence_before();
-        mbar_arrive(bar(BwdBar::kP + h));
+      const int h = hh;
+      const bool got = mbar_wait(bar(BwdBar::kS + h), s & 1, abort_flag);
+      if (!__all_sync(0xffffffffu, got)) {
+        if (lane == 0) bwd_timeout(abort_flag, p.err_flag);
+        ok = false;
+        break;
       }
+      tc_fence_after();
+      float sv[64], dp[64];
+      uint32_t pk[32];
+      tmem_ld64(tmem + lane_addr + C::kColS + kBH * h, sv);
+      tmem_ld64(tmem + lane_addr + C::kColDP + kBH * h, dp);
+      auto body = [&](auto attended) {
+#pragma unroll
+        for (int c = 0; c < 64; c += 2) {
+          const int key = kt * kBT + 64 * h + c;  // strided: the compacted index m
+          const bool a0 = attended(key), a1 = attended(key + 1);
+          const float p0 = a0 ? ex2_approx(fmaf(sv[c], sl2, -lse2)) : 0.f;
+          const float p1 = a1 ? ex2_approx(fmaf(sv[c + 1], sl2, -lse2)) : 0.f;
+          pk[c >> 1] = pack_bf16(p0 * (dp[c] - dd), p1 * (dp[c + 1] - dd));
+        }
+      };
+      // every (query, key) cell of this 128 x 64 block attended: no per-cell test
+      const int64_t k_lo = (int64_t)kt * kBT + kBH * h, k_hi = k_lo + kBH - 1;  // strided: compacted indices
+      const int i_lo = qt * kBT, i_hi = i_lo + kBT - 1;
+      const bool full = strided ? (k_hi * p.S < (int64_t)i_lo - p.W + 1 && i_hi < p.N && k_hi * p.S < p.N)
+                                : (k_hi <= i_lo && i_hi - k_lo < p.W && i_hi < p.N && k_hi < p.N);
+      if (full)
+        body([](int) { return true; });
+      else if (strided)
+        body([&](int m) { return bwd_stride_attended(i, m, p.W, p.S, p.N); });
+      else
+        body([&](int key) { return bwd_attended(i, key, p.W, p.N); });
+      // dS over S as bf16 pairs: the half's 64 keys in its own first 32
+      // columns, already read
+      tmem_st32_u(tmem + lane_addr + C::kColS + kBH * h, pk);
+      tc_fence_before();
+      mbar_arrive(bar(BwdBar::kP + h));
     }
     if (ok) {
       const bool got = mbar_wait(bar(BwdBar::kAcc), 0, abort_flag);
@@ -681,11 +722,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         ok = false;
       }
     }
-    if (ok) {
+    if (ok) {  // the half's warps write their half of dQ's columns
       tc_fence_after();
       __nv_bfloat16* dq = reinterpret_cast<__nv_bfloat16*>(p.dq) + ((int64_t)(b * p.Hq + hq) * p.N + i) * D;
 #pragma unroll 1
-      for (int c = 0; c < D; c += 32) {
+      for (int c = hh * (D / 2); c < (hh + 1) * (D / 2); c += 32) {
         float a[32];
         tmem_ld32(tmem + lane_addr + C::kColAcc + c, a);
         if (i < p.N && SWA_IN((int64_t)(b * p.Hq + hq) * p.N + i, 0, (int64_t)p.B * p.Hq * p.N, p.err_flag)) {
@@ -738,13 +779,13 @@ cudaError_t launch_bwd_d(const BwdMaps& m, const BwdParams& p, cudaStream_t stre
     bwd_dkdv_kernel<D, 1><<<gk, kBwdThreads, C::kSmemBytes, stream>>>(m.q, m.k, m.v, m.dO, m.ks, m.vs, p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    bwd_dq_kernel<D, true><<<gq, kBwdThreads, C::kSmemBytes, stream>>>(m.q, m.k, m.v, m.dO, m.ks, m.vs, p);
+    bwd_dq_kernel<D, true><<<gq, kDqThreads, C::kSmemBytes, stream>>>(m.q, m.k, m.v, m.dO, m.ks, m.vs, p);
     return cudaGetLastError();
   }
   bwd_dkdv_kernel<D, 0><<<gk, kBwdThreads, C::kSmemBytes, stream>>>(m.q, m.k, m.v, m.dO, m.ks, m.vs, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  bwd_dq_kernel<D, false><<<gq, kBwdThreads, C::kSmemBytes, stream>>>(m.q, m.k, m.v, m.dO, m.ks, m.vs, p);
+  bwd_dq_kernel<D, false><<<gq, kDqThreads, C::kSmemBytes, stream>>>(m.q, m.k, m.v, m.dO, m.ks, m.vs, p);
   return cudaGetLastError();
 }
 
