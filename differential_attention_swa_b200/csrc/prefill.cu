@@ -792,7 +792,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             m_tile = (mx == -FLT_MAX) ? -INFINITY : mx * cl2;
           } else {
             // 128-column tiles are partial only at a band's edges: select
-            // -inf for masked columns, two-input maxima
+            // -inf for masked columns; three-input maxima
             if (!__all_sync(0xffffffffu, full)) {
               const bool cut_lo = __any_sync(0xffffffffu, c0h > 0), cut_hi = __any_sync(0xffffffffu, c1h < BH - 1);
               if (cut_lo && cut_hi) {
@@ -810,9 +810,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int j = 0; j < 8; ++j) mx8[j] = s[j];
 #pragma unroll
-            for (int c = 8; c < BH; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], s[c]);
-            const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                                   fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+            for (int c = 8; c < BH; c += 2) mx8[(c >> 1) & 7] = fmax3(mx8[(c >> 1) & 7], s[c], s[c + 1]);
+            const float mx =
+                fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
             m_tile = mx * cl2;  // -inf stays -inf
           }
           float m_use = m_run, alpha = 1.f;
