@@ -107,6 +107,8 @@ def test_bad_arguments_rejected_before_launch(lib):
     assert st == swa.ERR_INVALID_ARG  # N < 1
     st = lib.swa_attn_fwd(good, good, good, good, None, 1, 2, 2, 256, 64, 4, -1.0, None)
     assert st == swa.ERR_INVALID_ARG  # scale
+    st = lib.swa_attn_fwd(good, good, good, good, None, 1, 2, 2, 256, 64, 4, 1e-31, None)
+    assert st == swa.ERR_INVALID_ARG  # scale below 1e-30: masked weights would no longer be exactly 0
     st = lib.swa_attn_fwd(good, good, good, good, None, 1, 2, 2, 256, 96, 4, 0.1, None)
     assert st == swa.ERR_UNSUPPORTED  # head dim
     st = lib.strided_attn_fwd(good, good, good, good, None, 1, 2, 2, 256, 64, 4, 0, 0.1, None)

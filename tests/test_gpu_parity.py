@@ -246,6 +246,31 @@ def test_diff_small_full(orc, N, W, dv, Hq, Hkv):
     compare(out, ref, "diff")
 
 
+@pytest.mark.parametrize("case", ["lambda0", "same_maps", "window_ragged"])
+def test_diff_degenerate_cases(orc, case):
+    """Differential attention where it reduces to something plainer: lambda = 0
+    is the causal attention of (Q1, K1, V); Q2 = Q1, K2 = K1 gives (1 - lambda)
+    times it ("Attention Variants -- Sliding Window, Sparse, Differential",
+    The Problem: one map subtracted from the other); and a window with a
+    ragged last tile."""
+    N, Hq, Hkv, dv = (200, 2, 2, 128) if case != "window_ragged" else (333, 4, 2, 64)
+    q1, k1, q2, k2, v = diff_inputs(1, Hq, Hkv, N, 64, dv, seed=17)
+    if case == "same_maps":
+        q2, k2 = q1.clone(), k1.clone()
+    lam = torch.zeros(Hq) if case == "lambda0" else torch.tensor([0.25, 0.8, 0.5, 0.1][:Hq])
+    W = 50 if case == "window_ragged" else None
+    out = swa.diff_attn_fwd(*gpu(q1, k1, q2, k2, v), lam.float().cuda(), window=W, scale=0.125)
+    assert swa.last_device_error() == swa.OK
+    ref = orc.diff_attention(q1, k1, q2, k2, v, lam, W=W, scale=0.125)
+    compare(out, ref, f"diff {case}")
+    if case == "lambda0":  # equal to the plain causal attention of (Q1, K1, V), within the same bar
+        plain = orc.attention("causal", q1, k1, v, scale=0.125)
+        compare(out, plain, "diff lambda 0 vs causal attention")
+    if case == "same_maps":
+        plain = orc.attention("causal", q1, k1, v, scale=0.125)
+        compare(out, plain * (1 - lam.numpy().astype(np.float64))[None, :, None, None], "diff same maps")
+
+
 # ---------------------------------------------------------------- decode --
 
 @pytest.mark.parametrize("B,Hq,Hkv,d,W,pos0,T", [(2, 4, 2, 128, 64, 3, 70), (3, 16, 8, 128, 1024, 131072, 3),
