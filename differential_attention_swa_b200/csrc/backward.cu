@@ -219,7 +219,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     // ------------------------------------------------------ producer ---
     if (lane == 0) {
       const int zkv = b * p.Hkv + hkv;
-      const int krows = STRIDE ? (p.N + p.S - 1) / p.S : p.N;  // rows of the stride view, or of K/V
+      const int krows = STRIDE ? (p.N - 1) / p.S + 1 : p.N;  // rows of the stride view, or of K/V
       (void)krows;
       mbar_arrive_expect_tx(bar(BwdBar::kFixed), 2 * C::kTile);
       for (int bx = 0; bx < D / 64; ++bx) {
@@ -542,7 +542,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         const int row = (strided ? s : kt_lo + (s - nst)) * kBT;
         const uint32_t base = sbase + C::kOffStages + st * C::kStage;
         mbar_arrive_expect_tx(bar(BwdBar::kFull + st), 2 * C::kTile);
-        const int krows = strided ? (p.N + p.S - 1) / p.S : p.N;
+        const int krows = strided ? (p.N - 1) / p.S + 1 : p.N;
         (void)krows;
         for (int bx = 0; bx < D / 64; ++bx) {
           if (!SWA_TMA_IN(bx * 64, D, row, krows, zkv, p.B * p.Hkv, p.err_flag)) continue;

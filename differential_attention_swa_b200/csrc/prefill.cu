@@ -390,7 +390,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int row = item_tile(it, u) * BN;
           // rows of the view the tile comes from: the stride view holds
           // ceil(N / S) rows, the global keys' view is K/V itself
-          const int vrows = (st && p.kind == kMaskStrided) ? (p.N + p.S - 1) / p.S : p.N;
+          const int vrows = (st && p.kind == kMaskStrided) ? (p.N - 1) / p.S + 1 : p.N;
           (void)vrows;
           {  // K (or K1 and K2)
             const int slot = L % C::kSlots, use = L / C::kSlots;
