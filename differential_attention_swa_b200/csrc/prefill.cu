@@ -748,6 +748,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           const bool got = mbar_wait(bar(BarLayout::kS + 2 * t + h), kglob & 1, abort_flag);
           if (!__all_sync(0xffffffffu, got)) { if (lane == 0) record_timeout(abort_flag, p.err_flag); ok = false; break; }
           tc_fence_after();
+          if (BH == 64 && __all_sync(0xffffffffu, c1h < c0h || c1h < 0 || c0h > BH - 1)) {
+            // no row of this warp attends a column of this half (a window
+            // edge, the stride view's unused keys, rows past N): P = 0 and
+            // the row max and sum stand, so the scores are not read. (The
+            // 128-column buffers of the d = 128 and differential kernels
+            // meet such a tile only at rows past N: the vote would cost more
+            // than it saves.)
+            uint32_t zero[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) zero[e] = 0u;
+            tmem_st32_u(s_tmem + h * BH, zero);
+            tc_fence_before();
+            mbar_arrive(bar(BarLayout::kP + 2 * t + h));
+            continue;
+          }
 
           float s[BH];
           if (BH == 128) tmem_ld128(s_tmem, s);
