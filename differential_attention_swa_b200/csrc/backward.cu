@@ -93,19 +93,6 @@ __device__ __forceinline__ void bwd_timeout(volatile int* abort_flag, int* err) 
   atomicExch(err, 4 /* SWA_ERR_TIMEOUT */);
 }
 
-// Query rows i of a key-tile / query-tile pair attended under the window:
-// key <= i, i - key < W, both below N.
-__device__ __forceinline__ bool bwd_attended(int i, int key, int W, int N) {
-  return key <= i && i - key < W && i < N && key < N;
-}
-
-// Row i attends the compacted stride key m (key m*S) as an extra key: the key
-// lies below the row's window (m*S < i - W + 1), both below N.
-__device__ __forceinline__ bool bwd_stride_attended(int i, int m, int W, int S, int N) {
-  const int64_t key = (int64_t)m * S;
-  return key < (int64_t)i - W + 1 && i < N && key < N;
-}
-
 // D_i = dO_i . O_i and L_i * log2(e), rows past N padded with zeros.
 template <int D>
 __global__ void __launch_bounds__(128) bwd_prep_kernel(const BwdParams p) {
@@ -341,11 +328,25 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int key = kt * kBT + kr;       // (STRIDE: the compacted index m; the key is m * S)
     const uint32_t lane_addr = static_cast<uint32_t>(qw * 32) << 16;
     const float sl2 = p.scale_log2;
+    // query rows [ilo, ihi] that attend this lane's key (empty: ilo > ihi):
+    // the window's rows key .. key + W - 1, or, for the stride key m*S, every
+    // row whose window starts after it (m*S < i - W + 1, i.e. i >= m*S + W);
+    // rows below N
+    int ilo, ihi;
+    if constexpr (STRIDE) {
+      const int64_t first = (int64_t)key * p.S + Wc;
+      ilo = (int)(first < p.N ? first : p.N);
+      ihi = p.N - 1;
+    } else {
+      const int64_t last = (int64_t)key + Wc - 1;
+      ilo = key;
+      ihi = key < p.N ? (int)(last < p.N - 1 ? last : p.N - 1) : -1;
+    }
     bool ok = true;
     for (int s = 0; s < nsteps && ok; ++s) {
       const int qt = qt_lo + s % nqt;
-      const float* lse2 = reinterpret_cast<const float*>(smem + C::kOffStages + (s & 1) * C::kStage + 2 * C::kTile);
-      const float* dd = lse2 + kBT;
+      // the step's row tables: L * log2(e), then D, 128 floats each
+      const uint32_t tables = sbase + C::kOffStages + (s & 1) * C::kStage + 2 * C::kTile;
 #pragma unroll 1
       for (int h = 0; h < 2; ++h) {  // two halves of 64 queries, each on its own barriers
         const bool got = mbar_wait(bar(BwdBar::kS + h), s & 1, abort_flag);
@@ -359,37 +360,45 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           break;
         }
         tc_fence_after();
-        float sv[64], dp[64];
+        const int c_lo = ilo - (qt * kBT + kBH * h), c_hi = ihi - (qt * kBT + kBH * h);  // attended columns
+        const uint32_t s_col = tmem + lane_addr + C::kColS + kBH * h;
+        const uint32_t dp_col = tmem + lane_addr + C::kColDP + kBH * h;
         uint32_t pk[32], dk[32];
-        tmem_ld64(tmem + lane_addr + C::kColS + kBH * h, sv);
-        tmem_ld64(tmem + lane_addr + C::kColDP + kBH * h, dp);
-        auto body = [&](auto attended) {
+        if (__all_sync(0xffffffffu, c_hi < 0 || c_lo > kBH - 1 || c_lo > c_hi)) {
+          // no query of this half attends a key of this warp: P^T = dS^T = 0,
+          // the scores are not read
 #pragma unroll
-          for (int c = 0; c < 64; c += 2) {
-            const int c0 = 64 * h + c;
-            const int i0 = qt * kBT + c0;
-            const bool a0 = attended(i0), a1 = attended(i0 + 1);
-            const float p0 = a0 ? ex2_approx(fmaf(sv[c], sl2, -lse2[c0])) : 0.f;
-            const float p1 = a1 ? ex2_approx(fmaf(sv[c + 1], sl2, -lse2[c0 + 1])) : 0.f;
-            pk[c >> 1] = pack_bf16(p0, p1);
-            dk[c >> 1] = pack_bf16(p0 * (dp[c] - dd[c0]), p1 * (dp[c + 1] - dd[c0 + 1]));
-          }
-        };
-        if constexpr (STRIDE) {
-          body([&](int i) { return bwd_stride_attended(i, key, p.W, p.S, p.N); });
+          for (int e = 0; e < 32; ++e) pk[e] = dk[e] = 0u;
         } else {
-          // every (key, query) cell of this 128 x 64 block attended: no per-cell test
-          const int i_lo = qt * kBT + kBH * h, i_hi = i_lo + kBH - 1;
-          const int k_hi = kt * kBT + kBT - 1;
-          if (k_hi <= i_lo && i_hi - kt * kBT < p.W && i_hi < p.N && k_hi < p.N)
+          float sv[64], dp[64];
+          tmem_ld64(s_col, sv);
+          tmem_ld64(dp_col, dp);
+          const uint32_t tab = tables + 4 * kBH * h;  // the half's rows (same for every lane)
+          auto body = [&](auto attended) {
+#pragma unroll
+            for (int c = 0; c < 64; c += 4) {
+              const float4 l4 = ld_shared_f4(tab + 4 * c), d4 = ld_shared_f4(tab + 4 * kBT + 4 * c);
+              const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dv[4] = {d4.x, d4.y, d4.z, d4.w};
+#pragma unroll
+              for (int e = 0; e < 4; e += 2) {
+                const bool a0 = attended(c + e), a1 = attended(c + e + 1);
+                const float p0 = a0 ? ex2_approx(fmaf(sv[c + e], sl2, -lv[e])) : 0.f;
+                const float p1 = a1 ? ex2_approx(fmaf(sv[c + e + 1], sl2, -lv[e + 1])) : 0.f;
+                pk[(c + e) >> 1] = pack_bf16(p0, p1);
+                dk[(c + e) >> 1] = pack_bf16(p0 * (dp[c + e] - dv[e]), p1 * (dp[c + e + 1] - dv[e + 1]));
+              }
+            }
+          };
+          // every (key, query) cell of the warp's 32 x 64 block attended: no per-cell test
+          if (__all_sync(0xffffffffu, c_lo <= 0 && c_hi >= kBH - 1))
             body([](int) { return true; });
           else
-            body([&](int i) { return bwd_attended(i, key, p.W, p.N); });
+            body([&](int c) { return c >= c_lo && c <= c_hi; });
         }
         // P^T over S^T and dS^T over dP^T as bf16 pairs: the half's 64
         // queries land in its own first 32 columns, already read
-        tmem_st32_u(tmem + lane_addr + C::kColS + kBH * h, pk);
-        tmem_st32_u(tmem + lane_addr + C::kColDP + kBH * h, dk);
+        tmem_st32_u(s_col, pk);
+        tmem_st32_u(dp_col, dk);
         tc_fence_before();
         mbar_arrive(bar(BwdBar::kP + h));
       }
@@ -642,6 +651,14 @@ __global__ void __launch_bounds__(kDqThreads, 1)
     const int64_t rt = (int64_t)(b * p.Hq + hq) * p.npad + i;  // padded: always in bounds
     const bool rt_ok = SWA_IN(rt, 0, (int64_t)p.B * p.Hq * p.npad, p.err_flag);
     const float lse2 = rt_ok ? p.lse2[rt] : 0.f, dd = rt_ok ? p.dd[rt] : 0.f;
+    // keys this row attends: the window's [wlo, whi], and the compacted
+    // stride keys m < mst (those below the window start); none past N
+    int wlo = 1, whi = 0, mst = 0;
+    if (i < p.N) {
+      wlo = imax(0, i - Wc + 1);
+      whi = i;
+      if (SM) mst = stride_rows_below(wlo, p.S);
+    }
     bool ok = true;
     {
       // this row of Q (half-0 warps) or of dO (half-1 warps) into TMEM, the
@@ -684,34 +701,37 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         break;
       }
       tc_fence_after();
-      float sv[64], dp[64];
+      const int kb = kt * kBT + kBH * h;  // the half's first key (strided: compacted index)
+      const int c_lo = (strided ? 0 : wlo) - kb, c_hi = (strided ? mst - 1 : whi) - kb;  // attended columns
+      const uint32_t s_col = tmem + lane_addr + C::kColS + kBH * h;
       uint32_t pk[32];
-      tmem_ld64(tmem + lane_addr + C::kColS + kBH * h, sv);
-      tmem_ld64(tmem + lane_addr + C::kColDP + kBH * h, dp);
-      auto body = [&](auto attended) {
+      if (__all_sync(0xffffffffu, c_hi < 0 || c_lo > kBH - 1 || c_lo > c_hi)) {
+        // no row of this warp attends a key of this half: dS = 0, the scores
+        // are not read
 #pragma unroll
-        for (int c = 0; c < 64; c += 2) {
-          const int key = kt * kBT + 64 * h + c;  // strided: the compacted index m
-          const bool a0 = attended(key), a1 = attended(key + 1);
-          const float p0 = a0 ? ex2_approx(fmaf(sv[c], sl2, -lse2)) : 0.f;
-          const float p1 = a1 ? ex2_approx(fmaf(sv[c + 1], sl2, -lse2)) : 0.f;
-          pk[c >> 1] = pack_bf16(p0 * (dp[c] - dd), p1 * (dp[c + 1] - dd));
-        }
-      };
-      // every (query, key) cell of this 128 x 64 block attended: no per-cell test
-      const int64_t k_lo = (int64_t)kt * kBT + kBH * h, k_hi = k_lo + kBH - 1;  // strided: compacted indices
-      const int i_lo = qt * kBT, i_hi = i_lo + kBT - 1;
-      const bool full = strided ? (k_hi * p.S < (int64_t)i_lo - p.W + 1 && i_hi < p.N && k_hi * p.S < p.N)
-                                : (k_hi <= i_lo && i_hi - k_lo < p.W && i_hi < p.N && k_hi < p.N);
-      if (full)
-        body([](int) { return true; });
-      else if (strided)
-        body([&](int m) { return bwd_stride_attended(i, m, p.W, p.S, p.N); });
-      else
-        body([&](int key) { return bwd_attended(i, key, p.W, p.N); });
+        for (int e = 0; e < 32; ++e) pk[e] = 0u;
+      } else {
+        float sv[64], dp[64];
+        tmem_ld64(s_col, sv);
+        tmem_ld64(tmem + lane_addr + C::kColDP + kBH * h, dp);
+        auto body = [&](auto attended) {
+#pragma unroll
+          for (int c = 0; c < 64; c += 2) {
+            const bool a0 = attended(c), a1 = attended(c + 1);
+            const float p0 = a0 ? ex2_approx(fmaf(sv[c], sl2, -lse2)) : 0.f;
+            const float p1 = a1 ? ex2_approx(fmaf(sv[c + 1], sl2, -lse2)) : 0.f;
+            pk[c >> 1] = pack_bf16(p0 * (dp[c] - dd), p1 * (dp[c + 1] - dd));
+          }
+        };
+        // every (query, key) cell of the warp's 32 x 64 block attended: no per-cell test
+        if (__all_sync(0xffffffffu, c_lo <= 0 && c_hi >= kBH - 1))
+          body([](int) { return true; });
+        else
+          body([&](int c) { return c >= c_lo && c <= c_hi; });
+      }
       // dS over S as bf16 pairs: the half's 64 keys in its own first 32
       // columns, already read
-      tmem_st32_u(tmem + lane_addr + C::kColS + kBH * h, pk);
+      tmem_st32_u(s_col, pk);
       tc_fence_before();
       mbar_arrive(bar(BwdBar::kP + h));
     }
