@@ -93,6 +93,14 @@ __device__ __forceinline__ void bwd_timeout(volatile int* abort_flag, int* err) 
   atomicExch(err, 4 /* SWA_ERR_TIMEOUT */);
 }
 
+// Four consecutive floats from shared memory (16-byte aligned address).
+// Volatile: it stays after the barrier wait that makes the data visible.
+__device__ __forceinline__ float4 ld_shared_f4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
+  return v;
+}
+
 // D_i = dO_i . O_i and L_i * log2(e), rows past N padded with zeros.
 template <int D>
 __global__ void __launch_bounds__(128) bwd_prep_kernel(const BwdParams p) {
