@@ -47,6 +47,7 @@ PROFILES = {
     "diff_causal": ("prefill_diff_causal.md", PREFILL_SOURCES),
     "local_strided_prefill": ("prefill_strided_local.md", PREFILL_SOURCES),
     "mistral_swa_backward": ("backward_swa_mistral.md", BWD_SOURCES),
+    "local_strided_backward": ("backward_strided_local.md", BWD_SOURCES),
     "gemma_swa_decode": ("decode_gemma.md", DECODE_SOURCES),
     "diff_gqa_decode": ("decode_diff_gqa.md", DIFF_DECODE_SOURCES),
 }
@@ -357,6 +358,15 @@ def prefill_kernel_name(w) -> str:
     return f"prefill_kernel<{w.d},{w.d}{gen}{pairs}>"
 
 
+def launches_per_step(w) -> int:
+    """Kernels one step of a workload launches: the persistent prefill kernel,
+    or the backward's row-statistics pass, the stride keys' dK/dV pass (local
+    + strided mask only), the dK/dV kernel and the dQ kernel."""
+    if w.kind == "swa_bwd":
+        return 3 + (1 if w.S else 0)
+    return 1
+
+
 def measure_ours(args, rank, world, peaks, peak_src, dist):
     import torch
 
@@ -406,7 +416,7 @@ def measure_ours(args, rank, world, peaks, peak_src, dist):
                      else "fallback 1.59 PFLOP/s",
                      "kernel": prefill_kernel_name(w)},
         "clocks": clk,
-        "gpu_launches": args.steps,
+        "gpu_launches": args.steps * launches_per_step(w),
     }
     if not args.no_e2e and out is not None:  # the backward workload has no single output to copy back
         res["e2e"] = whole_job_e2e(measure_e2e(call, ins, out, flops, stream), flops, world, dist, "cuda")

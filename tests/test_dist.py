@@ -78,3 +78,33 @@ def test_single_rank_e2e_record():
     assert e2e["ms_per_step"] == 4.3624 and abs(e2e["value"] - round(824.7e9 / 4.36237e-3 / 1e12, 3)) < 1e-9
     assert e2e["h2d_bytes_per_step"] == 201326592 and e2e["d2h_bytes_per_step"] == 134217728
     assert "ms_raw" not in e2e and e2e["unit"] == "TFLOP/s"
+
+
+def test_launches_per_step():
+    import bench
+    from differential_attention_swa_b200.inputs import WORKLOADS
+
+    # one persistent prefill kernel; the backward's row statistics, stride
+    # pass (local + strided only), dK/dV and dQ kernels
+    assert bench.launches_per_step(WORKLOADS["mistral_swa_prefill"]) == 1
+    assert bench.launches_per_step(WORKLOADS["local_strided_prefill"]) == 1
+    assert bench.launches_per_step(WORKLOADS["mistral_swa_backward"]) == 3
+    assert bench.launches_per_step(WORKLOADS["local_strided_backward"]) == 4
+
+
+def test_profiled_traffic_tracks_sources(tmp_path, monkeypatch):
+    import bench
+
+    # a summary counts only while the kernel's sources hash to what it records
+    src = tmp_path / "k.cu"
+    src.write_text("kernel v1")
+    (tmp_path / "profiles").mkdir()
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    h = bench.source_hash(["k.cu"])
+    (tmp_path / "profiles" / "k.md").write_text(f"dram_bytes_per_launch: 12345\nsource_sha256_16: {h}\n")
+    assert bench.profiled_traffic("k.md", ["k.cu"]) == 12345
+    src.write_text("kernel v2")
+    assert bench.profiled_traffic("k.md", ["k.cu"]) is None
+    assert bench.profiled_traffic("missing.md", ["k.cu"]) is None
+    for name, (summary, sources) in bench.PROFILES.items():  # every listed summary exists
+        assert os.path.exists(os.path.join(os.path.dirname(os.path.dirname(__file__)), "profiles", summary)), name
