@@ -101,6 +101,13 @@ __device__ __forceinline__ float4 ld_shared_f4(uint32_t addr) {
   return v;
 }
 
+// p[0..3] += (a, b, c, d) as one relaxed device-scope reduction (p 16-byte
+// aligned): a quarter of the atomic operations of four scalar adds.
+__device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
+  asm volatile("red.relaxed.gpu.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d)
+               : "memory");
+}
+
 // D_i = dO_i . O_i and L_i * log2(e), rows past N padded with zeros.
 template <int D>
 __global__ void __launch_bounds__(128) bwd_prep_kernel(const BwdParams p) {
@@ -429,9 +436,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           tmem_ld32(tmem + lane_addr + C::kColAcc + c, a);
           tmem_ld32(tmem + lane_addr + C::kColAcc + D + c, g);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            atomicAdd(p.sdv + row + c + e, a[e]);
-            atomicAdd(p.sdk + row + c + e, g[e]);
+          for (int e = 0; e < 32; e += 4) {
+            red_add_v4(p.sdv + row + c + e, a[e], a[e + 1], a[e + 2], a[e + 3]);
+            red_add_v4(p.sdk + row + c + e, g[e], g[e + 1], g[e + 2], g[e + 3]);
           }
         }
       }
