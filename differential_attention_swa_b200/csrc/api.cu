@@ -296,6 +296,8 @@ swa_status_t run_bwd(const void* q, const void* k, const void* v, const void* o,
   p.sdv = S > 0 ? p.sdk + (int64_t)B * Hkv * nspad * d : nullptr;
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
+  p.num_ctas = sm_count();
+  if (p.num_ctas < 1) return SWA_ERR_CUDA;
   p.err_flag = device_error_ptr();
   if (p.err_flag == nullptr) return SWA_ERR_CUDA;
   cudaError_t e = launch_backward(m, p, d, static_cast<cudaStream_t>(stream));

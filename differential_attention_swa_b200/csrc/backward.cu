@@ -54,19 +54,25 @@ struct BwdCfg {
   static constexpr int kTile = kBT * D * 2;              // one tile of D bf16 columns
   static constexpr int kStage = 2 * kTile + 2 * kBT * 4; // two tiles + two fp32 row tables
   static constexpr int kStages = 2;
-  static constexpr int kOffA = 0;                        // the CTA's fixed tiles
+  // the dK/dV kernel at d = 64 runs several key tiles per CTA: two sets of
+  // its fixed K and V tiles (the next tile's load overlaps this tile's
+  // steps) and of its TMEM accumulators (the second in the 128 columns one
+  // set leaves free), so a tile's epilogue overlaps the next tile's steps
+  static constexpr int kFixedSets = D == 64 ? 2 : 1;
+  static constexpr int kOffA = 0;                        // the CTA's fixed tiles (set f: + f * 2 * kTile)
   static constexpr int kOffB = kTile;
-  static constexpr int kOffStages = 2 * kTile;
+  static constexpr int kOffStages = 2 * kTile * kFixedSets;
   static constexpr int kOffBar = kOffStages + kStages * kStage;
   static constexpr int kSmemBytes = kOffBar + 1024 + 1024;  // barriers area + alignment slack
   static constexpr uint32_t kColS = 0;      // S (or S^T), then P / dS as bf16 pairs
   static constexpr uint32_t kColDP = 128;   // dP (or dP^T), then dS^T as bf16 pairs
-  static constexpr uint32_t kColAcc = 256;  // dQ, or dV then dK
+  static constexpr uint32_t kColAcc = 256;  // dQ, or dV then dK (set f: + f * kAccSet)
+  static constexpr uint32_t kAccSet = 2 * D;
   // dQ kernel: Q and dO rows as the score products' A operands (bf16 pairs)
   static constexpr uint32_t kColQ = 256 + D;
   static constexpr uint32_t kColDO = kColQ + D / 2;
   static_assert(kSmemBytes <= 227 * 1024, "shared memory");
-  static_assert(256 + 2 * D <= 512, "tensor memory");
+  static_assert(256 + kFixedSets * 2 * D <= 512, "tensor memory");
   static_assert(kColDO + D / 2 <= 512, "tensor memory (dQ kernel)");
 };
 
@@ -77,15 +83,18 @@ struct BwdCfg {
 constexpr int kBH = 64;  // columns of a half
 
 struct BwdBar {
-  static constexpr int kFixed = 0;
-  static constexpr int kFull = 1;   // + stage
-  static constexpr int kEmpty = 3;  // + stage
-  static constexpr int kS = 5;      // + half: score products of the half in TMEM
-  static constexpr int kP = 7;      // + half: elementwise done, P / dS of the half written
-  static constexpr int kAcc = 9;    // accumulators final
-  static constexpr int kFinal = 10; // MMA drain on abort
-  static constexpr int kA = 11;     // dQ kernel: Q and dO rows copied into TMEM
+  static constexpr int kFixed = 0;      // + set: the fixed tiles landed
+  static constexpr int kFull = 2;       // + stage
+  static constexpr int kEmpty = 4;      // + stage
+  static constexpr int kS = 6;          // + half: score products of the half in TMEM
+  static constexpr int kP = 8;          // + half: elementwise done, P / dS of the half written
+  static constexpr int kAcc = 10;       // + set: accumulators final
+  static constexpr int kFinal = 12;     // MMA drain on abort
+  static constexpr int kA = 13;         // dQ kernel: Q and dO rows copied into TMEM
+  static constexpr int kFixedFree = 14; // + set: the set's fixed tiles no longer read (multi-tile dK/dV)
+  static constexpr int kAccFree = 16;   // + set: the set's accumulators read out (multi-tile dK/dV)
   static constexpr int kWordsOff = 256;
+  static_assert(18 * 8 <= kWordsOff, "barrier block");
 };
 
 __device__ __forceinline__ void bwd_timeout(volatile int* abort_flag, int* err) {
@@ -160,6 +169,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     const __grid_constant__ CUtensorMap tm_ks, const __grid_constant__ CUtensorMap tm_vs,
                     const __grid_constant__ BwdParams p) {
   using C = BwdCfg<D>;
+  constexpr bool MULTI = C::kFixedSets == 2;  // several key tiles per CTA
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -169,32 +179,54 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(words + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  const int b = blockIdx.y / p.Hkv, hkv = blockIdx.y % p.Hkv;
-  // query tiles that see keys kt*128 .. kt*128+127: from the diagonal up to
-  // the last row whose window still reaches the tile's last key
   constexpr bool STRIDE = MODE == 2;
   const int Wc = imin(p.W, p.N);
-  int qt_lo, qt_hi;
-  int kt = blockIdx.x;
-  if (STRIDE) {
-    // row i has stride key m below its window iff m * S < i - W + 1
-    const int nchunk = (p.nq + kStrideChunk - 1) / kStrideChunk;
-    kt = blockIdx.x / nchunk;
-    const int chunk = blockIdx.x % nchunk;
-    const int64_t first = (int64_t)kt * kBT * p.S + Wc;  // first row that sees m = kt * 128
-    const int q0 = (int)(first < p.N ? first / kBT : p.nq);
-    qt_lo = q0 + chunk * kStrideChunk;
-    qt_hi = imin(p.nq - 1, qt_lo + kStrideChunk - 1);  // empty when past the last tile
-  } else {
-    qt_lo = kt;
-    const int reach = kt * kBT + kBT - 1 + Wc - 1;  // last query row that sees the tile's last key
-    qt_hi = imin(p.nq - 1, reach / kBT);
-  }
-  const int nqt = qt_hi - qt_lo + 1;
-  const int nsteps = nqt > 0 ? p.G * nqt : 0;
+  // Work tiles in one linear order: column x = key tile (stride pass: stride
+  // tile and chunk of query tiles), row y = b * Hkv + hkv. The CTA takes
+  // the tile of its grid cell, or (multi-tile) every gridDim.x-th tile from
+  // blockIdx.x; every role walks the same list.
+  const int nchunk = STRIDE ? (p.nq + kStrideChunk - 1) / kStrideChunk : 1;
+  const int ncol = STRIDE ? p.nspad / kBT * nchunk : p.nq;
+  const int ntiles = ncol * p.B * p.Hkv;
+  const int t_first = MULTI ? (int)blockIdx.x : (int)(blockIdx.y * ncol + blockIdx.x);
+  const int t_step = MULTI ? (int)gridDim.x : ntiles;
+  struct Tile {
+    int b, hkv, kt, qt_lo, nqt, nsteps;
+  };
+  // query tiles that see keys kt*128 .. kt*128+127: from the diagonal up to
+  // the last row whose window still reaches the tile's last key
+  auto tile_of = [&](int t) -> Tile {
+    Tile w;
+    const int x = t % ncol, y = t / ncol;
+    w.b = y / p.Hkv;
+    w.hkv = y % p.Hkv;
+    int qt_hi;
+    if (STRIDE) {
+      // row i has stride key m below its window iff m * S < i - W + 1
+      w.kt = x / nchunk;
+      const int chunk = x % nchunk;
+      const int64_t first = (int64_t)w.kt * kBT * p.S + Wc;  // first row that sees m = kt * 128
+      const int q0 = (int)(first < p.N ? first / kBT : p.nq);
+      w.qt_lo = q0 + chunk * kStrideChunk;
+      qt_hi = imin(p.nq - 1, w.qt_lo + kStrideChunk - 1);  // empty when past the last tile
+    } else {
+      w.kt = x;
+      w.qt_lo = x;
+      const int reach = x * kBT + kBT - 1 + Wc - 1;  // last query row that sees the tile's last key
+      qt_hi = imin(p.nq - 1, reach / kBT);
+    }
+    w.nqt = qt_hi - w.qt_lo + 1;
+    w.nsteps = w.nqt > 0 ? p.G * w.nqt : 0;
+    return w;
+  };
 
   if (threadIdx.x == 0) {
-    mbar_init(bar(BwdBar::kFixed), 1);
+    for (int f = 0; f < 2; ++f) {
+      mbar_init(bar(BwdBar::kFixed + f), 1);
+      mbar_init(bar(BwdBar::kAcc + f), 1);
+      mbar_init(bar(BwdBar::kFixedFree + f), 1);
+      mbar_init(bar(BwdBar::kAccFree + f), 128);
+    }
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(bar(BwdBar::kFull + s), 1);
       mbar_init(bar(BwdBar::kEmpty + s), 1);
@@ -203,7 +235,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(bar(BwdBar::kS + h), 1);
       mbar_init(bar(BwdBar::kP + h), 128);
     }
-    mbar_init(bar(BwdBar::kAcc), 1);
     mbar_init(bar(BwdBar::kFinal), 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -220,42 +251,61 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------ producer ---
     if (lane == 0) {
-      const int zkv = b * p.Hkv + hkv;
-      const int krows = STRIDE ? (p.N - 1) / p.S + 1 : p.N;  // rows of the stride view, or of K/V
-      (void)krows;
-      mbar_arrive_expect_tx(bar(BwdBar::kFixed), 2 * C::kTile);
-      for (int bx = 0; bx < D / 64; ++bx) {
-        if (!SWA_TMA_IN(bx * 64, D, kt * kBT, krows, zkv, p.B * p.Hkv, p.err_flag)) continue;
-        tma_load_3d(sbase + C::kOffA + bx * 16384, STRIDE ? &tm_ks : &tm_k, bar(BwdBar::kFixed), bx * 64, kt * kBT,
-                    zkv);
-        tma_load_3d(sbase + C::kOffB + bx * 16384, STRIDE ? &tm_vs : &tm_v, bar(BwdBar::kFixed), bx * 64, kt * kBT,
-                    zkv);
-      }
       int issued[C::kStages] = {0, 0};
-      for (int s = 0; s < nsteps; ++s) {
-        const int st = s & 1, use = s >> 1;
-        if (use > 0 && !mbar_wait(bar(BwdBar::kEmpty + st), (use - 1) & 1, abort_flag)) {
+      int fixed_issued[2] = {0, 0};
+      int g = 0;   // steps, across the CTA's tiles (stage ring)
+      int jj = 0;  // non-empty tiles (fixed-tile sets)
+      bool ok = true;
+      for (int t = t_first; t < ntiles && ok; t += t_step) {
+        const Tile w = tile_of(t);
+        if (w.nsteps == 0) continue;
+        const int fs = MULTI ? (jj & 1) : 0, fuse = MULTI ? (jj >> 1) : jj;
+        ++jj;
+        // the set's K and V are free once the tile before last has run its scores
+        if (fuse > 0 && !mbar_wait(bar(BwdBar::kFixedFree + fs), (fuse - 1) & 1, abort_flag)) {
           bwd_timeout(abort_flag, p.err_flag);
           break;
         }
-        const int hq = hkv * p.G + s / nqt, qt = qt_lo + s % nqt;
-        const int zq = b * p.Hq + hq;
-        const uint32_t base = sbase + C::kOffStages + st * C::kStage;
-        mbar_arrive_expect_tx(bar(BwdBar::kFull + st), 2 * C::kTile + 2 * kBT * 4);
+        const int zkv = w.b * p.Hkv + w.hkv;
+        const int krows = STRIDE ? (p.N - 1) / p.S + 1 : p.N;  // rows of the stride view, or of K/V
+        (void)krows;
+        const uint32_t set_off = fs * 2 * C::kTile;
+        mbar_arrive_expect_tx(bar(BwdBar::kFixed + fs), 2 * C::kTile);
         for (int bx = 0; bx < D / 64; ++bx) {
-          if (!SWA_TMA_IN(bx * 64, D, qt * kBT, p.N, zq, p.B * p.Hq, p.err_flag)) continue;
-          tma_load_3d(base + bx * 16384, &tm_q, bar(BwdBar::kFull + st), bx * 64, qt * kBT, zq);
-          tma_load_3d(base + C::kTile + bx * 16384, &tm_do, bar(BwdBar::kFull + st), bx * 64, qt * kBT, zq);
+          if (!SWA_TMA_IN(bx * 64, D, w.kt * kBT, krows, zkv, p.B * p.Hkv, p.err_flag)) continue;
+          tma_load_3d(sbase + C::kOffA + set_off + bx * 16384, STRIDE ? &tm_ks : &tm_k, bar(BwdBar::kFixed + fs),
+                      bx * 64, w.kt * kBT, zkv);
+          tma_load_3d(sbase + C::kOffB + set_off + bx * 16384, STRIDE ? &tm_vs : &tm_v, bar(BwdBar::kFixed + fs),
+                      bx * 64, w.kt * kBT, zkv);
         }
-        const int64_t rt = (int64_t)zq * p.npad + qt * kBT;
-        if (SWA_IN(rt, 0, (int64_t)p.B * p.Hq * p.npad - kBT + 1, p.err_flag)) {
-          bulk_load(base + 2 * C::kTile, p.lse2 + rt, kBT * 4, bar(BwdBar::kFull + st));
-          bulk_load(base + 2 * C::kTile + kBT * 4, p.dd + rt, kBT * 4, bar(BwdBar::kFull + st));
+        fixed_issued[fs] = fuse + 1;
+        for (int s = 0; s < w.nsteps; ++s, ++g) {
+          const int st = g & 1, use = g >> 1;
+          if (use > 0 && !mbar_wait(bar(BwdBar::kEmpty + st), (use - 1) & 1, abort_flag)) {
+            bwd_timeout(abort_flag, p.err_flag);
+            ok = false;
+            break;
+          }
+          const int hq = w.hkv * p.G + s / w.nqt, qt = w.qt_lo + s % w.nqt;
+          const int zq = w.b * p.Hq + hq;
+          const uint32_t base = sbase + C::kOffStages + st * C::kStage;
+          mbar_arrive_expect_tx(bar(BwdBar::kFull + st), 2 * C::kTile + 2 * kBT * 4);
+          for (int bx = 0; bx < D / 64; ++bx) {
+            if (!SWA_TMA_IN(bx * 64, D, qt * kBT, p.N, zq, p.B * p.Hq, p.err_flag)) continue;
+            tma_load_3d(base + bx * 16384, &tm_q, bar(BwdBar::kFull + st), bx * 64, qt * kBT, zq);
+            tma_load_3d(base + C::kTile + bx * 16384, &tm_do, bar(BwdBar::kFull + st), bx * 64, qt * kBT, zq);
+          }
+          const int64_t rt = (int64_t)zq * p.npad + qt * kBT;
+          if (SWA_IN(rt, 0, (int64_t)p.B * p.Hq * p.npad - kBT + 1, p.err_flag)) {
+            bulk_load(base + 2 * C::kTile, p.lse2 + rt, kBT * 4, bar(BwdBar::kFull + st));
+            bulk_load(base + 2 * C::kTile + kBT * 4, p.dd + rt, kBT * 4, bar(BwdBar::kFull + st));
+          }
+          issued[st] = use + 1;
         }
-        issued[st] = use + 1;
       }
       if (*abort_flag) {  // drain: every copy issued lands before the CTA may exit
-        mbar_wait_timed(bar(BwdBar::kFixed), 0);
+        for (int f = 0; f < 2; ++f)
+          if (fixed_issued[f] > 0) mbar_wait_timed(bar(BwdBar::kFixed + f), (fixed_issued[f] - 1) & 1);
         for (int st = 0; st < C::kStages; ++st)
           if (issued[st] > 0) mbar_wait_timed(bar(BwdBar::kFull + st), (issued[st] - 1) & 1);
       }
@@ -265,72 +315,95 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     if (lane == 0) {
       const uint32_t idesc_s = idesc_bf16_f32(kBT, kBH, false);
       const uint32_t idesc_acc = idesc_bf16_f32(kBT, D, true);
-      const uint64_t k_desc = sw128_desc(sbase + C::kOffA, 16, 1024);
-      const uint64_t v_desc = sw128_desc(sbase + C::kOffB, 16, 1024);
-      bool ok = mbar_wait(bar(BwdBar::kFixed), 0, abort_flag);
-      if (!ok) bwd_timeout(abort_flag, p.err_flag);
-      tc_fence_after();
-      // S^T = K Q^T and dP^T = V dO^T of queries 64h .. 64h+63 of step s
-      // (rows: keys, columns: queries; the half's Q and dO rows start 64
-      // rows = 8192 bytes into each 64-column box)
-      auto scores = [&](int s, int h) {
-        const uint32_t cur = sbase + C::kOffStages + (s & 1) * C::kStage + h * 8192;
-        const uint64_t q_k = sw128_desc(cur, 16, 1024);
-        const uint64_t do_k = sw128_desc(cur + C::kTile, 16, 1024);
+      bool ok = true;
+      int g = 0, jj = 0;
+      for (int t = t_first; t < ntiles && ok; t += t_step) {
+        const Tile w = tile_of(t);
+        if (w.nsteps == 0) continue;
+        const int fs = MULTI ? (jj & 1) : 0, fuse = MULTI ? (jj >> 1) : jj;
+        ++jj;
+        const uint32_t set_off = fs * 2 * C::kTile;
+        const uint64_t k_desc = sw128_desc(sbase + C::kOffA + set_off, 16, 1024);
+        const uint64_t v_desc = sw128_desc(sbase + C::kOffB + set_off, 16, 1024);
+        const uint32_t acc_col = C::kColAcc + fs * C::kAccSet;
+        if (!mbar_wait(bar(BwdBar::kFixed + fs), fuse & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        // the set's accumulators: read out by the epilogue of the tile before last
+        if (fuse > 0 && !mbar_wait(bar(BwdBar::kAccFree + fs), (fuse - 1) & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        // S^T = K Q^T and dP^T = V dO^T of queries 64h .. 64h+63 of step gs
+        // (rows: keys, columns: queries; the half's Q and dO rows start 64
+        // rows = 8192 bytes into each 64-column box)
+        auto scores = [&](int gs, int h) {
+          const uint32_t cur = sbase + C::kOffStages + (gs & 1) * C::kStage + h * 8192;
+          const uint64_t q_k = sw128_desc(cur, 16, 1024);
+          const uint64_t do_k = sw128_desc(cur + C::kTile, 16, 1024);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t off = (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
-          umma_bf16_ss(tmem + C::kColS + kBH * h, k_desc + off, q_k + off, idesc_s, kk > 0 ? 1u : 0u);
-          umma_bf16_ss(tmem + C::kColDP + kBH * h, v_desc + off, do_k + off, idesc_s, kk > 0 ? 1u : 0u);
-        }
-        umma_commit(bar(BwdBar::kS + h));
-      };
-      // dV += P^T dO and dK += dS^T Q over the half's 64 queries (P^T, dS^T
-      // as bf16 pairs in the half's first 32 columns)
-      auto accumulate = [&](int s, int h) {
-        const uint32_t cur = sbase + C::kOffStages + (s & 1) * C::kStage;
-        const uint64_t q_mn = sw128_desc(cur, 16384, 1024);
-        const uint64_t do_mn = sw128_desc(cur + C::kTile, 16384, 1024);
-#pragma unroll
-        for (int kk = 0; kk < kBH / 16; ++kk) {
-          const uint32_t acc = (s == 0 && h == 0 && kk == 0) ? 0u : 1u;
-          const uint64_t row = (uint64_t)(((kBH / 16) * h + kk) * 2048 >> 4);
-          umma_bf16_ts(tmem + C::kColAcc, tmem + C::kColS + kBH * h + kk * 8, do_mn + row, idesc_acc, acc);
-          umma_bf16_ts(tmem + C::kColAcc + D, tmem + C::kColDP + kBH * h + kk * 8, q_mn + row, idesc_acc, acc);
-        }
-      };
-      if (ok && nsteps > 0) {
-        ok = mbar_wait(bar(BwdBar::kFull), 0, abort_flag);
-        if (ok) {
-          tc_fence_after();
-          scores(0, 0);
-          scores(0, 1);
-        }
-      }
-      for (int s = 0; ok && s < nsteps; ++s) {
-        for (int h = 0; h < 2 && ok; ++h) {
-          if (!mbar_wait(bar(BwdBar::kP + h), s & 1, abort_flag)) {
-            ok = false;
-            break;
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t off = (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
+            umma_bf16_ss(tmem + C::kColS + kBH * h, k_desc + off, q_k + off, idesc_s, kk > 0 ? 1u : 0u);
+            umma_bf16_ss(tmem + C::kColDP + kBH * h, v_desc + off, do_k + off, idesc_s, kk > 0 ? 1u : 0u);
           }
-          tc_fence_after();
-          accumulate(s, h);
-          if (h == 1) umma_commit(bar(BwdBar::kEmpty + (s & 1)));  // Q, dO and the row tables of step s read
-          if (s + 1 < nsteps) {
-            if (h == 0) {
-              if (!mbar_wait(bar(BwdBar::kFull + ((s + 1) & 1)), ((s + 1) >> 1) & 1, abort_flag)) {
-                ok = false;
-                break;
-              }
-              tc_fence_after();
+          umma_commit(bar(BwdBar::kS + h));
+        };
+        // dV += P^T dO and dK += dS^T Q over the half's 64 queries (P^T, dS^T
+        // as bf16 pairs in the half's first 32 columns); the tile's first
+        // product overwrites the set's accumulators
+        auto accumulate = [&](int gs, bool first, int h) {
+          const uint32_t cur = sbase + C::kOffStages + (gs & 1) * C::kStage;
+          const uint64_t q_mn = sw128_desc(cur, 16384, 1024);
+          const uint64_t do_mn = sw128_desc(cur + C::kTile, 16384, 1024);
+#pragma unroll
+          for (int kk = 0; kk < kBH / 16; ++kk) {
+            const uint32_t acc = (first && h == 0 && kk == 0) ? 0u : 1u;
+            const uint64_t row = (uint64_t)(((kBH / 16) * h + kk) * 2048 >> 4);
+            umma_bf16_ts(tmem + acc_col, tmem + C::kColS + kBH * h + kk * 8, do_mn + row, idesc_acc, acc);
+            umma_bf16_ts(tmem + acc_col + D, tmem + C::kColDP + kBH * h + kk * 8, q_mn + row, idesc_acc, acc);
+          }
+        };
+        const int g0 = g;  // the tile's first step
+        if (!mbar_wait(bar(BwdBar::kFull + (g0 & 1)), (g0 >> 1) & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        scores(g0, 0);
+        scores(g0, 1);
+        for (int s = 0; ok && s < w.nsteps; ++s) {
+          const int gs = g0 + s;
+          for (int h = 0; h < 2 && ok; ++h) {
+            if (!mbar_wait(bar(BwdBar::kP + h), gs & 1, abort_flag)) {
+              ok = false;
+              break;
             }
-            // into the columns the accumulation above reads first (MMAs run in issue order)
-            scores(s + 1, h);
+            tc_fence_after();
+            accumulate(gs, s == 0, h);
+            if (h == 1) umma_commit(bar(BwdBar::kEmpty + (gs & 1)));  // Q, dO and the row tables of the step read
+            if (s + 1 < w.nsteps) {
+              if (h == 0) {
+                if (!mbar_wait(bar(BwdBar::kFull + ((gs + 1) & 1)), ((gs + 1) >> 1) & 1, abort_flag)) {
+                  ok = false;
+                  break;
+                }
+                tc_fence_after();
+              }
+              // into the columns the accumulation above reads first (MMAs run in issue order)
+              scores(gs + 1, h);
+            }
           }
         }
+        g = g0 + w.nsteps;
+        if (ok) {
+          umma_commit(bar(BwdBar::kAcc + fs));                    // the tile's dV and dK final
+          if (MULTI) umma_commit(bar(BwdBar::kFixedFree + fs));  // its K and V read by every score product
+        }
       }
-      if (ok) umma_commit(bar(BwdBar::kAcc));
-      else bwd_timeout(abort_flag, p.err_flag);
+      if (!ok) bwd_timeout(abort_flag, p.err_flag);
       if (!ok || *abort_flag) {
         umma_commit(bar(BwdBar::kFinal));
         mbar_wait_timed(bar(BwdBar::kFinal), 0);
@@ -340,141 +413,152 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     // --------------------------------------------------- elementwise ---
     const int qw = warp & 3;             // TMEM lane quarter
     const int kr = qw * 32 + lane;       // key row within the tile
-    const int key = kt * kBT + kr;       // (STRIDE: the compacted index m; the key is m * S)
     const uint32_t lane_addr = static_cast<uint32_t>(qw * 32) << 16;
     const float sl2 = p.scale_log2;
-    // query rows [ilo, ihi] that attend this lane's key (empty: ilo > ihi):
-    // the window's rows key .. key + W - 1, or, for the stride key m*S, every
-    // row whose window starts after it (m*S < i - W + 1, i.e. i >= m*S + W);
-    // rows below N
-    int ilo, ihi;
-    if constexpr (STRIDE) {
-      const int64_t first = (int64_t)key * p.S + Wc;
-      ilo = (int)(first < p.N ? first : p.N);
-      ihi = p.N - 1;
-    } else {
-      const int64_t last = (int64_t)key + Wc - 1;
-      ilo = key;
-      ihi = key < p.N ? (int)(last < p.N - 1 ? last : p.N - 1) : -1;
-    }
     bool ok = true;
-    for (int s = 0; s < nsteps && ok; ++s) {
-      const int qt = qt_lo + s % nqt;
-      // the step's row tables: L * log2(e), then D, 128 floats each
-      const uint32_t tables = sbase + C::kOffStages + (s & 1) * C::kStage + 2 * C::kTile;
+    int g = 0, jj = 0;
+    for (int t = t_first; t < ntiles && ok; t += t_step) {
+      const Tile w = tile_of(t);
+      if (w.nsteps == 0) continue;
+      const int fs = MULTI ? (jj & 1) : 0, fuse = MULTI ? (jj >> 1) : jj;
+      ++jj;
+      const uint32_t acc_col = C::kColAcc + fs * C::kAccSet;
+      const int key = w.kt * kBT + kr;  // (STRIDE: the compacted index m; the key is m * S)
+      // query rows [ilo, ihi] that attend this lane's key (empty: ilo > ihi):
+      // the window's rows key .. key + W - 1, or, for the stride key m*S, every
+      // row whose window starts after it (m*S < i - W + 1, i.e. i >= m*S + W);
+      // rows below N
+      int ilo, ihi;
+      if constexpr (STRIDE) {
+        const int64_t first = (int64_t)key * p.S + Wc;
+        ilo = (int)(first < p.N ? first : p.N);
+        ihi = p.N - 1;
+      } else {
+        const int64_t last = (int64_t)key + Wc - 1;
+        ilo = key;
+        ihi = key < p.N ? (int)(last < p.N - 1 ? last : p.N - 1) : -1;
+      }
+      for (int s = 0; s < w.nsteps && ok; ++s, ++g) {
+        const int qt = w.qt_lo + s % w.nqt;
+        // the step's row tables: L * log2(e), then D, 128 floats each
+        const uint32_t tables = sbase + C::kOffStages + (g & 1) * C::kStage + 2 * C::kTile;
 #pragma unroll 1
-      for (int h = 0; h < 2; ++h) {  // two halves of 64 queries, each on its own barriers
-        const bool got = mbar_wait(bar(BwdBar::kS + h), s & 1, abort_flag);
-        // the row tables were written by the copy engine: acquire them from
-        // the stage's own barrier (complete already; the stage cannot be
-        // refilled before this step's P^T and dS^T are consumed)
-        const bool have = got && (h == 1 || mbar_wait(bar(BwdBar::kFull + (s & 1)), (s >> 1) & 1, abort_flag));
-        if (!__all_sync(0xffffffffu, have)) {
+        for (int h = 0; h < 2; ++h) {  // two halves of 64 queries, each on its own barriers
+          const bool got = mbar_wait(bar(BwdBar::kS + h), g & 1, abort_flag);
+          // the row tables were written by the copy engine: acquire them from
+          // the stage's own barrier (complete already; the stage cannot be
+          // refilled before this step's P^T and dS^T are consumed)
+          const bool have = got && (h == 1 || mbar_wait(bar(BwdBar::kFull + (g & 1)), (g >> 1) & 1, abort_flag));
+          if (!__all_sync(0xffffffffu, have)) {
+            if (lane == 0) bwd_timeout(abort_flag, p.err_flag);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const int c_lo = ilo - (qt * kBT + kBH * h), c_hi = ihi - (qt * kBT + kBH * h);  // attended columns
+          const uint32_t s_col = tmem + lane_addr + C::kColS + kBH * h;
+          const uint32_t dp_col = tmem + lane_addr + C::kColDP + kBH * h;
+          uint32_t pk[32], dk[32];
+          if (__all_sync(0xffffffffu, c_hi < 0 || c_lo > kBH - 1 || c_lo > c_hi)) {
+            // no query of this half attends a key of this warp: P^T = dS^T = 0,
+            // the scores are not read
+#pragma unroll
+            for (int e = 0; e < 32; ++e) pk[e] = dk[e] = 0u;
+          } else {
+            float sv[64], dp[64];
+            tmem_ld64(s_col, sv);
+            tmem_ld64(dp_col, dp);
+            const uint32_t tab = tables + 4 * kBH * h;  // the half's rows (same for every lane)
+            auto body = [&](auto attended) {
+#pragma unroll
+              for (int c = 0; c < 64; c += 4) {
+                const float4 l4 = ld_shared_f4(tab + 4 * c), d4 = ld_shared_f4(tab + 4 * kBT + 4 * c);
+                const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dv[4] = {d4.x, d4.y, d4.z, d4.w};
+#pragma unroll
+                for (int e = 0; e < 4; e += 2) {
+                  const bool a0 = attended(c + e), a1 = attended(c + e + 1);
+                  const float p0 = a0 ? ex2_approx(fmaf(sv[c + e], sl2, -lv[e])) : 0.f;
+                  const float p1 = a1 ? ex2_approx(fmaf(sv[c + e + 1], sl2, -lv[e + 1])) : 0.f;
+                  pk[(c + e) >> 1] = pack_bf16(p0, p1);
+                  dk[(c + e) >> 1] = pack_bf16(p0 * (dp[c + e] - dv[e]), p1 * (dp[c + e + 1] - dv[e + 1]));
+                }
+              }
+            };
+            // every (key, query) cell of the warp's 32 x 64 block attended: no per-cell test
+            if (__all_sync(0xffffffffu, c_lo <= 0 && c_hi >= kBH - 1))
+              body([](int) { return true; });
+            else
+              body([&](int c) { return c >= c_lo && c <= c_hi; });
+          }
+          // P^T over S^T and dS^T over dP^T as bf16 pairs: the half's 64
+          // queries land in its own first 32 columns, already read
+          tmem_st32_u(s_col, pk);
+          tmem_st32_u(dp_col, dk);
+          tc_fence_before();
+          mbar_arrive(bar(BwdBar::kP + h));
+        }
+      }
+      if (!ok) break;
+      {
+        const bool got = mbar_wait(bar(BwdBar::kAcc + fs), fuse & 1, abort_flag);
+        if (!__all_sync(0xffffffffu, got)) {
           if (lane == 0) bwd_timeout(abort_flag, p.err_flag);
           ok = false;
-          break;
         }
-        tc_fence_after();
-        const int c_lo = ilo - (qt * kBT + kBH * h), c_hi = ihi - (qt * kBT + kBH * h);  // attended columns
-        const uint32_t s_col = tmem + lane_addr + C::kColS + kBH * h;
-        const uint32_t dp_col = tmem + lane_addr + C::kColDP + kBH * h;
-        uint32_t pk[32], dk[32];
-        if (__all_sync(0xffffffffu, c_hi < 0 || c_lo > kBH - 1 || c_lo > c_hi)) {
-          // no query of this half attends a key of this warp: P^T = dS^T = 0,
-          // the scores are not read
-#pragma unroll
-          for (int e = 0; e < 32; ++e) pk[e] = dk[e] = 0u;
-        } else {
-          float sv[64], dp[64];
-          tmem_ld64(s_col, sv);
-          tmem_ld64(dp_col, dp);
-          const uint32_t tab = tables + 4 * kBH * h;  // the half's rows (same for every lane)
-          auto body = [&](auto attended) {
-#pragma unroll
-            for (int c = 0; c < 64; c += 4) {
-              const float4 l4 = ld_shared_f4(tab + 4 * c), d4 = ld_shared_f4(tab + 4 * kBT + 4 * c);
-              const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dv[4] = {d4.x, d4.y, d4.z, d4.w};
-#pragma unroll
-              for (int e = 0; e < 4; e += 2) {
-                const bool a0 = attended(c + e), a1 = attended(c + e + 1);
-                const float p0 = a0 ? ex2_approx(fmaf(sv[c + e], sl2, -lv[e])) : 0.f;
-                const float p1 = a1 ? ex2_approx(fmaf(sv[c + e + 1], sl2, -lv[e + 1])) : 0.f;
-                pk[(c + e) >> 1] = pack_bf16(p0, p1);
-                dk[(c + e) >> 1] = pack_bf16(p0 * (dp[c + e] - dv[e]), p1 * (dp[c + e + 1] - dv[e + 1]));
-              }
-            }
-          };
-          // every (key, query) cell of the warp's 32 x 64 block attended: no per-cell test
-          if (__all_sync(0xffffffffu, c_lo <= 0 && c_hi >= kBH - 1))
-            body([](int) { return true; });
-          else
-            body([&](int c) { return c >= c_lo && c <= c_hi; });
-        }
-        // P^T over S^T and dS^T over dP^T as bf16 pairs: the half's 64
-        // queries land in its own first 32 columns, already read
-        tmem_st32_u(s_col, pk);
-        tmem_st32_u(dp_col, dk);
-        tc_fence_before();
-        mbar_arrive(bar(BwdBar::kP + h));
       }
-    }
-    if (ok) {
-      const bool got = mbar_wait(bar(BwdBar::kAcc), 0, abort_flag);
-      if (!__all_sync(0xffffffffu, got)) {
-        if (lane == 0) bwd_timeout(abort_flag, p.err_flag);
-        ok = false;
-      }
-    }
-    if (ok && STRIDE) {
-      // this chunk's fp32 partials of the stride keys, added to the others'
-      if (nsteps > 0) {
+      if (ok && STRIDE) {
+        // this chunk's fp32 partials of the stride keys, added to the others'
         tc_fence_after();
-        const int64_t row = ((int64_t)(b * p.Hkv + hkv) * p.nspad + key) * D;
+        const int64_t row = ((int64_t)(w.b * p.Hkv + w.hkv) * p.nspad + key) * D;
 #pragma unroll 1
         for (int c = 0; c < D && SWA_IN(row, 0, (int64_t)p.B * p.Hkv * p.nspad * D - D + 1, p.err_flag); c += 32) {
-          float a[32], g[32];
-          tmem_ld32(tmem + lane_addr + C::kColAcc + c, a);
-          tmem_ld32(tmem + lane_addr + C::kColAcc + D + c, g);
+          float a[32], gk[32];
+          tmem_ld32(tmem + lane_addr + acc_col + c, a);
+          tmem_ld32(tmem + lane_addr + acc_col + D + c, gk);
 #pragma unroll
           for (int e = 0; e < 32; e += 4) {
             red_add_v4(p.sdv + row + c + e, a[e], a[e + 1], a[e + 2], a[e + 3]);
-            red_add_v4(p.sdk + row + c + e, g[e], g[e + 1], g[e + 2], g[e + 3]);
+            red_add_v4(p.sdk + row + c + e, gk[e], gk[e + 1], gk[e + 2], gk[e + 3]);
+          }
+        }
+      } else if (ok) {
+        tc_fence_after();
+        const int64_t row = ((int64_t)(w.b * p.Hkv + w.hkv) * p.N + key) * D;
+        __nv_bfloat16* dv = reinterpret_cast<__nv_bfloat16*>(p.dv) + row;
+        __nv_bfloat16* dkp = reinterpret_cast<__nv_bfloat16*>(p.dk) + row;
+        // a stride key also gets the stride pass's partials before the one rounding
+        const bool add = MODE == 1 && key < p.N && key % p.S == 0;
+        const int64_t srow = ((int64_t)(w.b * p.Hkv + w.hkv) * p.nspad + (add ? key / p.S : 0)) * D;
+        const bool in_rows = key >= p.N || SWA_IN(row, 0, (int64_t)p.B * p.Hkv * p.N * D - D + 1, p.err_flag);
+        const bool in_srow = !add || SWA_IN(srow, 0, (int64_t)p.B * p.Hkv * p.nspad * D - D + 1, p.err_flag);
+#pragma unroll 1
+        for (int c = 0; c < D; c += 32) {
+          float a[32], gk[32];
+          tmem_ld32(tmem + lane_addr + acc_col + c, a);
+          tmem_ld32(tmem + lane_addr + acc_col + D + c, gk);
+          if (add && in_srow) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              a[e] += p.sdv[srow + c + e];
+              gk[e] += p.sdk[srow + c + e];
+            }
+          }
+          if (key < p.N && in_rows) {
+#pragma unroll
+            for (int e = 0; e < 32; e += 8) {
+              st_global_v4(dv + c + e, pack_bf16(a[e], a[e + 1]), pack_bf16(a[e + 2], a[e + 3]),
+                           pack_bf16(a[e + 4], a[e + 5]), pack_bf16(a[e + 6], a[e + 7]));
+              st_global_v4(dkp + c + e, pack_bf16(gk[e] * p.scale, gk[e + 1] * p.scale),
+                           pack_bf16(gk[e + 2] * p.scale, gk[e + 3] * p.scale),
+                           pack_bf16(gk[e + 4] * p.scale, gk[e + 5] * p.scale),
+                           pack_bf16(gk[e + 6] * p.scale, gk[e + 7] * p.scale));
+            }
           }
         }
       }
-    } else if (ok) {
-      tc_fence_after();
-      const int64_t row = ((int64_t)(b * p.Hkv + hkv) * p.N + key) * D;
-      __nv_bfloat16* dv = reinterpret_cast<__nv_bfloat16*>(p.dv) + row;
-      __nv_bfloat16* dkp = reinterpret_cast<__nv_bfloat16*>(p.dk) + row;
-      // a stride key also gets the stride pass's partials before the one rounding
-      const bool add = MODE == 1 && key < p.N && key % p.S == 0;
-      const int64_t srow = ((int64_t)(b * p.Hkv + hkv) * p.nspad + (add ? key / p.S : 0)) * D;
-      const bool in_rows = key >= p.N || SWA_IN(row, 0, (int64_t)p.B * p.Hkv * p.N * D - D + 1, p.err_flag);
-      const bool in_srow = !add || SWA_IN(srow, 0, (int64_t)p.B * p.Hkv * p.nspad * D - D + 1, p.err_flag);
-#pragma unroll 1
-      for (int c = 0; c < D; c += 32) {
-        float a[32], g[32];
-        tmem_ld32(tmem + lane_addr + C::kColAcc + c, a);
-        tmem_ld32(tmem + lane_addr + C::kColAcc + D + c, g);
-        if (add && in_srow) {
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            a[e] += p.sdv[srow + c + e];
-            g[e] += p.sdk[srow + c + e];
-          }
-        }
-        if (key < p.N && in_rows) {
-#pragma unroll
-          for (int e = 0; e < 32; e += 8) {
-            st_global_v4(dv + c + e, pack_bf16(a[e], a[e + 1]), pack_bf16(a[e + 2], a[e + 3]),
-                         pack_bf16(a[e + 4], a[e + 5]), pack_bf16(a[e + 6], a[e + 7]));
-            st_global_v4(dkp + c + e, pack_bf16(g[e] * p.scale, g[e + 1] * p.scale),
-                         pack_bf16(g[e + 2] * p.scale, g[e + 3] * p.scale),
-                         pack_bf16(g[e + 4] * p.scale, g[e + 5] * p.scale),
-                         pack_bf16(g[e + 6] * p.scale, g[e + 7] * p.scale));
-          }
-        }
+      if (MULTI && ok) {  // the set's accumulators read: a later tile may overwrite them
+        tc_fence_before();
+        mbar_arrive(bar(BwdBar::kAccFree + fs));
       }
     }
   }
@@ -804,20 +888,28 @@ cudaError_t launch_bwd_d(const BwdMaps& m, const BwdParams& p, cudaStream_t stre
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int nk = p.nq;  // key tiles of 128 (same count as query tiles)
-  const dim3 gk(nk, p.B * p.Hkv), gq(p.nq, p.B * p.Hq);
+  const dim3 gq(p.nq, p.B * p.Hq);
+  // dK/dV grid over ncol x (B * Hkv) work tiles: a CTA per tile, or, when
+  // the kernel runs several tiles per CTA, one CTA per SM
+  auto dkdv_grid = [&](int ncol) -> dim3 {
+    if (C::kFixedSets == 1) return dim3(ncol, p.B * p.Hkv);
+    const int64_t ntiles = (int64_t)ncol * p.B * p.Hkv;
+    return dim3((unsigned)(ntiles < p.num_ctas ? ntiles : p.num_ctas));
+  };
   if (p.S > 0) {  // stride keys first: their partials feed the window pass
     const int nchunk = (p.nq + kStrideChunk - 1) / kStrideChunk;
-    bwd_dkdv_kernel<D, 2><<<dim3(p.nspad / kBT * nchunk, p.B * p.Hkv), kBwdThreads, C::kSmemBytes, stream>>>(
+    bwd_dkdv_kernel<D, 2><<<dkdv_grid(p.nspad / kBT * nchunk), kBwdThreads, C::kSmemBytes, stream>>>(
         m.q, m.k, m.v, m.dO, m.ks, m.vs, p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    bwd_dkdv_kernel<D, 1><<<gk, kBwdThreads, C::kSmemBytes, stream>>>(m.q, m.k, m.v, m.dO, m.ks, m.vs, p);
+    bwd_dkdv_kernel<D, 1><<<dkdv_grid(nk), kBwdThreads, C::kSmemBytes, stream>>>(m.q, m.k, m.v, m.dO, m.ks, m.vs,
+                                                                                    p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     bwd_dq_kernel<D, true><<<gq, kDqThreads, C::kSmemBytes, stream>>>(m.q, m.k, m.v, m.dO, m.ks, m.vs, p);
     return cudaGetLastError();
   }
-  bwd_dkdv_kernel<D, 0><<<gk, kBwdThreads, C::kSmemBytes, stream>>>(m.q, m.k, m.v, m.dO, m.ks, m.vs, p);
+  bwd_dkdv_kernel<D, 0><<<dkdv_grid(nk), kBwdThreads, C::kSmemBytes, stream>>>(m.q, m.k, m.v, m.dO, m.ks, m.vs, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   bwd_dq_kernel<D, false><<<gq, kDqThreads, C::kSmemBytes, stream>>>(m.q, m.k, m.v, m.dO, m.ks, m.vs, p);

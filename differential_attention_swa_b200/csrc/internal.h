@@ -55,6 +55,7 @@ struct BwdParams {
   int B, Hq, Hkv, N, W, G, nq, npad;
   int S, nspad;      // stride (0: window mask only), compacted stride rows padded to tiles
   float scale, scale_log2;
+  int num_ctas;      // SMs of the device: the multi-tile dK/dV grid
   int* err_flag;
 };
 struct BwdMaps {
