@@ -101,3 +101,34 @@ def test_strided_backward_vs_oracle(orc, B, Hq, Hkv, N, d, W, S):
         compare_grad(dq.reshape(-1, d)[torch.from_numpy(qr).cuda()], rq, "dq rows")
         compare_grad(dk.reshape(-1, d)[torch.from_numpy(kr).cuda()], rk, "dk rows")
         compare_grad(dv.reshape(-1, d)[torch.from_numpy(kr).cuda()], rv, "dv rows")
+
+
+def _sampled_rows_check(orc, kind, B, Hq, Hkv, N, d, W, S, seed):
+    (q, k, v, d_o), (dq, dk, dv) = run(B, Hq, Hkv, N, d, W, seed=seed, S=S)
+    rng = np.random.default_rng(seed)
+    # dK/dV rows from every (batch, KV head): the first, last and a few inner
+    # keys of each (stride keys among them), plus random ones
+    keys = [0, 127, 133, 2 * 128 + 64, N // 2 + 77, N - 1] + ([S, 7 * S] if S else [])
+    kr = np.unique(np.concatenate([[y * N + key for y in range(B * Hkv) for key in keys],
+                                   rng.integers(0, B * Hkv * N, 24)]))
+    qr = np.unique(np.concatenate([rng.integers(0, B * Hq * N, 24), [0, N - 1, (B * Hq - 1) * N + 5]]))
+    rq, rk, rv = orc.attention_bwd(kind, q, k, v, d_o, W=W, S=S, scale=1 / math.sqrt(d), dq_rows=qr, dkv_rows=kr)
+    compare_grad(dq.reshape(-1, d)[torch.from_numpy(qr).cuda()], rq, "dq rows")
+    compare_grad(dk.reshape(-1, d)[torch.from_numpy(kr).cuda()], rk, "dk rows")
+    compare_grad(dv.reshape(-1, d)[torch.from_numpy(kr).cuda()], rv, "dv rows")
+
+
+def test_backward_multi_tile_sets_reused(orc):
+    """At d = 64 the dK/dV kernel runs several key tiles per CTA (one CTA per
+    SM, two sets of fixed K/V tiles and of accumulators): 2 x 4 KV heads x 64
+    key tiles = 512 tiles give every CTA three or four, so each set is
+    refilled and its accumulators overwritten after an epilogue. Window 96
+    (cut tiles at both edges), GQA group 2."""
+    _sampled_rows_check(orc, "swa", 2, 8, 4, 8192, 64, 96, 0, seed=21)
+
+
+def test_strided_backward_multi_tile_sets_reused(orc):
+    """The same multi-tile dK/dV path with the local + strided mask: the
+    window pass's 512 tiles add the stride pass's fp32 partials to their
+    stride keys (every 64th key) before rounding."""
+    _sampled_rows_check(orc, "strided", 2, 8, 4, 8192, 64, 64, 64, seed=22)
