@@ -132,3 +132,10 @@ def test_strided_backward_multi_tile_sets_reused(orc):
     window pass's 512 tiles add the stride pass's fp32 partials to their
     stride keys (every 64th key) before rounding."""
     _sampled_rows_check(orc, "strided", 2, 8, 4, 8192, 64, 64, 64, seed=22)
+
+
+def test_backward_multi_tile_odd_step_counts(orc):
+    """Group 1 and W = 300: a key tile has one to four query-tile steps, so
+    the stage ring and the half-step barriers run on across tiles at odd as
+    well as even alignments (2 x 8 KV heads x 32 key tiles = 512 tiles)."""
+    _sampled_rows_check(orc, "swa", 2, 8, 8, 4096, 64, 300, 0, seed=23)
