@@ -117,37 +117,46 @@ __device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, 
                : "memory");
 }
 
-// D_i = dO_i . O_i and L_i * log2(e), rows past N padded with zeros.
+// D_i = dO_i . O_i and L_i * log2(e), rows past N padded with zeros. Each
+// row is read by D / 8 lanes, 16 bytes of O and of dO each (a warp's loads
+// cover consecutive rows whole), whose partial dot products meet through
+// shuffles within the row's lane group.
+constexpr int kPrepThreads = 256;
 template <int D>
-__global__ void __launch_bounds__(128) bwd_prep_kernel(const BwdParams p) {
-  const int64_t r = (int64_t)blockIdx.x * 128 + threadIdx.x;  // (b*Hq + hq) * npad + i
+__global__ void __launch_bounds__(kPrepThreads) bwd_prep_kernel(const BwdParams p) {
+  constexpr int LPR = D / 8;               // lanes per row
+  constexpr int RPB = kPrepThreads / LPR;  // rows per block
   const int64_t total = (int64_t)p.B * p.Hq * p.npad;
-  if (r >= total) return;
-  const int64_t bh = r / p.npad;
-  const int i = (int)(r % p.npad);
-  float d = 0.f, l2 = 0.f;
+  const int64_t r = (int64_t)blockIdx.x * RPB + threadIdx.x / LPR;  // (b*Hq + hq) * npad + i
+  const int e = threadIdx.x % LPR;
+  const bool valid = r < total;  // every lane stays for the shuffles
+  const int64_t bh = valid ? r / p.npad : 0;
+  const int i = valid ? (int)(r % p.npad) : p.N;
+  const int64_t row = bh * p.N + i;
+  float d = 0.f;
   if (i < p.N) {
-    const int64_t row = bh * p.N + i;
-    const uint4* o = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(p.o) + row * D);
-    const uint4* g = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(p.dO) + row * D);
-#pragma unroll 4
-    for (int c = 0; c < D / 8; ++c) {
-      const uint4 a = o[c], b = g[c];
-      const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w};
+    const uint4 a = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(p.o) + row * D)[e];
+    const uint4 b = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(p.dO) + row * D)[e];
+    const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        d = fmaf(__uint_as_float(wa[e] << 16), __uint_as_float(wb[e] << 16), d);
-        d = fmaf(__uint_as_float(wa[e] & 0xffff0000u), __uint_as_float(wb[e] & 0xffff0000u), d);
-      }
+    for (int k = 0; k < 4; ++k) {
+      d = fmaf(__uint_as_float(wa[k] << 16), __uint_as_float(wb[k] << 16), d);
+      d = fmaf(__uint_as_float(wa[k] & 0xffff0000u), __uint_as_float(wb[k] & 0xffff0000u), d);
     }
-    if (SWA_IN(row, 0, (int64_t)p.B * p.Hq * p.N, p.err_flag)) l2 = p.lse[row] * 1.4426950408889634f;
   }
-  p.dd[r] = d;
-  p.lse2[r] = l2;
+#pragma unroll
+  for (int off = LPR / 2; off > 0; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
+  if (valid && e == 0) {
+    float l2 = 0.f;
+    if (i < p.N && SWA_IN(row, 0, (int64_t)p.B * p.Hq * p.N, p.err_flag)) l2 = p.lse[row] * 1.4426950408889634f;
+    p.dd[r] = d;
+    p.lse2[r] = l2;
+  }
   // the stride pass adds its partials into zeroed memory
   if (p.S > 0) {
     const int64_t nz = (int64_t)p.B * p.Hkv * p.nspad * D;
-    for (int64_t z = r; z < nz; z += total) {
+    const int64_t nthreads = (int64_t)gridDim.x * kPrepThreads;
+    for (int64_t z = (int64_t)blockIdx.x * kPrepThreads + threadIdx.x; z < nz; z += nthreads) {
       p.sdk[z] = 0.f;
       p.sdv[z] = 0.f;
     }
@@ -884,7 +893,8 @@ cudaError_t launch_bwd_d(const BwdMaps& m, const BwdParams& p, cudaStream_t stre
     }
   }
   const int64_t rows = (int64_t)p.B * p.Hq * p.npad;
-  bwd_prep_kernel<D><<<(unsigned)((rows + 127) / 128), 128, 0, stream>>>(p);
+  constexpr int kPrepRows = kPrepThreads / (D / 8);
+  bwd_prep_kernel<D><<<(unsigned)((rows + kPrepRows - 1) / kPrepRows), kPrepThreads, 0, stream>>>(p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int nk = p.nq;  // key tiles of 128 (same count as query tiles)
