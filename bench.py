@@ -592,6 +592,8 @@ def cpu_baseline(min_seconds=10.0):
 def run_reference(args):
     """The reference arm: the fp64 oracle as it stands on the host cores."""
     import oracle
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
     from differential_attention_swa_b200.inputs import WORKLOADS, attn_inputs
 
     w = WORKLOADS["mistral_swa_prefill"]
@@ -611,8 +613,12 @@ def run_reference(args):
             "warmup": max(3, args.warmup), "ms_per_step": round(1e3 * total / args.steps, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic N(0,1) bf16 widened to fp64",
+            # the config of this arm's comparison line: the same as the GPU
+            # arm's for the same launch (what the oracle actually ran is in
+            # cpu_baseline.sample)
             "config": {"workload": "mistral_swa_prefill", "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d,
-                       "W": w.W, "S": w.S, "parallelism": "host threads"},
+                       "W": w.W, "S": w.S, "parallelism": f"dp{world} (independent batches)",
+                       "l2": "flushed between steps"},
             "impl": "reference",
             "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": oracle.default_threads(),
                              "kind": "oracle", "sample": sample},

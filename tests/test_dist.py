@@ -108,3 +108,18 @@ def test_profiled_traffic_tracks_sources(tmp_path, monkeypatch):
     assert bench.profiled_traffic("missing.md", ["k.cu"]) is None
     for name, (summary, sources) in bench.PROFILES.items():  # every listed summary exists
         assert os.path.exists(os.path.join(os.path.dirname(os.path.dirname(__file__)), "profiles", summary)), name
+
+
+def test_reference_arm_line(monkeypatch):
+    import bench
+
+    # the oracle arm prints the GPU arm's metric and config (one bounded step)
+    monkeypatch.delenv("WORLD_SIZE", raising=False)
+    d = bench.run_reference(bench.parse_args(["--impl", "reference", "--steps", "1", "--warmup", "3"]))
+    assert d["impl"] == "reference" and d["metric"] == bench.METRIC and d["unit"] == "TFLOP/s"
+    assert d["higher_is_better"] is True and d["value"] > 0
+    assert d["config"] == {"workload": "mistral_swa_prefill", "B": 2, "Hq": 32, "Hkv": 8, "N": 8192, "d": 128,
+                           "W": 4096, "S": 0, "parallelism": "dp1 (independent batches)",
+                           "l2": "flushed between steps"}
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
