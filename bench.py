@@ -46,6 +46,8 @@ PROFILES = {
     "gemma_swa_prefill": ("prefill_swa_gemma.md", PREFILL_SOURCES),
     "diff_causal": ("prefill_diff_causal.md", PREFILL_SOURCES),
     "local_strided_prefill": ("prefill_strided_local.md", PREFILL_SOURCES),
+    "longformer_global_prefill": ("prefill_global_longformer.md", PREFILL_SOURCES),
+    "longformer_dilated_prefill": ("prefill_dilated_longformer.md", PREFILL_SOURCES),
     "mistral_swa_backward": ("backward_swa_mistral.md", BWD_SOURCES),
     "local_strided_backward": ("backward_strided_local.md", BWD_SOURCES),
     "gemma_swa_decode": ("decode_gemma.md", DECODE_SOURCES),
